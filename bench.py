@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of the ZeRO partitioned mixed-precision Adam step on B200.
+
+One step = one pass of the hot path over one batch of synthetic gradients:
+the emulated reduce-scatter of Nd fp16 gradient vectors (rank-ordered fp32
+sum), unscale + global overflow check, Adam on the fp32 master/m/v of every
+partition, fp16 cast and all-gather write-back (stage 1/2) or shard write
+plus the forward and backward layer gathers (stage 3). Inputs are resident in
+HBM when the timed region starts; everything moved per step (tens of GB at
+the default workload) exceeds the 126 MB L2, so no flush is needed.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the plain CPU
+oracle on a bounded sample of the same workload instead.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--variant fused|two-pass] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ZeRO Adam step Gparams/s and HBM GB/s (% of peak) on 1 B200 vs CPU oracle"
+UNIT = "Gparams/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "zero_partitioned_mixed_02_b200", "csrc", "zero_kernels.cu")
+
+WORKLOADS = {
+    "flat-1m": 1, "stress-16m": 2, "gpt2-1.5b": 3, "7.5b-rank-view": 4, "llama-2.7b": 5,
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
+    p.add_argument("--variant", choices=["fused", "two-pass"], default="fused")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the oracle baseline sample")
+    return p.parse_args()
+
+
+def workload(name):
+    from zero_partitioned_mixed_02_b200.synth import workloads as W
+    return W.ALL[WORKLOADS[name]]()
+
+
+# ---------------------------------------------------------------- bytes
+def owned_range(wl):
+    if wl.rank_view >= 0:
+        p = -(-wl.psi // wl.nd)
+        b = min(wl.rank_view * p, wl.psi)
+        return b, min(b + p, wl.psi)
+    return 0, wl.psi
+
+
+def algorithmic_bytes(wl, variant):
+    """Minimum bytes one step of the method must move (the floor), and per
+    launch of the dominant kernel. n = elements this GPU updates."""
+    b0, e0 = owned_range(wl)
+    n = e0 - b0
+    grads = 2 * wl.nd * n                    # every rank's fp16 gradient of each element
+    state = 24 * n                           # fp32 master, m, v read and written
+    n_out = wl.nd if (wl.stage <= 2 and wl.rank_view < 0) else 1
+    params = 2 * n * n_out                   # fp16 write-back to every replica / the shard
+    floor = grads + state + params
+    if variant == "fused":
+        per_launch = {"step_kernel<fused>": floor}
+    else:
+        per_launch = {"step_kernel<reduce>": grads + 4 * n,
+                      "step_kernel<update>": 4 * n + state + params}
+    gathers = 8 * wl.psi if wl.stage == 3 else 0  # 2 psi read + 2 psi written, forward and back
+    return n, floor, per_launch, gathers
+
+
+# ---------------------------------------------------------------- environment
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sha():
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def recorded_traffic(wl_name, variant):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"ncu_step_{wl_name}_{variant}.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", txt)
+    if not m or not h or h.group(1) != kernel_sha():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 8]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_info():
+    model = ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+# ---------------------------------------------------------------- oracle leg
+def oracle_sample_step(wl, n_s, step, state):
+    """One oracle step over the first n_s owned elements of the workload (the
+    sample): the stage's own partitioned emulation with the same Nd. Returns
+    CPU seconds of the oracle call alone."""
+    import numpy as np
+
+    from oracle import zero_ref as Z
+    from zero_partitioned_mixed_02_b200 import synth as S
+
+    b0, _ = owned_range(wl)
+    gs = [S.host_f16_bits(n_s, b0, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad)
+          for k in range(wl.nd)]
+    hp = Z.hyper(**wl.hyper)
+    if state.get("w") is None:
+        w0 = S.host_f32(n_s, b0, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master)
+        if wl.stage <= 2 and wl.rank_view < 0:
+            parts = [Z.partition(n_s, wl.nd, r) for r in range(wl.nd)]
+            state["w"] = [w0[b:e].copy() for b, e in parts]
+            state["m"] = [np.zeros(e - b, np.float32) for b, e in parts]
+            state["v"] = [np.zeros(e - b, np.float32) for b, e in parts]
+            state["p"] = [Z.f16_from_f32(w0) for _ in range(wl.nd)]
+        elif wl.stage == 3:
+            numel, left = [], n_s
+            for n, _ in wl.tensors:
+                take = min(n, left)
+                if take <= 0:
+                    break
+                numel.append(take)
+                left -= take
+            state["numel"] = numel
+            offs = np.concatenate([[0], np.cumsum(numel)])
+            state["w"] = []
+            for r in range(wl.nd):
+                pieces = [w0[offs[t] + b: offs[t] + e]
+                          for t, n in enumerate(numel) for b, e in [Z.chunk(n, wl.nd, r)]]
+                state["w"].append(np.concatenate(pieces).astype(np.float32))
+            state["m"] = [np.zeros_like(x) for x in state["w"]]
+            state["v"] = [np.zeros_like(x) for x in state["w"]]
+            state["p"] = [Z.f16_from_f32(x) for x in state["w"]]
+        else:
+            state["w"], state["m"], state["v"] = w0, np.zeros(n_s, np.float32), np.zeros(n_s, np.float32)
+            state["p"] = np.zeros(n_s, np.uint16)
+        state["t"] = 0
+    t0 = time.perf_counter()
+    if wl.stage <= 2 and wl.rank_view < 0:
+        _, state["t"] = Z.zero12_step(n_s, gs, state["w"], state["m"], state["v"], state["p"],
+                                      wl.loss_scale, hp, state["t"])
+    elif wl.stage == 3:
+        _, state["t"] = Z.zero3_step(state["numel"], gs, state["w"], state["m"], state["v"],
+                                     state["p"], wl.loss_scale, hp, state["t"])
+    else:
+        _, state["t"] = Z.dp_step(gs, state["w"], state["m"], state["v"], state["p"],
+                                  wl.loss_scale, hp, state["t"])
+    return time.perf_counter() - t0
+
+
+def calibrate_sample(wl, seconds):
+    n0 = 1 << 17
+    dt = oracle_sample_step(wl, n0, 0, {})
+    rate = n0 / max(dt, 1e-6)
+    b0, e0 = owned_range(wl)
+    return int(max(4096, min(e0 - b0, rate * seconds)))
+
+
+def cpu_baseline(wl, seconds):
+    n_s = calibrate_sample(wl, seconds)
+    dt = oracle_sample_step(wl, n_s, 0, {})
+    model, ncpu = cpu_info()
+    return {"value": n_s / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {n_s} of the workload's {owned_range(wl)[1] - owned_range(wl)[0]} "
+                      f"elements, Nd={wl.nd}, stage {wl.stage}, one step, single thread",
+            "seconds": dt, "host_cpu": model, "host_cpus": ncpu}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workload(args.workload)
+    budget = 150.0  # seconds of CPU for warm-up + timed steps
+    per_step = budget / max(1, args.steps + args.warmup)
+    n_s = calibrate_sample(wl, per_step)
+    state = {}
+    for i in range(args.warmup):
+        oracle_sample_step(wl, n_s, i, state)
+    times = [oracle_sample_step(wl, n_s, args.warmup + i, state) for i in range(args.steps)]
+    total = sum(times)
+    value = n_s * args.steps / total / 1e9
+    model, ncpu = cpu_info()
+    sample = (f"first {n_s} elements of the workload per step, Nd={wl.nd}, stage {wl.stage}, "
+              f"single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_of(wl, args.variant),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cpu": model, "host_cpus": ncpu},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, variant):
+    n, floor, _, gathers = algorithmic_bytes(wl, variant)
+    return {"workload": wl.name, "psi": wl.psi, "nd": wl.nd, "stage": wl.stage,
+            "rank_view": wl.rank_view, "variant": variant, "elements_updated": n,
+            "loss_scale": wl.loss_scale, "weight_decay": wl.weight_decay,
+            "l2": f"inputs larger than L2: {(floor + gathers) / 1e9:.1f} GB moved per step, no flush",
+            "parallelism": "replicas (Nd virtual ranks emulated per GPU)"}
+
+
+# ---------------------------------------------------------------- GPU leg
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+    from zero_partitioned_mixed_02_b200 import synth as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    wl = workload(args.workload)
+    variant = A.ZERO_VARIANT_FUSED if args.variant == "fused" else A.ZERO_VARIANT_TWO_PASS
+    cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, variant=variant,
+                   tensors=wl.tensors)
+    L = A.zero_state_bytes(cfg)
+    b0, e0 = owned_range(wl)
+    n_own = e0 - b0
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    ws = torch.empty(L.workspace_bytes, dtype=torch.uint8, device="cuda")
+    m_init = torch.empty(n_own, dtype=torch.float32, device="cuda")
+    S.fill_f32(m_init.data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master, s)
+    bufs = []
+    if wl.stage <= 2:
+        bufs = [torch.empty(wl.psi, dtype=torch.int16, device="cuda")
+                for _ in range(wl.nd if wl.rank_view < 0 else 1)]
+    grads = [torch.empty(n_own, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    for k in range(wl.nd):
+        S.fill_f16(grads[k].data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, 0, k), wl.grad, s)
+    h = A.zero_init(cfg, ws.data_ptr(), L.workspace_bytes, m_init.data_ptr(),
+                    [b.data_ptr() for b in bufs] if bufs else None, s)
+    del m_init
+    gptrs = [g.data_ptr() for g in grads]
+    hp = A.zero_hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay)
+    gather_out = None
+    if wl.stage == 3:
+        gather_out = torch.empty(L.transient_bytes // 2, dtype=torch.int16, device="cuda")
+    order = (list(range(L.n_units)) + list(reversed(range(L.n_units)))) if wl.stage == 3 else []
+
+    kernel_events = []
+
+    def one_step(timed):
+        if timed:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        A.zero_step_launch(h, gptrs, wl.loss_scale, hp, s)
+        if timed:
+            b.record(stream)
+            kernel_events.append((a, b))
+        rc = A.zero_step_commit(h, s)
+        if rc != A.ZERO_OK:
+            raise RuntimeError("unexpected skip in the benchmark workload")
+        for u in order:
+            A.zero_gather_layer(h, u, gather_out.data_ptr(), s)
+
+    for _ in range(args.warmup):
+        one_step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        one_step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop() if clocks else None
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = [a.elapsed_time(b) for a, b in kernel_events]
+    if world > 1:
+        tt = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+        dist.barrier()
+
+    n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant)
+    launches_per_step = (1 if args.variant == "fused" else 2) + len(order)
+    step_s = total_ms / 1e3 / args.steps
+    value = world * n / step_s / 1e9
+    peak, peak_src = measured_peak()
+    # dominant kernel: the step kernel (both kernels of the two-pass variant timed together)
+    k_s = statistics.mean(kern_ms) / 1e3
+    dom_bytes = floor
+    achieved = dom_bytes / k_s / 1e9
+    traffic = recorded_traffic(args.workload, args.variant)
+    kname = "step_kernel<fused>" if args.variant == "fused" else "step_kernel<reduce>+<update>"
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_of(wl, args.variant),
+        "hbm_gbs": (floor + gathers) / step_s / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": kname,
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "kernel_ms": statistics.mean(kern_ms), "peak_source": peak_src},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+    }
+
+    # ---- end to end through the public API from pinned host buffers ----
+    if not args.no_e2e and args.e2e_steps > 0:
+        line["e2e"] = e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world)
+    A.zero_destroy(h)
+
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
+    import psutil
+    import torch
+    import torch.distributed as dist
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+
+    n_own = grads[0].numel()
+    if wl.stage <= 2:
+        result = bufs[0]  # the step's result: one rank's all-gathered fp16 parameters
+    else:
+        result = ws[L.off_shard16: L.off_shard16 + 2 * L.state_elems].view(torch.int16)
+    need = (len(grads) * n_own + result.numel()) * 2
+    avail = psutil.virtual_memory().available
+    if need > 0.7 * avail:
+        return {"value": None, "unit": UNIT,
+                "unavailable": f"needs {need / 1e9:.1f} GB pinned host memory, "
+                               f"{avail / 1e9:.1f} GB available"}
+    s = torch.cuda.current_stream()
+    host_g = [torch.empty(n_own, dtype=torch.int16, pin_memory=True) for _ in grads]
+    for hg, g in zip(host_g, grads):
+        hg.copy_(g)
+    host_out = torch.empty(result.numel(), dtype=torch.int16, pin_memory=True)
+
+    def step():
+        for g, hg in zip(grads, host_g):
+            g.copy_(hg, non_blocking=True)
+        rc = A.zero_step(h, gptrs, wl.loss_scale, hp, s.cuda_stream)
+        if rc != A.ZERO_OK:
+            raise RuntimeError("unexpected skip")
+        for u in order:
+            A.zero_gather_layer(h, u, gather_out.data_ptr(), s.cuda_stream)
+        host_out.copy_(result, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(s)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    n = L.state_elems
+    return {"value": world * n * args.e2e_steps / (ms / 1e3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": len(grads) * n_own * 2, "d2h_bytes_per_step": result.numel() * 2,
+            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+/*
+ * zero.h -- C ABI of libzero: the ZeRO stage 1/2/3 partitioned mixed-precision
+ * Adam step on one B200, with Nd data-parallel ranks emulated as virtual ranks.
+ *
+ * The operation (pages cited by title and section):
+ *   [P1] "Your 7.5B model's weights fit in 15 GB. Training state was 120 GB per
+ *        GPU" (blog.teqners.com) -- "Where 16 bytes per parameter comes from",
+ *        "Why you can't just delete the fp32 copies", "The replication nobody
+ *        questioned" (stage table), "The part that sounds too good:
+ *        communication".
+ *   [P2] "Engine Room" ch. 10, "ZeRO and the Memory Tricks" -- "The Mathematics"
+ *        (M_states(p, Nd)), "What It Enabled" (stage table).
+ *   [P3] "DeepSpeed ZeRO: account for every training state" -- "What each ZeRO
+ *        stage partitions", "Partitioned parameters still have to participate
+ *        in computation", "Check your understanding".
+ *
+ * One step, for every element i owned by rank r ([P1] "communication": each
+ * rank reduce-scatters the gradients, updates only its slice, and the ranks
+ * all-gather the updated fp16 parameters):
+ *   s   = fp32(g_0[i]) + fp32(g_1[i]) + ... + fp32(g_{Nd-1}[i])  (rank order, fp32)
+ *   g   = s * inv_scale,  inv_scale = (float)(1.0 / (double)loss_scale)
+ *   skip the whole step if any g over all partitions is inf or NaN
+ *   m   = b1*m + (1-b1)*g ;  v = b2*v + (1-b2)*(g*g)
+ *   u   = (m / bc1) / (sqrt(v / bc2) + eps),  bc_k = (float)(1 - beta_k^t)
+ *   w   = w - lr*(u + wd*w)                              (fp32 master)
+ *   p16 = fp16(w), round to nearest even, written to every rank's replica
+ *         (stage 1/2) or to rank r's fp16 shard (stage 3).
+ * Each binary32 operation is one IEEE-rounded operation in that order (no FMA
+ * contraction, no flush to zero). Stage 3 adds zero_gather_layer, the
+ * on-demand gather of one layer's full fp16 weights ([P1] "communication",
+ * stage 3; [P3] "Partitioned parameters still have to participate").
+ *
+ * Conventions for every call:
+ *   - fp16 values are IEEE binary16 bit patterns (uint16_t).
+ *   - "device" pointers are CUDA global-memory addresses on the current device;
+ *     every device pointer passed in must be 16-byte aligned (ZERO_ERR_ALIGN).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All device
+ *     work of a call is ordered on it.
+ *   - The caller owns and allocates all device memory (workspace, gradients,
+ *     parameter buffers, gather output). The library never allocates device
+ *     memory; a handle is a small host object freed by zero_destroy.
+ *   - Handles are not thread-safe; one handle serves one caller thread.
+ */
+#ifndef ZERO_H
+#define ZERO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ---- */
+#define ZERO_OK 0
+#define ZERO_SKIPPED 1          /* informational: overflow, step skipped, state untouched */
+#define ZERO_ERR_ARG (-1)       /* invalid argument or configuration */
+#define ZERO_ERR_ALIGN (-2)     /* a device pointer is not 16-byte aligned */
+#define ZERO_ERR_STAGE (-3)     /* call not valid for this stage (gather on stage 1/2) */
+#define ZERO_ERR_WORKSPACE (-4) /* workspace smaller than zero_state_bytes says */
+#define ZERO_ERR_CUDA (-5)      /* a CUDA call failed; see zero_last_cuda_error */
+#define ZERO_ERR_INTERNAL (-6)  /* internal consistency check failed */
+
+/* ---- step variants ---- */
+/* One pass: reads the gradients and the current master/m/v, writes the next
+ * master/m/v into a second state buffer and the fp16 parameters in place.
+ * Commits by switching buffers; on overflow the buffers stay and the fp16
+ * parameters are rewritten from the unchanged master (a pure function of it).
+ * Moves the minimum (24 + 4 Nd) bytes per element (stage 1/2). */
+#define ZERO_VARIANT_FUSED 0
+/* Two passes: the reduce pass writes the unscaled fp32 reduced gradient of
+ * every partition and the overflow flag; the update pass checks the flag and
+ * runs Adam in place. One state buffer; 8 more bytes per element. */
+#define ZERO_VARIANT_TWO_PASS 1
+
+#define ZERO_MAX_ND 1024
+
+/* One tensor of the flat parameter vector, in flat order. `unit` is the layer
+ * unit a stage-3 gather rebuilds (units are numbered 0, 1, ... and appear in
+ * non-decreasing order along the tensor list). */
+typedef struct zero_tensor {
+    int64_t numel;
+    int32_t unit;
+    int32_t reserved; /* must be 0 */
+} zero_tensor;
+
+typedef struct zero_config {
+    int64_t psi;       /* number of parameters of the flat vector */
+    int32_t nd;        /* virtual data-parallel ranks, 1 .. ZERO_MAX_ND */
+    int32_t stage;     /* ZeRO stage 1, 2 or 3 */
+    int32_t rank_view; /* -1: emulate all Nd ranks; r >= 0 (stage 1/2 only):
+                          act as rank r alone, owning partition r */
+    int32_t variant;   /* ZERO_VARIANT_FUSED or ZERO_VARIANT_TWO_PASS */
+    int32_t n_tensors; /* 0 allowed for stage 1/2 (one flat tensor) */
+    int32_t reserved;  /* must be 0 */
+    const zero_tensor* tensors; /* host array of n_tensors; sum of numel == psi;
+                                   required for stage 3 */
+} zero_config;
+
+typedef struct zero_hyper {
+    float lr;
+    float beta1;
+    float beta2;
+    float eps;
+    float weight_decay; /* decoupled, scaled by lr; 0 = plain Adam */
+} zero_hyper;
+
+/* Memory ledger and layout ([P1] "Where 16 bytes per parameter comes from":
+ * 2 + 2 + K bytes, K = 12; [P1] stage table and [P2] "The Mathematics"). */
+typedef struct zero_ledger {
+    /* per-rank model-state bytes from the pages' formulas:
+       [0] 16 psi, [1] 4 psi + 12 psi/Nd, [2] 2 psi + 14 psi/Nd, [3] 16 psi/Nd */
+    double formula_bytes[4];
+    /* the same for the rank holding the most under the ceil split, exact */
+    int64_t exact_bytes[4];
+    /* elements sent per step summed over ranks, ring collectives:
+       [0] reduce-scatter, [1] all-gather, [2] DP all-reduce, [3..5] stage 1..3
+       ([P1] "communication": 2 psi for DP and stages 1/2, 3 psi for stage 3,
+       reached as Nd grows) */
+    int64_t comm_elements[6];
+    int64_t allreduce_buffer_bytes; /* flat fp32 buffer of the model, 4 psi
+                                       ([P1] "What the 16 Psi formula doesn't cover") */
+    int64_t transient_bytes;   /* stage 3: largest layer unit gathered (fp16), else 0 */
+    int64_t peak_stage3_bytes; /* exact_bytes[3] + transient_bytes: the persistent
+                                  estimate is not the peak ([P3] "Check your
+                                  understanding") */
+    int64_t workspace_bytes;   /* bytes zero_init needs */
+    int64_t partition_len;     /* P = ceil(psi / Nd) */
+    int64_t state_elems;       /* elements of each state array (master, m, v) */
+    int64_t grad_len;          /* elements each grads[k] must hold */
+    int64_t off_master[2];     /* byte offsets in the workspace of state buffer 0 and */
+    int64_t off_m[2];          /*   1 (fused variant; -1 for two-pass)               */
+    int64_t off_v[2];
+    int64_t off_shard16;       /* stage 3: fp16 shard array (state order), else -1 */
+    int64_t off_reduced;       /* two-pass: fp32 reduced gradients (state order), else -1 */
+    int32_t n_units;           /* stage 3 layer units, else 0 */
+    int32_t n_out;             /* parameter buffers zero_init takes (stage 1/2) */
+} zero_ledger;
+
+typedef struct zero_handle zero_handle;
+
+/* Ledger, layout and workspace size for `cfg`. Host only: no device work, no
+ * allocation. Returns ZERO_OK or ZERO_ERR_ARG. */
+int zero_state_bytes(const zero_config* cfg, zero_ledger* out);
+
+/* Where rank `rank`'s shard sits in the state arrays: elements
+ * [*state_begin, *state_begin + *len) of master/m/v (and of the stage-3 fp16
+ * shard array). Stage 1/2 with all ranks: the flat partition [r*P, ...).
+ * Stage 3: rank r's chunk of every tensor, in tensor order, ranks back to back
+ * ([P3] "What each ZeRO stage partitions"). Single-rank view: the viewed
+ * rank's partition starts at 0, other ranks hold nothing here. Host only. */
+int zero_rank_shard(const zero_config* cfg, int32_t rank, int64_t* state_begin, int64_t* len);
+
+/* Flat range [*flat_begin, *flat_begin + *numel) of stage-3 layer unit
+ * `unit`; zero_gather_layer writes *numel fp16 values. Host only. */
+int zero_unit_range(const zero_config* cfg, int32_t unit, int64_t* flat_begin, int64_t* numel);
+
+/* Bind a workspace and initialise the optimizer state.
+ *   workspace     device, >= ledger.workspace_bytes, owned by the caller and
+ *                 used by the handle until zero_destroy.
+ *   master_init   device fp32: the initial master weights of the elements this
+ *                 handle owns, in flat order (psi values; the single-rank view
+ *                 takes the P_r values of partition r; NULL if that is empty).
+ *   param_bufs    host array of device fp16 buffers that receive the all-
+ *                 gathered parameters: stage 1/2 with all ranks: Nd replicas
+ *                 of psi values each; single-rank view: one full psi-value
+ *                 buffer of which partition r is written; stage 3: NULL (the
+ *                 fp16 parameters live in the workspace shards).
+ * Sets m = v = 0, master = master_init, t = 0, and writes fp16(master) to the
+ * parameter buffers (or shards). Synchronises `stream` before returning. */
+int zero_init(const zero_config* cfg, void* workspace, size_t workspace_bytes,
+              const float* master_init, uint16_t* const* param_bufs, void* stream,
+              zero_handle** out);
+
+/* One optimizer step.
+ *   grads       host array of Nd device fp16 gradient buffers, rank order.
+ *               All ranks: each holds psi values (the rank's full gradient).
+ *               Single-rank view: each holds rank k's P_r gradients of the
+ *               viewed partition r.
+ *   loss_scale  > 0 and finite; gradients are multiplied by 1/loss_scale.
+ *   skipped     optional out: 1 if the step was skipped for overflow.
+ * Returns ZERO_OK, or ZERO_SKIPPED when some unscaled reduced gradient is inf
+ * or NaN: then master/m/v, t and the fp16 parameters are as before the call.
+ * Reads one 4-byte flag back and synchronises `stream` once. */
+int zero_step(zero_handle* h, const uint16_t* const* grads, float loss_scale,
+              const zero_hyper* hp, void* stream, int* skipped);
+
+/* zero_step in two halves, for callers that overlap host work with the step
+ * or time its kernels on the stream. zero_step_launch validates and enqueues
+ * the step's kernels on `stream` and returns without waiting. zero_step_commit
+ * waits for `stream` to reach the end of the step, reads the overflow flag and
+ * commits (ZERO_OK) or rolls back (ZERO_SKIPPED) exactly as zero_step. Every
+ * launch must be followed by its commit before the next launch or gather on
+ * the handle (ZERO_ERR_ARG otherwise). */
+int zero_step_launch(zero_handle* h, const uint16_t* const* grads, float loss_scale,
+                     const zero_hyper* hp, void* stream);
+int zero_step_commit(zero_handle* h, void* stream, int* skipped);
+
+/* Stage 3: write layer unit `unit`'s full fp16 weights into `out` (device,
+ * >= the numel zero_unit_range reports): its tensors in tensor order, each whole
+ * and contiguous, back to back. Call it per unit in forward order and again in
+ * reverse for backward ([P1] "communication": parameters are gathered on demand
+ * in the forward and backward passes, then discarded). ZERO_ERR_STAGE on 1/2. */
+int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream);
+
+/* Current state: device pointers to the live master/m/v arrays (the fused
+ * variant alternates between two buffers) and the step count t. Any output
+ * pointer may be NULL. */
+int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t);
+
+/* Memory bandwidth reference: copy `bytes` (a multiple of 16, both pointers
+ * 16-byte aligned) from src to dst with 16-byte streaming loads and stores. */
+int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);
+
+/* The cudaError_t of the last failed CUDA call made through `h` (0 if none). */
+int zero_last_cuda_error(const zero_handle* h);
+
+/* Static text for a return code. */
+const char* zero_error_string(int code);
+
+/* Release the handle (host memory only; the caller frees the workspace). */
+void zero_destroy(zero_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

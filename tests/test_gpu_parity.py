@@ -1,0 +1,286 @@
+"""GPU vs oracle, element by element, through the C ABI.
+
+Sizes the oracle finishes in seconds: a grid of tiny and ragged cases (every
+stage and variant, Nd 1..9, Psi from 1 to a few thousand with ragged tails and
+empty partitions, stage-3 tensor lists with odd sizes), the single-rank view
+with out-of-phase partitions, overflow skips (inf, -inf, NaN, an unscale that
+overflows) injected where the injecting rank does not own the element, and
+the two small workloads in full (Psi = 1,048,576, Nd = 4, stage 2;
+Psi = 16,777,216, Nd = 8, stage 1, precision stress with a skip).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import zero_ref as Z
+from zero_partitioned_mixed_02_b200 import _abi as A
+from zero_partitioned_mixed_02_b200 import synth as S
+from zero_partitioned_mixed_02_b200.synth import workloads as W
+
+from gpu_common import (GuardedF16, GuardedWorkspace, SENTINEL16, compare_f16, compare_f32,
+                        dev_u16, hyper, state_offsets)
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, never run there
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+
+def _tensor_list(rng, psi, n_max=6):
+    k = int(rng.integers(1, min(n_max, psi) + 1))
+    cuts = np.sort(rng.choice(np.arange(1, psi), size=k - 1, replace=False)) if k > 1 else []
+    sizes = np.diff(np.concatenate([[0], cuts, [psi]])).astype(int)
+    units = np.sort(rng.integers(0, 3, size=k))
+    units = np.searchsorted(np.unique(units), units)
+    return [(int(n), int(u)) for n, u in zip(sizes, units)]
+
+
+class Case:
+    """One configuration driven step by step on the GPU and in the oracle."""
+
+    def __init__(self, psi, nd, stage, variant, *, tensors=None, view=-1, loss_scale=1024.0,
+                 hp=None, grad_dist=None, master_dist=None, seed=0):
+        self.psi, self.nd, self.stage, self.variant, self.view = psi, nd, stage, variant, view
+        self.tensors = tensors
+        self.numel = [n for n, _ in tensors] if tensors else [psi]
+        self.units = [u for _, u in tensors] if tensors else [0]
+        self.loss_scale = loss_scale
+        self.hp = hp or {}
+        self.grad_dist = grad_dist or S.normal(1e-3, loss_scale)
+        self.master_dist = master_dist or S.uniform(-0.1, 0.1)
+        self.seed = seed
+        self.cfg = A.Config(psi, nd, stage, rank_view=view, variant=variant, tensors=tensors)
+        self.L = A.zero_state_bytes(self.cfg)
+        if view >= 0:
+            self.b0, self.e0 = Z.partition(psi, nd, view)
+        else:
+            self.b0, self.e0 = 0, psi
+        n_own = self.e0 - self.b0
+        self.master0 = S.host_f32(n_own, self.b0, S.key(seed, S.STREAM_MASTER, 0, 0),
+                                  self.master_dist)
+        # ---- GPU ----
+        self.ws = GuardedWorkspace(self.L.workspace_bytes)
+        self.m_init = torch.from_numpy(self.master0.copy()).cuda()
+        self.bufs = []
+        ptrs = None
+        if stage <= 2:
+            self.bufs = [GuardedF16(psi) for _ in range(nd if view < 0 else 1)]
+            ptrs = [b.ptr() for b in self.bufs]
+        self.stream = torch.cuda.current_stream().cuda_stream
+        self.h = A.zero_init(self.cfg, self.ws.ptr(), self.L.workspace_bytes,
+                             self.m_init.data_ptr(), ptrs, self.stream)
+        self.g_dev = [torch.empty(max(n_own, 1), dtype=torch.int16, device="cuda")
+                      for _ in range(nd)]
+        # ---- oracle ----
+        self.t = 0
+        if stage <= 2 and view < 0:
+            parts = [Z.partition(psi, nd, r) for r in range(nd)]
+            self.w_sh = [self.master0[b:e].copy() for b, e in parts]
+            self.m_sh = [np.zeros(e - b, np.float32) for b, e in parts]
+            self.v_sh = [np.zeros(e - b, np.float32) for b, e in parts]
+            self.reps = [Z.f16_from_f32(self.master0) for _ in range(nd)]
+        elif view >= 0:
+            self.w = self.master0.copy()
+            self.m = np.zeros(n_own, np.float32)
+            self.v = np.zeros(n_own, np.float32)
+            self.p16 = Z.f16_from_f32(self.w)
+        else:
+            offs = np.concatenate([[0], np.cumsum(self.numel)])
+            self.w_sh = []
+            for r in range(nd):
+                pieces = [self.master0[offs[t] + b: offs[t] + e]
+                          for t, n in enumerate(self.numel) for b, e in [Z.chunk(n, nd, r)]]
+                self.w_sh.append(np.concatenate(pieces).astype(np.float32))
+            self.m_sh = [np.zeros_like(x) for x in self.w_sh]
+            self.v_sh = [np.zeros_like(x) for x in self.w_sh]
+            self.p_sh = [Z.f16_from_f32(x) for x in self.w_sh]
+
+    def grads(self, step):
+        n = self.e0 - self.b0
+        return [S.host_f16_bits(n, self.b0, S.key(self.seed, S.STREAM_GRAD, step, k),
+                                self.grad_dist) for k in range(self.nd)]
+
+    def step(self, gs):
+        n = self.e0 - self.b0
+        for k in range(self.nd):
+            if n:
+                self.g_dev[k][:n].copy_(torch.from_numpy(gs[k].view(np.int16)))
+        rc = A.zero_step(self.h, [g.data_ptr() for g in self.g_dev], self.loss_scale,
+                         hyper(**self.hp), self.stream)
+        hp = Z.hyper(**self.hp)
+        if self.stage <= 2 and self.view < 0:
+            sk, self.t = Z.zero12_step(self.psi, gs, self.w_sh, self.m_sh, self.v_sh, self.reps,
+                                       self.loss_scale, hp, self.t)
+        elif self.view >= 0:
+            sk, self.t = Z.dp_step(gs, self.w, self.m, self.v, self.p16, self.loss_scale, hp, self.t)
+        else:
+            sk, self.t = Z.zero3_step(self.numel, gs, self.w_sh, self.m_sh, self.v_sh, self.p_sh,
+                                      self.loss_scale, hp, self.t)
+        assert (rc == A.ZERO_SKIPPED) == sk, (rc, sk)
+        return sk
+
+    def check(self, tag=""):
+        wo, mo, vo, t = state_offsets(self.h, self.ws)
+        assert t == self.t
+        n = self.L.state_elems
+        if self.view >= 0:
+            ww, wm, wv = self.w, self.m, self.v
+        else:
+            ww, wm, wv = (np.concatenate(x) for x in (self.w_sh, self.m_sh, self.v_sh))
+        compare_f32(self.ws.f32(wo, n), ww, f"master {tag}")
+        compare_f32(self.ws.f32(mo, n), wm, f"m {tag}")
+        compare_f32(self.ws.f32(vo, n), wv, f"v {tag}")
+        if self.stage <= 2 and self.view < 0:
+            for k, b in enumerate(self.bufs):
+                compare_f16(b.bits(), self.reps[k], f"replica {k} {tag}")
+        elif self.view >= 0:
+            got = self.bufs[0].bits()
+            compare_f16(got[self.b0:self.e0], self.p16, f"partition params {tag}")
+            assert (got[:self.b0] == SENTINEL16).all() and (got[self.e0:] == SENTINEL16).all()
+        else:
+            compare_f16(self.ws.u16(self.L.off_shard16, n), np.concatenate(self.p_sh),
+                        f"fp16 shards {tag}")
+            for u in range(self.L.n_units):
+                fb, cnt = A.zero_unit_range(self.cfg, u)
+                out = GuardedF16(cnt)
+                A.zero_gather_layer(self.h, u, out.ptr(), self.stream)
+                want = Z.zero3_gather(self.numel, self.units, self.nd, u, self.p_sh)
+                compare_f16(out.bits(), want, f"gather unit {u} {tag}")
+                assert out.guards_intact()
+        for b in self.bufs:
+            assert b.guards_intact(), f"param buffer guard band written {tag}"
+        assert self.ws.guards_intact(), f"workspace guard band written {tag}"
+
+    def close(self):
+        A.zero_destroy(self.h)
+
+
+def _run(case: Case, steps: int, inject=()):
+    case.check("after init")
+    skips = []
+    for s in range(steps):
+        gs = case.grads(s)
+        for (st, k, i, bits) in inject:
+            if st == s and case.b0 <= i < case.e0:
+                gs[k][i - case.b0] = bits
+        skips.append(case.step(gs))
+        case.check(f"after step {s}")
+    case.close()
+    return skips
+
+
+PSIS = [1, 2, 3, 7, 8, 9, 15, 16, 17, 31, 33, 40, 255, 256, 257, 1000, 4099, 8197, 70001]
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("stage", [1, 2])
+@pytest.mark.parametrize("nd", [1, 2, 3, 4, 5, 8, 9])
+def test_stage12_grid(nd, stage, variant):
+    for psi in PSIS:
+        _run(Case(psi, nd, stage, variant, hp=dict(lr=1e-2, weight_decay=0.01 * (psi % 2))), 2)
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("nd", [1, 2, 3, 4, 5, 8, 9])
+def test_stage3_grid(nd, variant):
+    rng = np.random.default_rng(nd * 10 + variant)
+    for psi in PSIS:
+        _run(Case(psi, nd, 3, variant, tensors=_tensor_list(rng, psi)), 2)
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+def test_single_rank_view_out_of_phase(variant):
+    # partitions whose start is 2, 4 or 6 bytes off a 16-byte boundary in the
+    # full parameter buffer, and a trailing rank that is short or empty
+    for psi, nd in [(1003, 8), (8 * 1000 + 4, 8), (117, 3), (64 * 37 + 5, 64), (10, 16)]:
+        for r in range(nd):
+            _run(Case(psi, nd, 1 + r % 2, variant, view=r), 2)
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("bits", [0x7C00, 0xFC00, 0x7E00])
+def test_skip_is_global(variant, bits):
+    # inf/-inf/NaN on the last rank at an element owned by rank 0, at step 1
+    for stage in (1, 2, 3):
+        rng = np.random.default_rng(bits + stage)
+        psi, nd = 1001, 4
+        tensors = _tensor_list(rng, psi) if stage == 3 else None
+        skips = _run(Case(psi, nd, stage, variant, tensors=tensors), 3,
+                     inject=[(1, nd - 1, 0, bits)])
+        assert skips == [False, True, False]
+        skips = _run(Case(psi, nd, stage, variant, tensors=tensors), 3,
+                     inject=[(0, 0, psi - 1, bits), (2, 1, 500, bits)])
+        assert skips == [True, False, True]
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+def test_skip_when_unscale_overflows(variant):
+    # finite fp16 gradients, but 1/loss_scale pushes their sum past FLT_MAX
+    c = Case(300, 2, 2, variant, loss_scale=1e-36, grad_dist=S.normal(1.0, 10000.0))
+    skips = _run(c, 2)
+    assert skips == [True, True]
+
+
+def test_rank_order_of_the_sum():
+    # 0.001 vanishes against 65504 in fp32; the rank order decides the result
+    c = Case(16, 3, 2, A.ZERO_VARIANT_FUSED, loss_scale=1.0, hp=dict(beta1=0.0, beta2=0.0))
+    c.check("init")
+    g = [np.full(16, b, np.uint16) for b in
+         np.array([65504.0, 0.001, -65504.0], np.float16).view(np.uint16)]
+    c.step(g)
+    c.check("step")
+    _, mo, _, _ = state_offsets(c.h, c.ws)
+    assert (c.ws.f32(mo, 16) == 0.0).all()
+    c.close()
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+def test_zero_gradients_and_non_power_of_two_scale(variant):
+    c = Case(4099, 5, 2, variant, loss_scale=3000.0, grad_dist=S.normal(0.0, 1.0))
+    _run(c, 2)
+    c = Case(4099, 5, 2, variant, loss_scale=3000.0, hp=dict(weight_decay=0.1, lr=0.05))
+    _run(c, 3)
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+def test_workload_flat_1m(variant):
+    wl = W.flat_1m()
+    c = Case(wl.psi, wl.nd, wl.stage, variant, loss_scale=wl.loss_scale, hp=wl.hyper,
+             grad_dist=wl.grad, master_dist=wl.master, seed=wl.seed)
+    assert _run(c, wl.steps) == [False] * wl.steps
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+def test_workload_precision_stress(variant):
+    wl = W.stress_16m()
+    c = Case(wl.psi, wl.nd, wl.stage, variant, loss_scale=wl.loss_scale, hp=wl.hyper,
+             grad_dist=wl.grad, master_dist=wl.master, seed=wl.seed)
+    w_before = c.master0.copy()
+    p_before = Z.f16_from_f32(w_before)
+    c.check("after init")
+    skips = []
+    w_hist = [w_before]
+    for s in range(wl.steps):
+        gs = c.grads(s)
+        for (st, k, i, bits) in wl.inject:
+            if st == s:
+                gs[k][i] = bits
+        skips.append(c.step(gs))
+        c.check(f"after step {s}")
+        wo, _, _, _ = state_offsets(c.h, c.ws)
+        w_hist.append(c.ws.f32(wo, wl.psi))
+    assert skips == [False, True, False]  # the inf on rank 3 at step 2 skips it everywhere
+    assert (w_hist[2].view(np.uint32) == w_hist[1].view(np.uint32)).all()
+    # fp32 master absorbs every update; a direct fp16 update would lose most
+    dw = (w_hist[1].astype(np.float64) - w_before).astype(np.float32)
+    moved = w_hist[1] != w_before
+    assert moved.mean() > 0.999
+    lost = Z.direct_f16_update(p_before, dw) == p_before
+    assert lost.mean() > 0.8  # |w| >= 2.048 is ~88% of U(1, 10)
+    # after the steps some fp16 params have moved although no single direct
+    # fp16 update of those elements would have moved them
+    p_after = c.bufs[0].bits()
+    assert ((p_after != p_before) & lost).sum() > 0
+    c.close()

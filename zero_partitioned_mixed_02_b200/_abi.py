@@ -1,0 +1,206 @@
+"""ctypes binding of libzero's C ABI (include/zero.h), same names, argument
+marshalling only: every step of the optimizer runs in libzero's kernels.
+
+Device pointers are passed as Python ints (``tensor.data_ptr()``), streams as
+``torch.cuda.Stream.cuda_stream`` ints. Errors raise ``ZeroError``; the
+informational ZERO_SKIPPED is returned, not raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Sequence
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libzero.so")
+
+ZERO_OK = 0
+ZERO_SKIPPED = 1
+ZERO_ERR_ARG = -1
+ZERO_ERR_ALIGN = -2
+ZERO_ERR_STAGE = -3
+ZERO_ERR_WORKSPACE = -4
+ZERO_ERR_CUDA = -5
+ZERO_ERR_INTERNAL = -6
+
+ZERO_VARIANT_FUSED = 0
+ZERO_VARIANT_TWO_PASS = 1
+ZERO_MAX_ND = 1024
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, code: int, where: str, cuda: int = 0):
+        msg = f"{where}: {error_string(code)} ({code})"
+        if cuda:
+            msg += f", cudaError {cuda}"
+        super().__init__(msg)
+        self.code = code
+
+
+class zero_tensor(C.Structure):
+    _fields_ = [("numel", C.c_int64), ("unit", C.c_int32), ("reserved", C.c_int32)]
+
+
+class zero_config(C.Structure):
+    _fields_ = [("psi", C.c_int64), ("nd", C.c_int32), ("stage", C.c_int32),
+                ("rank_view", C.c_int32), ("variant", C.c_int32), ("n_tensors", C.c_int32),
+                ("reserved", C.c_int32), ("tensors", C.POINTER(zero_tensor))]
+
+
+class zero_hyper(C.Structure):
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
+                ("eps", C.c_float), ("weight_decay", C.c_float)]
+
+
+class zero_ledger(C.Structure):
+    _fields_ = [("formula_bytes", C.c_double * 4), ("exact_bytes", C.c_int64 * 4),
+                ("comm_elements", C.c_int64 * 6), ("allreduce_buffer_bytes", C.c_int64),
+                ("transient_bytes", C.c_int64), ("peak_stage3_bytes", C.c_int64),
+                ("workspace_bytes", C.c_int64), ("partition_len", C.c_int64),
+                ("state_elems", C.c_int64), ("grad_len", C.c_int64),
+                ("off_master", C.c_int64 * 2), ("off_m", C.c_int64 * 2), ("off_v", C.c_int64 * 2),
+                ("off_shard16", C.c_int64), ("off_reduced", C.c_int64),
+                ("n_units", C.c_int32), ("n_out", C.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libzero.so. Raises if the extension is not built: there is no
+    fallback path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libzero.so not built at {LIB_PATH}; "
+                               "run python -m zero_partitioned_mixed_02_b200.build")
+        L = C.CDLL(LIB_PATH)
+        P = C.c_void_p
+        sig = {
+            "zero_state_bytes": (C.c_int, [C.POINTER(zero_config), C.POINTER(zero_ledger)]),
+            "zero_rank_shard": (C.c_int, [C.POINTER(zero_config), C.c_int32,
+                                          C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
+            "zero_unit_range": (C.c_int, [C.POINTER(zero_config), C.c_int32,
+                                          C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
+            "zero_init": (C.c_int, [C.POINTER(zero_config), P, C.c_size_t, P, C.POINTER(P), P,
+                                    C.POINTER(P)]),
+            "zero_step": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P,
+                                    C.POINTER(C.c_int)]),
+            "zero_step_launch": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P]),
+            "zero_step_commit": (C.c_int, [P, P, C.POINTER(C.c_int)]),
+            "zero_gather_layer": (C.c_int, [P, C.c_int32, P, P]),
+            "zero_current_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
+                                             C.POINTER(C.c_int64)]),
+            "zero_stream_copy": (C.c_int, [P, P, C.c_size_t, P]),
+            "zero_last_cuda_error": (C.c_int, [P]),
+            "zero_error_string": (C.c_char_p, [C.c_int]),
+            "zero_destroy": (None, [P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return lib().zero_error_string(code).decode()
+
+
+class Config:
+    """zero_config plus the tensor array it points to (kept alive together)."""
+
+    def __init__(self, psi: int, nd: int, stage: int, rank_view: int = -1,
+                 variant: int = ZERO_VARIANT_FUSED,
+                 tensors: Sequence[tuple[int, int]] | None = None):
+        self._tensors = None
+        n = 0
+        ptr = None
+        if tensors:
+            n = len(tensors)
+            self._tensors = (zero_tensor * n)(*[zero_tensor(int(a), int(u), 0) for a, u in tensors])
+            ptr = C.cast(self._tensors, C.POINTER(zero_tensor))
+        self.c = zero_config(int(psi), int(nd), int(stage), int(rank_view), int(variant), n, 0, ptr)
+
+    def byref(self):
+        return C.byref(self.c)
+
+
+def _check(rc: int, where: str, h=None) -> int:
+    if rc < 0:
+        cuda = lib().zero_last_cuda_error(h) if h else 0
+        raise ZeroError(rc, where, cuda)
+    return rc
+
+
+def zero_state_bytes(cfg: Config) -> zero_ledger:
+    out = zero_ledger()
+    _check(lib().zero_state_bytes(cfg.byref(), C.byref(out)), "zero_state_bytes")
+    return out
+
+
+def zero_rank_shard(cfg: Config, rank: int) -> tuple[int, int]:
+    b, n = C.c_int64(), C.c_int64()
+    _check(lib().zero_rank_shard(cfg.byref(), rank, C.byref(b), C.byref(n)), "zero_rank_shard")
+    return b.value, n.value
+
+
+def zero_unit_range(cfg: Config, unit: int) -> tuple[int, int]:
+    b, n = C.c_int64(), C.c_int64()
+    _check(lib().zero_unit_range(cfg.byref(), unit, C.byref(b), C.byref(n)), "zero_unit_range")
+    return b.value, n.value
+
+
+def _ptr_array(ptrs: Sequence[int] | None):
+    if ptrs is None:
+        return None
+    return (C.c_void_p * max(len(ptrs), 1))(*[int(p) for p in ptrs])
+
+
+def zero_init(cfg: Config, workspace: int, workspace_bytes: int, master_init: int,
+              param_bufs: Sequence[int] | None, stream: int) -> int:
+    h = C.c_void_p()
+    arr = _ptr_array(param_bufs)
+    _check(lib().zero_init(cfg.byref(), workspace, workspace_bytes, master_init, arr, stream,
+                           C.byref(h)), "zero_init")
+    return h.value
+
+
+def zero_step(h: int, grads: Sequence[int], loss_scale: float, hp: zero_hyper, stream: int) -> int:
+    arr = _ptr_array(grads)
+    sk = C.c_int(0)
+    return _check(lib().zero_step(h, arr, float(loss_scale), C.byref(hp), stream, C.byref(sk)),
+                  "zero_step", h)
+
+
+def zero_step_launch(h: int, grads: Sequence[int], loss_scale: float, hp: zero_hyper,
+                     stream: int) -> None:
+    arr = _ptr_array(grads)
+    _check(lib().zero_step_launch(h, arr, float(loss_scale), C.byref(hp), stream),
+           "zero_step_launch", h)
+
+
+def zero_step_commit(h: int, stream: int) -> int:
+    sk = C.c_int(0)
+    return _check(lib().zero_step_commit(h, stream, C.byref(sk)), "zero_step_commit", h)
+
+
+def zero_gather_layer(h: int, unit: int, out: int, stream: int) -> None:
+    _check(lib().zero_gather_layer(h, unit, out, stream), "zero_gather_layer", h)
+
+
+def zero_current_state(h: int) -> tuple[int, int, int, int]:
+    w, m, v = C.c_void_p(), C.c_void_p(), C.c_void_p()
+    t = C.c_int64()
+    _check(lib().zero_current_state(h, C.byref(w), C.byref(m), C.byref(v), C.byref(t)),
+           "zero_current_state")
+    return w.value, m.value, v.value, t.value
+
+
+def zero_stream_copy(dst: int, src: int, nbytes: int, stream: int) -> None:
+    _check(lib().zero_stream_copy(dst, src, nbytes, stream), "zero_stream_copy")
+
+
+def zero_destroy(h: int) -> None:
+    lib().zero_destroy(h)

@@ -1,0 +1,69 @@
+"""Build the package's native libraries in-tree for sm_100a.
+
+  libzero.so          the ZeRO step library (csrc/*.cu, C ABI in include/zero.h)
+  synth/libzsynth.so  the seeded synthetic-input generator (host + device)
+
+Flags: arithmetic is IEEE binary32 as written -- no FMA contraction
+(-fmad=false), correctly rounded division and square root, no flush to zero.
+``python -m zero_partitioned_mixed_02_b200.build [--force]``.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+SYNTH = os.path.join(PKG, "synth")
+
+LIBZERO = os.path.join(PKG, "libzero.so")
+LIBSYNTH = os.path.join(SYNTH, "libzsynth.so")
+PTXAS_LOG = os.path.join(PKG, "libzero.ptxas.txt")
+
+NVCC = os.environ.get("NVCC", "nvcc")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+COMMON = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-fmad=false", "-ftz=false",
+          "-prec-div=true", "-prec-sqrt=true", "-Xcompiler", "-fPIC,-ffp-contract=off"]
+
+ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu")]
+ZERO_DEPS = ZERO_SOURCES + [os.path.join(CSRC, "zero_internal.h"), os.path.join(INCLUDE, "zero.h")]
+SYNTH_SOURCES = [os.path.join(SYNTH, "zsynth.cu")]
+SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(SYNTH, "zsynth.h")]
+
+
+def _stale(target: str, deps: list[str]) -> bool:
+    if not os.path.exists(target):
+        return True
+    t = os.path.getmtime(target)
+    return any(os.path.getmtime(d) > t for d in deps + [__file__])
+
+
+def _nvcc(out: str, sources: list[str], extra: list[str], log: str | None = None) -> None:
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [NVCC, *COMMON, *extra, "-o", tmp, *sources]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError(f"nvcc failed building {os.path.basename(out)}")
+    if log is not None:
+        with open(log, "w") as f:
+            f.write(res.stdout + res.stderr)
+    os.replace(tmp, out)
+
+
+def build(force: bool = False) -> None:
+    if force or _stale(LIBZERO, ZERO_DEPS):
+        _nvcc(LIBZERO, ZERO_SOURCES,
+              ["-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v"],
+              log=PTXAS_LOG)
+    if force or _stale(LIBSYNTH, SYNTH_DEPS):
+        _nvcc(LIBSYNTH, SYNTH_SOURCES, ["-I", SYNTH])
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv)
+    print(LIBZERO)
+    print(LIBSYNTH)

@@ -1,0 +1,657 @@
+// Host side of libzero: validation, the partitioner and descriptor tables, the
+// memory ledger, and the C ABI declared in include/zero.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "zero.h"
+#include "zero_internal.h"
+
+#define ZERO_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr int64_t kAlign = 256;
+constexpr int64_t kMaxPsi = int64_t(1) << 42;
+
+int64_t align_up(int64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Ceil split ([P1] "The replication nobody questioned": the state is divided
+// across the Nd ranks; trailing ranks may be short or empty).
+void split(int64_t n, int nd, int r, int64_t* b, int64_t* e)
+{
+    const int64_t p = (n + nd - 1) / nd;
+    *b = std::min<int64_t>((int64_t)r * p, n);
+    *e = std::min<int64_t>(*b + p, n);
+}
+
+struct Unit {
+    int64_t seg0 = 0;     // first gather run of the unit
+    int64_t n_segs = 0;
+    int64_t n_chunks = 0;
+    int64_t flat_begin = 0;
+    int64_t numel = 0;
+};
+
+// Everything that follows from a configuration: partitions, run tables,
+// ledger and workspace layout.
+struct Layout {
+    int64_t psi = 0;
+    int nd = 0, stage = 0, view = -1, variant = 0;
+    std::vector<int64_t> numel;  // tensor sizes (one flat tensor if none given)
+    std::vector<int32_t> unit_of;
+    int64_t P = 0, state_elems = 0, grad_len = 0;
+    int n_out = 0, n_units = 0;
+    std::vector<int64_t> shard_begin, shard_len;  // per rank, in state elements
+    std::vector<zk::SegDesc> step_segs;
+    int64_t step_chunks = 0;
+    std::vector<zk::SegDesc> gather_segs;
+    std::vector<Unit> units;
+    int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
+            off_gather_segs = 0, off_reduced = -1, off_shard16 = -1, total = 0;
+    int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
+    int64_t transient_elems = 0;
+};
+
+// Cut a run at the first 8-aligned gradient index and give it its chunks.
+void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, int64_t state_begin,
+             int64_t out_begin, int64_t len)
+{
+    if (len <= 0) return;
+    zk::SegDesc d{};
+    d.grad_begin = grad_begin;
+    d.state_begin = state_begin;
+    d.out_begin = out_begin;
+    d.len = len;
+    int64_t head = (zk::kGroup - (grad_begin % zk::kGroup)) % zk::kGroup;
+    if (head > len) head = len;
+    const int64_t groups = (len - head) / zk::kGroup;
+    d.head = (int)head;
+    d.tail = (int)(len - head - groups * zk::kGroup);
+    d.chunk_begin = *chunks;
+    const int64_t vec = (groups + zk::kChunkGroups - 1) / zk::kChunkGroups;
+    *chunks += vec + ((d.head + d.tail) > 0 ? 1 : 0);
+    v.push_back(d);
+}
+
+int build_layout(const zero_config* cfg, Layout* L)
+{
+    if (!cfg) return ZERO_ERR_ARG;
+    if (cfg->psi < 1 || cfg->psi > kMaxPsi) return ZERO_ERR_ARG;
+    if (cfg->nd < 1 || cfg->nd > ZERO_MAX_ND) return ZERO_ERR_ARG;
+    if (cfg->stage < 1 || cfg->stage > 3) return ZERO_ERR_ARG;
+    if (cfg->variant != ZERO_VARIANT_FUSED && cfg->variant != ZERO_VARIANT_TWO_PASS) return ZERO_ERR_ARG;
+    if (cfg->reserved != 0 || cfg->n_tensors < 0) return ZERO_ERR_ARG;
+    if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
+    if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
+    if (cfg->stage == 3 && cfg->n_tensors == 0) return ZERO_ERR_ARG;
+    if (cfg->n_tensors > 0 && !cfg->tensors) return ZERO_ERR_ARG;
+
+    L->psi = cfg->psi;
+    L->nd = cfg->nd;
+    L->stage = cfg->stage;
+    L->view = cfg->rank_view;
+    L->variant = cfg->variant;
+    const int nd = cfg->nd;
+    if (cfg->n_tensors > 0) {
+        int64_t sum = 0;
+        int32_t prev_unit = 0;
+        for (int i = 0; i < cfg->n_tensors; ++i) {
+            const zero_tensor& t = cfg->tensors[i];
+            if (t.numel < 1 || t.reserved != 0 || t.unit < 0) return ZERO_ERR_ARG;
+            if (i == 0 ? t.unit != 0 : (t.unit != prev_unit && t.unit != prev_unit + 1)) return ZERO_ERR_ARG;
+            prev_unit = t.unit;
+            sum += t.numel;
+            if (sum > kMaxPsi) return ZERO_ERR_ARG;
+            L->numel.push_back(t.numel);
+            L->unit_of.push_back(t.unit);
+        }
+        if (sum != cfg->psi) return ZERO_ERR_ARG;
+        L->n_units = prev_unit + 1;
+    } else {
+        L->numel.push_back(cfg->psi);
+        L->unit_of.push_back(0);
+        L->n_units = 1;
+    }
+    L->P = (cfg->psi + nd - 1) / nd;
+
+    // ---- partitions and the step's run table ----
+    L->shard_begin.assign(nd, 0);
+    L->shard_len.assign(nd, 0);
+    if (cfg->stage <= 2) {
+        if (cfg->rank_view < 0) {
+            for (int r = 0; r < nd; ++r) {
+                int64_t b, e;
+                split(cfg->psi, nd, r, &b, &e);
+                L->shard_begin[r] = b;
+                L->shard_len[r] = e - b;
+                add_run(L->step_segs, &L->step_chunks, b, b, b, e - b);
+            }
+            L->state_elems = cfg->psi;
+            L->grad_len = cfg->psi;
+            L->n_out = nd;
+        } else {
+            int64_t b, e;
+            split(cfg->psi, nd, cfg->rank_view, &b, &e);
+            L->shard_len[cfg->rank_view] = e - b;
+            add_run(L->step_segs, &L->step_chunks, 0, 0, b, e - b);
+            L->state_elems = e - b;
+            L->grad_len = e - b;
+            L->n_out = 1;
+        }
+    } else {
+        // stage 3: every tensor split per rank; rank r's shard is its chunks
+        // in tensor order, shards back to back in rank order
+        int64_t pos = 0;
+        for (int r = 0; r < nd; ++r) {
+            L->shard_begin[r] = pos;
+            int64_t off = 0, q = 0;
+            for (size_t t = 0; t < L->numel.size(); ++t) {
+                int64_t b, e;
+                split(L->numel[t], nd, r, &b, &e);
+                add_run(L->step_segs, &L->step_chunks, off + b, pos + q, pos + q, e - b);
+                q += e - b;
+                off += L->numel[t];
+            }
+            L->shard_len[r] = q;
+            pos += q;
+        }
+        L->state_elems = cfg->psi;
+        L->grad_len = cfg->psi;
+        L->n_out = 1;  // the fp16 shard array
+
+        // gather runs, unit by unit: tensor order, rank order within a tensor
+        L->units.assign(L->n_units, Unit{});
+        std::vector<int64_t> tensor_off(L->numel.size() + 1, 0);
+        for (size_t t = 0; t < L->numel.size(); ++t) tensor_off[t + 1] = tensor_off[t] + L->numel[t];
+        // position of rank r's chunk of tensor t inside the state arrays
+        std::vector<int64_t> chunk_pos(L->numel.size() * (size_t)nd);
+        for (int r = 0; r < nd; ++r) {
+            int64_t q = L->shard_begin[r];
+            for (size_t t = 0; t < L->numel.size(); ++t) {
+                int64_t b, e;
+                split(L->numel[t], nd, r, &b, &e);
+                chunk_pos[t * nd + r] = q;
+                q += e - b;
+            }
+        }
+        size_t t = 0;
+        for (int u = 0; u < L->n_units; ++u) {
+            Unit& U = L->units[u];
+            U.seg0 = (int64_t)L->gather_segs.size();
+            U.flat_begin = tensor_off[t];
+            int64_t chunks = 0;
+            while (t < L->numel.size() && L->unit_of[t] == u) {
+                for (int r = 0; r < nd; ++r) {
+                    int64_t b, e;
+                    split(L->numel[t], nd, r, &b, &e);
+                    add_run(L->gather_segs, &chunks, chunk_pos[t * nd + r],
+                            0, tensor_off[t] - U.flat_begin + b, e - b);
+                }
+                U.numel += L->numel[t];
+                ++t;
+            }
+            U.n_segs = (int64_t)L->gather_segs.size() - U.seg0;
+            U.n_chunks = chunks;
+            L->transient_elems = std::max(L->transient_elems, U.numel);
+        }
+    }
+
+    // ---- workspace layout ----
+    int64_t off = 0;
+    L->off_flag = off;
+    off += kAlign;
+    L->off_grad_tab = off;
+    off += align_up((int64_t)nd * 8);
+    L->off_out_tab = off;
+    off += align_up((int64_t)std::max(L->n_out, 1) * 8);
+    L->off_step_segs = off;
+    off += align_up((int64_t)std::max<size_t>(L->step_segs.size(), 1) * sizeof(zk::SegDesc));
+    L->off_gather_segs = off;
+    off += align_up((int64_t)L->gather_segs.size() * sizeof(zk::SegDesc));
+    const int n_buf = cfg->variant == ZERO_VARIANT_FUSED ? 2 : 1;
+    for (int b = 0; b < n_buf; ++b)
+        for (int k = 0; k < 3; ++k) {
+            L->off_state[b][k] = off;
+            off += align_up(L->state_elems * 4);
+        }
+    if (cfg->variant == ZERO_VARIANT_TWO_PASS) {
+        L->off_reduced = off;
+        off += align_up(L->state_elems * 4);
+    }
+    if (cfg->stage == 3) {
+        L->off_shard16 = off;
+        off += align_up(L->state_elems * 2);
+    }
+    L->total = off;
+    return ZERO_OK;
+}
+
+void fill_ledger(const Layout& L, zero_ledger* out)
+{
+    std::memset(out, 0, sizeof(*out));
+    const double psi = (double)L.psi, nd = (double)L.nd, K = 12.0;
+    // [P1] "Where 16 bytes per parameter comes from": 2 + 2 + K, K = 12;
+    // [P2] "The Mathematics": M_states(p, Nd)
+    out->formula_bytes[0] = (2.0 + 2.0 + K) * psi;
+    out->formula_bytes[1] = 4.0 * psi + K * psi / nd;
+    out->formula_bytes[2] = 2.0 * psi + (2.0 + K) * psi / nd;
+    out->formula_bytes[3] = (2.0 + 2.0 + K) * psi / nd;
+    int64_t max_part = 0, max_shard = 0;
+    for (int r = 0; r < L.nd; ++r) {
+        int64_t b, e;
+        split(L.psi, L.nd, r, &b, &e);
+        max_part = std::max(max_part, e - b);
+        int64_t s = 0;
+        for (int64_t n : L.numel) {
+            int64_t cb, ce;
+            split(n, L.nd, r, &cb, &ce);
+            s += ce - cb;
+        }
+        max_shard = std::max(max_shard, s);
+    }
+    out->exact_bytes[0] = 16 * L.psi;
+    out->exact_bytes[1] = 4 * L.psi + 12 * max_part;
+    out->exact_bytes[2] = 2 * L.psi + 14 * max_part;
+    out->exact_bytes[3] = 16 * max_shard;
+    // ring collectives: each rank sends everything but the chunk it keeps
+    const int64_t rs = (int64_t)L.nd * L.psi - L.psi;
+    out->comm_elements[0] = rs;
+    out->comm_elements[1] = rs;
+    out->comm_elements[2] = 2 * rs;
+    out->comm_elements[3] = 2 * rs;
+    out->comm_elements[4] = 2 * rs;
+    out->comm_elements[5] = 3 * rs;
+    out->allreduce_buffer_bytes = 4 * L.psi;
+    out->transient_bytes = L.stage == 3 ? 2 * L.transient_elems : 0;
+    out->peak_stage3_bytes = out->exact_bytes[3] + 2 * L.transient_elems;
+    out->workspace_bytes = L.total;
+    out->partition_len = L.P;
+    out->state_elems = L.state_elems;
+    out->grad_len = L.grad_len;
+    for (int b = 0; b < 2; ++b) {
+        out->off_master[b] = L.off_state[b][0];
+        out->off_m[b] = L.off_state[b][1];
+        out->off_v[b] = L.off_state[b][2];
+    }
+    out->off_shard16 = L.off_shard16;
+    out->off_reduced = L.off_reduced;
+    out->n_units = L.stage == 3 ? L.n_units : 0;
+    out->n_out = L.stage == 3 ? 0 : L.n_out;
+}
+
+}  // namespace
+
+struct zero_handle {
+    Layout L;
+    char* ws = nullptr;
+    int device = 0;
+    int sms = 0;
+    int occ[zk::K_COUNT] = {};
+    zk::SegDesc* d_step_segs = nullptr;
+    zk::SegDesc* d_gather_segs = nullptr;
+    const uint16_t** d_grad_tab = nullptr;
+    uint16_t** d_out_tab = nullptr;
+    unsigned* d_flag = nullptr;
+    std::vector<const uint16_t*> grad_tab;  // host copy of what d_grad_tab holds
+    bool grad_tab_valid = false;
+    std::vector<uint16_t*> out_tab;
+    int cur = 0;  // live state buffer (fused variant)
+    int64_t t = 0;
+    unsigned call_id = 0;
+    unsigned host_flag = 0;
+    int last_cuda = 0;
+    bool pending = false;  // launched, not yet committed
+    int64_t pending_t = 0;
+    int pending_next = 0;
+    zk::StepArgs args{};   // arguments of the pending launch
+    // beta^t products for the last t computed (t-fold double products)
+    float bc_b1 = -1.0f, bc_b2 = -1.0f;
+    int64_t bc_t = -1;
+    double bc_p1 = 1.0, bc_p2 = 1.0;
+
+    float* state(int buf, int k) const { return reinterpret_cast<float*>(ws + L.off_state[buf][k]); }
+};
+
+namespace {
+
+int cuda_fail(zero_handle* h, cudaError_t e)
+{
+    if (h) h->last_cuda = (int)e;
+    return ZERO_ERR_CUDA;
+}
+
+int grid_for(const zero_handle* h, zk::Kernel k, int64_t chunks)
+{
+    const int64_t warps_per_block = zk::kThreads / 32;
+    const int64_t want = std::max<int64_t>(1, (chunks + warps_per_block - 1) / warps_per_block);
+    const int64_t cap = (int64_t)h->sms * std::max(1, h->occ[k]);
+    return (int)std::min(want, cap);
+}
+
+// (double)b^t as the t-fold product, continued from the previous call when
+// possible (same multiplications in the same order as a fresh loop).
+void bias_corrections(zero_handle* h, float b1, float b2, int64_t t, float* bc1, float* bc2)
+{
+    if (!(b1 == h->bc_b1 && b2 == h->bc_b2 && h->bc_t >= 0 && h->bc_t <= t)) {
+        h->bc_b1 = b1;
+        h->bc_b2 = b2;
+        h->bc_t = 0;
+        h->bc_p1 = 1.0;
+        h->bc_p2 = 1.0;
+    }
+    while (h->bc_t < t) {
+        h->bc_p1 = h->bc_p1 * (double)b1;
+        h->bc_p2 = h->bc_p2 * (double)b2;
+        ++h->bc_t;
+    }
+    *bc1 = (float)(1.0 - h->bc_p1);
+    *bc2 = (float)(1.0 - h->bc_p2);
+}
+
+}  // namespace
+
+ZERO_API int zero_state_bytes(const zero_config* cfg, zero_ledger* out)
+{
+    if (!out) return ZERO_ERR_ARG;
+    Layout L;
+    const int rc = build_layout(cfg, &L);
+    if (rc != ZERO_OK) return rc;
+    fill_ledger(L, out);
+    return ZERO_OK;
+}
+
+ZERO_API int zero_rank_shard(const zero_config* cfg, int32_t rank, int64_t* state_begin, int64_t* len)
+{
+    if (!state_begin || !len) return ZERO_ERR_ARG;
+    Layout L;
+    const int rc = build_layout(cfg, &L);
+    if (rc != ZERO_OK) return rc;
+    if (rank < 0 || rank >= L.nd) return ZERO_ERR_ARG;
+    *state_begin = L.shard_begin[rank];
+    *len = L.shard_len[rank];
+    return ZERO_OK;
+}
+
+ZERO_API int zero_unit_range(const zero_config* cfg, int32_t unit, int64_t* flat_begin, int64_t* numel)
+{
+    if (!flat_begin || !numel) return ZERO_ERR_ARG;
+    Layout L;
+    const int rc = build_layout(cfg, &L);
+    if (rc != ZERO_OK) return rc;
+    if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (unit < 0 || unit >= L.n_units) return ZERO_ERR_ARG;
+    *flat_begin = L.units[unit].flat_begin;
+    *numel = L.units[unit].numel;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace_bytes,
+                       const float* master_init, uint16_t* const* param_bufs, void* stream,
+                       zero_handle** out)
+{
+    if (!out) return ZERO_ERR_ARG;
+    *out = nullptr;
+    zero_handle* h = new (std::nothrow) zero_handle();
+    if (!h) return ZERO_ERR_INTERNAL;
+    int rc = build_layout(cfg, &h->L);
+    if (rc != ZERO_OK) {
+        delete h;
+        return rc;
+    }
+    const Layout& L = h->L;
+    // master_init may be NULL only when this handle owns no element (an
+    // empty partition in the single-rank view)
+    if (!workspace || (!master_init && L.state_elems > 0)) rc = ZERO_ERR_ARG;
+    else if (!aligned16(workspace) || !aligned16(master_init)) rc = ZERO_ERR_ALIGN;
+    else if ((int64_t)workspace_bytes < L.total) rc = ZERO_ERR_WORKSPACE;
+    if (rc == ZERO_OK && L.stage <= 2) {
+        if (!param_bufs) {
+            rc = ZERO_ERR_ARG;
+        } else {
+            for (int k = 0; k < L.n_out && rc == ZERO_OK; ++k) {
+                if (!param_bufs[k]) rc = ZERO_ERR_ARG;
+                else if (!aligned16(param_bufs[k])) rc = ZERO_ERR_ALIGN;
+            }
+        }
+    }
+    if (rc != ZERO_OK) {
+        delete h;
+        return rc;
+    }
+    h->ws = static_cast<char*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+    const int smem = zk::step_smem_bytes(L.nd, L.n_out);
+    for (int k = 0; k < zk::K_COUNT && e == cudaSuccess; ++k)
+        e = zk::occupancy((zk::Kernel)k, k == zk::K_GATHER ? 0 : smem, &h->occ[k]);
+    if (e != cudaSuccess) {
+        rc = cuda_fail(h, e);
+        delete h;
+        return rc;
+    }
+    h->d_flag = reinterpret_cast<unsigned*>(h->ws + L.off_flag);
+    h->d_grad_tab = reinterpret_cast<const uint16_t**>(h->ws + L.off_grad_tab);
+    h->d_out_tab = reinterpret_cast<uint16_t**>(h->ws + L.off_out_tab);
+    h->d_step_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_step_segs);
+    h->d_gather_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_gather_segs);
+    if (L.stage <= 2)
+        h->out_tab.assign(param_bufs, param_bufs + L.n_out);
+    else
+        h->out_tab.assign(1, reinterpret_cast<uint16_t*>(h->ws + L.off_shard16));
+
+    e = cudaMemsetAsync(h->ws + L.off_flag, 0, 256, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(h->d_out_tab, h->out_tab.data(), h->out_tab.size() * sizeof(uint16_t*),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !L.step_segs.empty())
+        e = cudaMemcpyAsync(h->d_step_segs, L.step_segs.data(), L.step_segs.size() * sizeof(zk::SegDesc),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !L.gather_segs.empty())
+        e = cudaMemcpyAsync(h->d_gather_segs, L.gather_segs.data(),
+                            L.gather_segs.size() * sizeof(zk::SegDesc), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && L.step_chunks > 0) {
+        zk::StepArgs a{};
+        a.segs = h->d_step_segs;
+        a.n_segs = (int)L.step_segs.size();
+        a.n_chunks = L.step_chunks;
+        a.outs = h->d_out_tab;
+        a.n_out = (int)h->out_tab.size();
+        a.nd = L.nd;
+        a.w_out = h->state(0, 0);
+        a.m_out = h->state(0, 1);
+        a.v_out = h->state(0, 2);
+        a.master_init = master_init;
+        a.flag = h->d_flag;
+        e = zk::launch_step(zk::K_INIT, a, grid_for(h, zk::K_INIT, L.step_chunks), s);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        rc = cuda_fail(h, e);
+        delete h;
+        return rc;
+    }
+    *out = h;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, float loss_scale,
+                              const zero_hyper* hp, void* stream)
+{
+    if (!h || !grads || !hp) return ZERO_ERR_ARG;
+    if (h->pending) return ZERO_ERR_ARG;  // the previous launch was not committed
+    if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale)) return ZERO_ERR_ARG;
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->beta1) || !std::isfinite(hp->beta2) ||
+        !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
+        return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    for (int k = 0; k < L.nd; ++k) {
+        if (!grads[k]) return ZERO_ERR_ARG;
+        if (!aligned16(grads[k])) return ZERO_ERR_ALIGN;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (!h->grad_tab_valid || !std::equal(grads, grads + L.nd, h->grad_tab.begin())) {
+        h->grad_tab.assign(grads, grads + L.nd);
+        e = cudaMemcpyAsync(h->d_grad_tab, h->grad_tab.data(), L.nd * sizeof(uint16_t*),
+                            cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+        h->grad_tab_valid = true;
+    }
+    if (++h->call_id == 0) ++h->call_id;  // 0 is the flag's initial value
+
+    const int64_t t_new = h->t + 1;
+    zk::StepArgs& a = h->args;
+    a = zk::StepArgs{};
+    a.segs = h->d_step_segs;
+    a.n_segs = (int)L.step_segs.size();
+    a.n_chunks = L.step_chunks;
+    a.grads = h->d_grad_tab;
+    a.outs = h->d_out_tab;
+    a.nd = L.nd;
+    a.n_out = (int)h->out_tab.size();
+    a.flag = h->d_flag;
+    a.call_id = h->call_id;
+    a.c.inv_scale = (float)(1.0 / (double)loss_scale);
+    a.c.lr = hp->lr;
+    a.c.b1 = hp->beta1;
+    a.c.b2 = hp->beta2;
+    a.c.omb1 = 1.0f - hp->beta1;
+    a.c.omb2 = 1.0f - hp->beta2;
+    a.c.eps = hp->eps;
+    a.c.wd = hp->weight_decay;
+    bias_corrections(h, hp->beta1, hp->beta2, t_new, &a.c.bc1, &a.c.bc2);
+
+    const bool fused = L.variant == ZERO_VARIANT_FUSED;
+    const int nxt = fused ? 1 - h->cur : h->cur;
+    a.w_in = h->state(h->cur, 0);
+    a.m_in = h->state(h->cur, 1);
+    a.v_in = h->state(h->cur, 2);
+    a.w_out = h->state(nxt, 0);
+    a.m_out = h->state(nxt, 1);
+    a.v_out = h->state(nxt, 2);
+    if (L.step_chunks > 0) {
+        if (fused) {
+            e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
+        } else {
+            a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
+            e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s);
+            if (e == cudaSuccess)
+                e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s);
+        }
+        if (e != cudaSuccess) return cuda_fail(h, e);
+    }
+    h->pending = true;
+    h->pending_t = t_new;
+    h->pending_next = nxt;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
+{
+    if (skipped) *skipped = 0;
+    if (!h || !h->pending) return ZERO_ERR_ARG;
+    h->pending = false;
+    const Layout& L = h->L;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // a copy into pageable host memory returns once the stream has reached it
+    cudaError_t e = cudaMemcpyAsync(&h->host_flag, h->d_flag, sizeof(unsigned),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    if (h->host_flag == h->call_id) {
+        // Overflow: the state buffers do not switch (fused) or were never
+        // written (two-pass). The fused pass already wrote fp16 parameters,
+        // so rewrite them from the unchanged master.
+        if (L.variant == ZERO_VARIANT_FUSED && L.step_chunks > 0) {
+            zk::StepArgs a = h->args;
+            a.w_in = h->state(h->cur, 0);
+            e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
+            if (e != cudaSuccess) return cuda_fail(h, e);
+        }
+        if (skipped) *skipped = 1;
+        return ZERO_SKIPPED;
+    }
+    h->t = h->pending_t;
+    h->cur = h->pending_next;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_step(zero_handle* h, const uint16_t* const* grads, float loss_scale,
+                       const zero_hyper* hp, void* stream, int* skipped)
+{
+    if (skipped) *skipped = 0;
+    const int rc = zero_step_launch(h, grads, loss_scale, hp, stream);
+    if (rc != ZERO_OK) return rc;
+    return zero_step_commit(h, stream, skipped);
+}
+
+ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
+{
+    if (!h || h->pending) return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (unit < 0 || unit >= L.n_units || !out) return ZERO_ERR_ARG;
+    if (!aligned16(out)) return ZERO_ERR_ALIGN;
+    const Unit& U = L.units[unit];
+    if (U.n_chunks == 0) return ZERO_OK;
+    zk::GatherArgs g{};
+    g.segs = h->d_gather_segs + U.seg0;
+    g.n_segs = (int)U.n_segs;
+    g.n_chunks = U.n_chunks;
+    g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
+    g.dst = out;
+    const cudaError_t e = zk::launch_gather(g, grid_for(h, zk::K_GATHER, U.n_chunks),
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+}
+
+ZERO_API int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t)
+{
+    if (!h) return ZERO_ERR_ARG;
+    if (master) *master = h->state(h->cur, 0);
+    if (m) *m = h->state(h->cur, 1);
+    if (v) *v = h->state(h->cur, 2);
+    if (t) *t = h->t;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream)
+{
+    if (!dst || !src || bytes % 16 != 0) return ZERO_ERR_ARG;
+    if (!aligned16(dst) || !aligned16(src)) return ZERO_ERR_ALIGN;
+    if (bytes == 0) return ZERO_OK;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ZERO_ERR_CUDA;
+    const cudaError_t e = zk::launch_copy(dst, src, bytes, sms * 8, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA;
+}
+
+ZERO_API int zero_last_cuda_error(const zero_handle* h) { return h ? h->last_cuda : 0; }
+
+ZERO_API const char* zero_error_string(int code)
+{
+    switch (code) {
+        case ZERO_OK: return "ok";
+        case ZERO_SKIPPED: return "step skipped: non-finite unscaled gradient";
+        case ZERO_ERR_ARG: return "invalid argument";
+        case ZERO_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        case ZERO_ERR_STAGE: return "call not valid for this ZeRO stage";
+        case ZERO_ERR_WORKSPACE: return "workspace too small";
+        case ZERO_ERR_CUDA: return "CUDA error";
+        case ZERO_ERR_INTERNAL: return "internal error";
+        default: return "unknown error code";
+    }
+}
+
+ZERO_API void zero_destroy(zero_handle* h) { delete h; }

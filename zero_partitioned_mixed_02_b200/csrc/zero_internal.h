@@ -1,0 +1,84 @@
+// Internal interface between the host ABI (zero_abi.cu) and the kernels
+// (zero_kernels.cu). Not installed; the public boundary is include/zero.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zk {
+
+constexpr int kThreads = 256;           // threads per block of every kernel
+constexpr int kGroup = 8;               // elements one lane handles per vector item (16 B of fp16)
+constexpr int kChunkGroups = 32;        // groups per warp chunk (one per lane)
+constexpr int kChunkElems = kGroup * kChunkGroups;
+
+// One contiguous run of elements. A run is a piece of one rank's partition
+// (stage 1/2) or one rank's chunk of one tensor (stage 3). Three index spaces:
+// the gradient buffers (grad), the state arrays (state), the fp16 output
+// buffers (out). The run is cut, relative to the gradient index, into a scalar
+// head up to the first multiple of 8, a body of 8-element groups, and a scalar
+// tail. Work is handed out in warp chunks: ceil(groups / 32) vector chunks,
+// then one scalar chunk if the head or tail is non-empty.
+struct alignas(16) SegDesc {
+    long long grad_begin;
+    long long state_begin;
+    long long out_begin;
+    long long len;
+    long long chunk_begin;  // first chunk of this run in the launch's chunk numbering
+    int head;               // scalar elements before the body
+    int tail;               // scalar elements after the body
+};
+static_assert(sizeof(SegDesc) == 48, "SegDesc layout");
+
+// Per-step binary32 constants, computed on the host.
+struct Coef {
+    float inv_scale, lr, b1, b2, omb1, omb2, bc1, bc2, eps, wd;
+};
+
+struct StepArgs {
+    const SegDesc* segs;
+    int n_segs;
+    long long n_chunks;
+    const uint16_t* const* grads;  // device table, nd entries
+    uint16_t* const* outs;         // device table, n_out entries
+    int nd;
+    int n_out;
+    const float* w_in;
+    const float* m_in;
+    const float* v_in;
+    float* w_out;
+    float* m_out;
+    float* v_out;
+    float* red;                    // two-pass: reduced unscaled gradients (state order)
+    const float* master_init;      // init: initial master weights (gradient order)
+    unsigned* flag;                // overflow word: holds the id of the last call that overflowed
+    unsigned call_id;
+    Coef c;
+};
+
+struct GatherArgs {
+    const SegDesc* segs;  // grad_begin = index into src, out_begin = index into dst
+    int n_segs;
+    long long n_chunks;
+    const uint16_t* src;
+    uint16_t* dst;
+};
+
+enum Kernel : int {
+    K_STEP_FUSED = 0,  // reduce + unscale + flag + Adam into the next buffer + fp16 write-back
+    K_REDUCE = 1,      // two-pass, pass 1: reduce + unscale + flag into red
+    K_UPDATE = 2,      // two-pass, pass 2: flag check, Adam in place + fp16 write-back
+    K_CAST = 3,        // fp16 write-back of the current master (overflow roll-back)
+    K_INIT = 4,        // master = master_init, m = v = 0, fp16 write-back
+    K_GATHER = 5,      // stage-3 layer gather
+    K_COUNT = 6
+};
+
+// Blocks per SM the kernel reaches with `smem` bytes of dynamic shared memory.
+cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm);
+cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cudaStream_t s);
+int step_smem_bytes(int nd, int n_out);
+
+}  // namespace zk

@@ -1,0 +1,418 @@
+// Device kernels of libzero (sm_100a).
+//
+// All kernels share one work decomposition: a table of runs (SegDesc), each
+// cut into warp chunks of 32 x 8 elements plus one scalar chunk for its ragged
+// head and tail. A persistent grid walks the chunks warp by warp (warp w takes
+// chunks w, w + W, w + 2W, ...), so at any moment the whole GPU streams one
+// narrow window of every buffer. Each lane moves 16-byte vectors of 8 fp16
+// values; the fp32 state uses 16-byte vectors when its alignment allows and
+// narrower accesses when a run's state index is out of phase with its
+// gradient index. Every access is a streaming (evict-first) load or store:
+// each byte is touched once per step.
+//
+// The path is pure streaming arithmetic (about 20 flops per element against
+// at least 56 bytes at Nd = 8), bounded by HBM bandwidth, so no tensor cores.
+//
+// Arithmetic is written with explicit round-to-nearest intrinsics in the
+// order the step defines, so the results do not depend on FMA contraction.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zero_internal.h"
+
+namespace zk {
+namespace {
+
+__device__ __forceinline__ bool nonfinite(float x)
+{
+    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+__device__ __forceinline__ float h2f(unsigned short b) { return __half2float(__ushort_as_half(b)); }
+
+__device__ __forceinline__ unsigned short f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+__device__ __forceinline__ void unpack8(const uint4 q, float (&x)[8])
+{
+    const unsigned u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        x[2 * k] = h2f((unsigned short)(u[k] & 0xffffu));
+        x[2 * k + 1] = h2f((unsigned short)(u[k] >> 16));
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&x)[8])
+{
+    unsigned u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = (unsigned)f2h(x[2 * k]) | ((unsigned)f2h(x[2 * k + 1]) << 16);
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// ---- alignment-adaptive vector accesses (the branch is uniform over a run) ----
+
+__device__ __forceinline__ void ld8(const float* p, float (&x)[8])
+{
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0) {
+        const float4 lo = __ldcs(reinterpret_cast<const float4*>(p));
+        const float4 hi = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+        x[0] = lo.x; x[1] = lo.y; x[2] = lo.z; x[3] = lo.w;
+        x[4] = hi.x; x[5] = hi.y; x[6] = hi.z; x[7] = hi.w;
+    } else if ((a & 7u) == 0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 t = __ldcs(reinterpret_cast<const float2*>(p) + k);
+            x[2 * k] = t.x;
+            x[2 * k + 1] = t.y;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = __ldcs(p + k);
+    }
+}
+
+__device__ __forceinline__ void st8(float* p, const float (&x)[8])
+{
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0) {
+        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+        __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
+    } else if ((a & 7u) == 0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            __stcs(reinterpret_cast<float2*>(p) + k, make_float2(x[2 * k], x[2 * k + 1]));
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) __stcs(p + k, x[k]);
+    }
+}
+
+__device__ __forceinline__ void st_h8(uint16_t* p, const uint4 q)
+{
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0) {
+        __stcs(reinterpret_cast<uint4*>(p), q);
+    } else if ((a & 7u) == 0) {
+        __stcs(reinterpret_cast<uint2*>(p), make_uint2(q.x, q.y));
+        __stcs(reinterpret_cast<uint2*>(p) + 1, make_uint2(q.z, q.w));
+    } else if ((a & 3u) == 0) {
+        unsigned* u = reinterpret_cast<unsigned*>(p);
+        __stcs(u, q.x);
+        __stcs(u + 1, q.y);
+        __stcs(u + 2, q.z);
+        __stcs(u + 3, q.w);
+    } else {
+        unsigned short* h = reinterpret_cast<unsigned short*>(p);
+        const unsigned u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            __stcs(h + 2 * k, (unsigned short)(u[k] & 0xffffu));
+            __stcs(h + 2 * k + 1, (unsigned short)(u[k] >> 16));
+        }
+    }
+}
+
+__device__ __forceinline__ uint4 ld_h8(const uint16_t* p)
+{
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+// ---- the step's arithmetic ----
+
+// Rank-ordered binary32 sum of the Nd fp16 gradients of 8 consecutive
+// elements (16-byte aligned). Loads are issued 8 ranks at a time ahead of the
+// additions, so up to 8 x 16 bytes per lane are in flight.
+__device__ __forceinline__ void reduce8(const uint16_t* const* gp, int nd, long long gi,
+                                        float (&s)[8])
+{
+    uint4 q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < nd) q[j] = ld_h8(gp[j] + gi);
+    unpack8(q[0], s);
+#pragma unroll
+    for (int j = 1; j < 8; ++j) {
+        if (j < nd) {
+            float x[8];
+            unpack8(q[j], x);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
+        }
+    }
+    for (int r0 = 8; r0 < nd; r0 += 8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (r0 + j < nd) q[j] = ld_h8(gp[r0 + j] + gi);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (r0 + j < nd) {
+                float x[8];
+                unpack8(q[j], x);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float reduce1(const uint16_t* const* gp, int nd, long long gi)
+{
+    float s = h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[0] + gi)));
+    for (int r = 1; r < nd; ++r)
+        s = __fadd_rn(s, h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[r] + gi))));
+    return s;
+}
+
+// One element of mixed-precision Adam (bias-corrected, decoupled weight decay
+// scaled by lr), binary32, in the order of the step's definition.
+__device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, const Coef& c)
+{
+    const float m1 = __fadd_rn(__fmul_rn(c.b1, m), __fmul_rn(c.omb1, g));
+    const float v1 = __fadd_rn(__fmul_rn(c.b2, v), __fmul_rn(c.omb2, __fmul_rn(g, g)));
+    const float mh = __fdiv_rn(m1, c.bc1);
+    const float vh = __fdiv_rn(v1, c.bc2);
+    const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), c.eps));
+    w = __fsub_rn(w, __fmul_rn(c.lr, __fadd_rn(u, __fmul_rn(c.wd, w))));
+    m = m1;
+    v = v1;
+}
+
+// ---- per-item bodies of the step kernels ----
+
+template <int K>
+__device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* const* gp,
+                                         uint16_t* const* op, const SegDesc& d, long long e,
+                                         bool& bad)
+{
+    const long long gi = d.grad_begin + e, si = d.state_begin + e, oi = d.out_begin + e;
+    float w[8], m[8], v[8], g[8];
+    if (K == K_INIT) {
+        ld8(a.master_init + gi, w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = 0.0f;
+        st8(a.w_out + si, w);
+        st8(a.m_out + si, m);
+        st8(a.v_out + si, m);
+    } else if (K == K_CAST) {
+        ld8(a.w_in + si, w);
+    } else {
+        if (K == K_STEP_FUSED || K == K_UPDATE) {
+            ld8(a.w_in + si, w);
+            ld8(a.m_in + si, m);
+            ld8(a.v_in + si, v);
+        }
+        if (K == K_STEP_FUSED || K == K_REDUCE) {
+            reduce8(gp, a.nd, gi, g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                g[j] = __fmul_rn(g[j], a.c.inv_scale);
+                bad |= nonfinite(g[j]);
+            }
+        }
+        if (K == K_REDUCE) {
+            st8(a.red + si, g);
+            return;
+        }
+        if (K == K_UPDATE) ld8(a.red + si, g);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], a.c);
+        st8(a.w_out + si, w);
+        st8(a.m_out + si, m);
+        st8(a.v_out + si, v);
+    }
+    const uint4 h = pack8(w);
+    for (int k = 0; k < a.n_out; ++k) st_h8(op[k] + oi, h);
+}
+
+template <int K>
+__device__ __forceinline__ void step_scalar(const StepArgs& a, const uint16_t* const* gp,
+                                            uint16_t* const* op, const SegDesc& d, long long e,
+                                            bool& bad)
+{
+    const long long gi = d.grad_begin + e, si = d.state_begin + e, oi = d.out_begin + e;
+    float w = 0.0f, m = 0.0f, v = 0.0f, g = 0.0f;
+    if (K == K_INIT) {
+        w = __ldcs(a.master_init + gi);
+        __stcs(a.w_out + si, w);
+        __stcs(a.m_out + si, 0.0f);
+        __stcs(a.v_out + si, 0.0f);
+    } else if (K == K_CAST) {
+        w = __ldcs(a.w_in + si);
+    } else {
+        if (K == K_STEP_FUSED || K == K_UPDATE) {
+            w = __ldcs(a.w_in + si);
+            m = __ldcs(a.m_in + si);
+            v = __ldcs(a.v_in + si);
+        }
+        if (K == K_STEP_FUSED || K == K_REDUCE) {
+            g = __fmul_rn(reduce1(gp, a.nd, gi), a.c.inv_scale);
+            bad |= nonfinite(g);
+        }
+        if (K == K_REDUCE) {
+            __stcs(a.red + si, g);
+            return;
+        }
+        if (K == K_UPDATE) g = __ldcs(a.red + si);
+        adam1(g, w, m, v, a.c);
+        __stcs(a.w_out + si, w);
+        __stcs(a.m_out + si, m);
+        __stcs(a.v_out + si, v);
+    }
+    const unsigned short h = f2h(w);
+    for (int k = 0; k < a.n_out; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);
+}
+
+// Largest run index whose first chunk is <= c.
+__device__ __forceinline__ int find_run(const SegDesc* segs, int n, long long c)
+{
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (segs[mid].chunk_begin <= c)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Walk the chunks of a run table; call vec(d, e) for each 8-element group at
+// run offset e and scal(d, e) for each head/tail element.
+template <class Vec, class Scal>
+__device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long n_chunks, Vec vec,
+                                     Scal scal)
+{
+    const int lane = threadIdx.x & 31;
+    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+    SegDesc d;
+    long long lo = 0, hi = 0;  // chunk range of the cached run d (empty at start)
+    for (long long c = warp; c < n_chunks; c += n_warps) {
+        if (c < lo || c >= hi) {
+            const int s = find_run(segs, n_segs, c);
+            d = segs[s];
+            lo = d.chunk_begin;
+            hi = (s + 1 < n_segs) ? segs[s + 1].chunk_begin : n_chunks;
+        }
+        const long long groups = (d.len - d.head - d.tail) >> 3;
+        const long long vec_chunks = (groups + kChunkGroups - 1) / kChunkGroups;
+        const long long k = c - d.chunk_begin;
+        if (k < vec_chunks) {
+            const long long gidx = k * kChunkGroups + lane;
+            if (gidx < groups) vec(d, (long long)d.head + gidx * kGroup);
+        } else {
+            long long e = -1;
+            if (lane < d.head)
+                e = lane;
+            else if (lane >= 8 && lane - 8 < d.tail)
+                e = d.len - d.tail + (lane - 8);
+            if (e >= 0) scal(d, e);
+        }
+    }
+}
+
+template <int K>
+__global__ void __launch_bounds__(kThreads) step_kernel(const StepArgs a)
+{
+    extern __shared__ uintptr_t s_ptr[];
+    if (K == K_UPDATE) {
+        // pass 2 of the two-pass variant: the whole step is skipped on overflow
+        if (*reinterpret_cast<volatile unsigned*>(a.flag) == a.call_id) return;
+    }
+    constexpr bool kGrads = (K == K_STEP_FUSED || K == K_REDUCE);
+    const int n_g = kGrads ? a.nd : 0;
+    const int n_o = (K == K_REDUCE) ? 0 : a.n_out;
+    for (int i = threadIdx.x; i < n_g + n_o; i += blockDim.x)
+        s_ptr[i] = (i < n_g) ? reinterpret_cast<uintptr_t>(a.grads[i])
+                             : reinterpret_cast<uintptr_t>(a.outs[i - n_g]);
+    __syncthreads();
+    const uint16_t* const* gp = reinterpret_cast<const uint16_t* const*>(s_ptr);
+    uint16_t* const* op = reinterpret_cast<uint16_t* const*>(s_ptr + n_g);
+
+    bool bad = false;
+    walk(
+        a.segs, a.n_segs, a.n_chunks,
+        [&](const SegDesc& d, long long e) { step_vec<K>(a, gp, op, d, e, bad); },
+        [&](const SegDesc& d, long long e) { step_scalar<K>(a, gp, op, d, e, bad); });
+
+    if (kGrads) {
+        // one atomic per warp that saw a non-finite unscaled gradient
+        if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicMax(a.flag, a.call_id);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) gather_kernel(const GatherArgs a)
+{
+    walk(
+        a.segs, a.n_segs, a.n_chunks,
+        [&](const SegDesc& d, long long e) {
+            st_h8(a.dst + d.out_begin + e, ld_h8(a.src + d.grad_begin + e));
+        },
+        [&](const SegDesc& d, long long e) {
+            __stcs(reinterpret_cast<unsigned short*>(a.dst + d.out_begin + e),
+                   __ldcs(reinterpret_cast<const unsigned short*>(a.src + d.grad_begin + e)));
+        });
+}
+
+__global__ void __launch_bounds__(kThreads) copy_kernel(uint4* dst, const uint4* src, long long n)
+{
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        __stcs(dst + i, __ldcs(src + i));
+}
+
+const void* kernel_ptr(Kernel k)
+{
+    switch (k) {
+        case K_STEP_FUSED: return reinterpret_cast<const void*>(&step_kernel<K_STEP_FUSED>);
+        case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE>);
+        case K_UPDATE: return reinterpret_cast<const void*>(&step_kernel<K_UPDATE>);
+        case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST>);
+        case K_INIT: return reinterpret_cast<const void*>(&step_kernel<K_INIT>);
+        case K_GATHER: return reinterpret_cast<const void*>(&gather_kernel);
+        default: return nullptr;
+    }
+}
+
+}  // namespace
+
+int step_smem_bytes(int nd, int n_out) { return (nd + n_out) * (int)sizeof(uintptr_t); }
+
+cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm)
+{
+    const void* f = kernel_ptr(k);
+    if (!f) return cudaErrorInvalidValue;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, f, kThreads, smem);
+}
+
+cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s)
+{
+    const int smem = step_smem_bytes(a.nd, a.n_out);
+    switch (k) {
+        case K_STEP_FUSED: step_kernel<K_STEP_FUSED><<<grid, kThreads, smem, s>>>(a); break;
+        case K_REDUCE: step_kernel<K_REDUCE><<<grid, kThreads, smem, s>>>(a); break;
+        case K_UPDATE: step_kernel<K_UPDATE><<<grid, kThreads, smem, s>>>(a); break;
+        case K_CAST: step_kernel<K_CAST><<<grid, kThreads, smem, s>>>(a); break;
+        case K_INIT: step_kernel<K_INIT><<<grid, kThreads, smem, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s)
+{
+    gather_kernel<<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cudaStream_t s)
+{
+    copy_kernel<<<grid, kThreads, 0, s>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src),
+                                          (long long)(bytes / 16));
+    return cudaGetLastError();
+}
+
+}  // namespace zk

@@ -1,0 +1,87 @@
+"""User-facing object over the C ABI: PyTorch allocates the device memory and
+supplies the stream; libzero does all the work.
+
+    opt = ZeroAdam(psi, nd, stage, master_init, param_bufs, tensors=..., variant=...)
+    skipped = opt.step(grads, loss_scale, lr=..., betas=..., eps=..., weight_decay=...)
+    opt.gather_layer(unit, out)          # stage 3
+    w, m, v = opt.state()                # live fp32 state (views of the workspace)
+"""
+from __future__ import annotations
+
+from typing import Sequence
+
+import torch
+
+from . import _abi as A
+
+
+class ZeroAdam:
+    def __init__(self, psi: int, nd: int, stage: int, master_init: torch.Tensor,
+                 param_bufs: Sequence[torch.Tensor] | None = None, *, rank_view: int = -1,
+                 variant: int = A.ZERO_VARIANT_FUSED,
+                 tensors: Sequence[tuple[int, int]] | None = None,
+                 stream: torch.cuda.Stream | None = None):
+        self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors)
+        self.ledger = A.zero_state_bytes(self.cfg)
+        dev = master_init.device
+        if dev.type != "cuda":
+            raise ValueError("master_init must be a CUDA tensor")
+        if master_init.dtype != torch.float32 or not master_init.is_contiguous():
+            raise ValueError("master_init must be contiguous float32")
+        self.stream = stream or torch.cuda.current_stream(dev)
+        self.workspace = torch.empty(self.ledger.workspace_bytes, dtype=torch.uint8, device=dev)
+        self.param_bufs = list(param_bufs) if param_bufs is not None else None
+        ptrs = [p.data_ptr() for p in self.param_bufs] if self.param_bufs is not None else None
+        self.h = A.zero_init(self.cfg, self.workspace.data_ptr(), self.ledger.workspace_bytes,
+                             master_init.data_ptr(), ptrs, self.stream.cuda_stream)
+        self.nd = nd
+
+    def step(self, grads: Sequence[torch.Tensor] | Sequence[int], loss_scale: float, *, lr=1e-3,
+             betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0) -> bool:
+        ptrs = [g if isinstance(g, int) else g.data_ptr() for g in grads]
+        if len(ptrs) != self.nd:
+            raise ValueError(f"expected {self.nd} gradient buffers, got {len(ptrs)}")
+        hp = A.zero_hyper(lr, betas[0], betas[1], eps, weight_decay)
+        rc = A.zero_step(self.h, ptrs, loss_scale, hp, self.stream.cuda_stream)
+        return rc == A.ZERO_SKIPPED
+
+    def gather_layer(self, unit: int, out: torch.Tensor) -> None:
+        A.zero_gather_layer(self.h, unit, out.data_ptr(), self.stream.cuda_stream)
+
+    def unit_range(self, unit: int) -> tuple[int, int]:
+        return A.zero_unit_range(self.cfg, unit)
+
+    def rank_shard(self, rank: int) -> tuple[int, int]:
+        return A.zero_rank_shard(self.cfg, rank)
+
+    @property
+    def t(self) -> int:
+        return A.zero_current_state(self.h)[3]
+
+    def _view_f32(self, ptr: int) -> torch.Tensor:
+        off = ptr - self.workspace.data_ptr()
+        n = self.ledger.state_elems
+        return self.workspace[off: off + 4 * n].view(torch.float32)
+
+    def state(self) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        w, m, v, _ = A.zero_current_state(self.h)
+        return self._view_f32(w), self._view_f32(m), self._view_f32(v)
+
+    def shard16(self) -> torch.Tensor:
+        """Stage 3: the fp16 parameter shards of all ranks (state order), as int16 bits."""
+        off = self.ledger.off_shard16
+        if off < 0:
+            raise ValueError("only stage 3 keeps fp16 shards")
+        n = self.ledger.state_elems
+        return self.workspace[off: off + 2 * n].view(torch.int16)
+
+    def close(self) -> None:
+        if self.h:
+            A.zero_destroy(self.h)
+            self.h = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
