@@ -60,7 +60,7 @@ struct Layout {
     int64_t transient_elems = 0;
 };
 
-// Cut a run at the first 8-aligned gradient index and give it its chunks.
+// Cut a run at the first line-aligned gradient index and give it its chunks.
 void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, int64_t state_begin,
              int64_t out_begin, int64_t len)
 {
@@ -70,14 +70,14 @@ void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, i
     d.state_begin = state_begin;
     d.out_begin = out_begin;
     d.len = len;
-    int64_t head = (zk::kGroup - (grad_begin % zk::kGroup)) % zk::kGroup;
+    int64_t head = (zk::kLineElems - (grad_begin % zk::kLineElems)) % zk::kLineElems;
     if (head > len) head = len;
-    const int64_t groups = (len - head) / zk::kGroup;
+    const int64_t quads = (len - head) / zk::kQuad;
     d.head = (int)head;
-    d.tail = (int)(len - head - groups * zk::kGroup);
+    d.tail = (int)(len - head - quads * zk::kQuad);
     d.chunk_begin = *chunks;
-    const int64_t vec = (groups + zk::kChunkGroups - 1) / zk::kChunkGroups;
-    *chunks += vec + ((d.head + d.tail) > 0 ? 1 : 0);
+    const int64_t vec = (quads + zk::kQuadsPerChunk - 1) / zk::kQuadsPerChunk;
+    *chunks += vec + (d.head + d.tail + 31) / 32;
     v.push_back(d);
 }
 

@@ -7,18 +7,27 @@
 
 namespace zk {
 
-constexpr int kThreads = 256;           // threads per block of every kernel
-constexpr int kGroup = 8;               // elements one lane handles per vector item (16 B of fp16)
-constexpr int kChunkGroups = 32;        // groups per warp chunk (one per lane)
-constexpr int kChunkElems = kGroup * kChunkGroups;
+constexpr int kThreads = 256;  // threads per block of every kernel
+// Vector work moves "quads" of 4 consecutive elements: 8 bytes of fp16, 16 of
+// fp32. A warp chunk is 64 quads (256 elements); lane L takes quads L and
+// L + 32, so each warp instruction touches one contiguous, sector-aligned run
+// (256 B of fp16, 512 B of fp32) and a lane keeps 8 elements in flight.
+constexpr int kQuad = 4;
+constexpr int kQuadsPerChunk = 64;
+constexpr int kChunkElems = kQuad * kQuadsPerChunk;
+// Vector bodies start on a multiple of kLineElems gradient elements: one
+// 128-byte line of fp16 (two of fp32). Every warp chunk then covers whole
+// 32-byte sectors, so no sector is written in halves by two different warps
+// (a partial-sector write costs the memory system a read-modify-write).
+constexpr int kLineElems = 64;
 
 // One contiguous run of elements. A run is a piece of one rank's partition
 // (stage 1/2) or one rank's chunk of one tensor (stage 3). Three index spaces:
 // the gradient buffers (grad), the state arrays (state), the fp16 output
 // buffers (out). The run is cut, relative to the gradient index, into a scalar
-// head up to the first multiple of 8, a body of 8-element groups, and a scalar
-// tail. Work is handed out in warp chunks: ceil(groups / 32) vector chunks,
-// then one scalar chunk if the head or tail is non-empty.
+// head up to the first multiple of kLineElems, a body of quads, and a scalar
+// tail (< kQuad). Work is handed out in warp chunks: ceil(quads / 64) vector
+// chunks, then ceil((head + tail) / 32) scalar chunks.
 struct alignas(16) SegDesc {
     long long grad_begin;
     long long state_begin;

@@ -1,12 +1,15 @@
 // Device kernels of libzero (sm_100a).
 //
-// All kernels share one work decomposition: a table of runs (SegDesc), each
-// cut into warp chunks of 32 x 8 elements plus one scalar chunk for its ragged
-// head and tail. A persistent grid walks the chunks warp by warp (warp w takes
+// All kernels share one work decomposition: a table of runs (SegDesc). A run
+// is cut into warp chunks of 256 elements whose vector body starts on a
+// 128-byte line of the fp16 gradients, plus scalar chunks for the ragged head
+// and tail. A persistent grid walks the chunks warp by warp (warp w takes
 // chunks w, w + W, w + 2W, ...), so at any moment the whole GPU streams one
-// narrow window of every buffer. Each lane moves 16-byte vectors of 8 fp16
-// values; the fp32 state uses 16-byte vectors when its alignment allows and
-// narrower accesses when a run's state index is out of phase with its
+// narrow window of every buffer. Within a chunk lane L owns quads L and L + 32
+// (a quad is 4 consecutive elements): every warp load or store is then one
+// contiguous, sector-aligned run of 256 bytes (fp16) or 512 bytes (fp32), and
+// each lane keeps 8 elements of every stream in flight. fp32 state falls back
+// to narrower accesses when a run's state index is out of phase with its
 // gradient index. Every access is a streaming (evict-first) load or store:
 // each byte is touched once per step.
 //
@@ -21,6 +24,12 @@
 
 #include "zero_internal.h"
 
+// Minimum resident blocks per SM the step kernels are compiled for (caps
+// registers per thread at 65536 / (256 * ZK_MIN_BLOCKS)).
+#ifndef ZK_MIN_BLOCKS
+#define ZK_MIN_BLOCKS 1
+#endif
+
 namespace zk {
 namespace {
 
@@ -33,124 +42,148 @@ __device__ __forceinline__ float h2f(unsigned short b) { return __half2float(__u
 
 __device__ __forceinline__ unsigned short f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
 
-__device__ __forceinline__ void unpack8(const uint4 q, float (&x)[8])
+// ---- quads: 4 fp16 values packed in a uint2, 4 fp32 values ----
+
+__device__ __forceinline__ void unpack(const uint2 q, float* x)
 {
-    const unsigned u[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        x[2 * k] = h2f((unsigned short)(u[k] & 0xffffu));
-        x[2 * k + 1] = h2f((unsigned short)(u[k] >> 16));
-    }
+    x[0] = h2f((unsigned short)(q.x & 0xffffu));
+    x[1] = h2f((unsigned short)(q.x >> 16));
+    x[2] = h2f((unsigned short)(q.y & 0xffffu));
+    x[3] = h2f((unsigned short)(q.y >> 16));
 }
 
-__device__ __forceinline__ uint4 pack8(const float (&x)[8])
+__device__ __forceinline__ unsigned pack2(float lo, float hi)
 {
-    unsigned u[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = (unsigned)f2h(x[2 * k]) | ((unsigned)f2h(x[2 * k + 1]) << 16);
-    return make_uint4(u[0], u[1], u[2], u[3]);
+    return (unsigned)f2h(lo) | ((unsigned)f2h(hi) << 16);
 }
 
-// ---- alignment-adaptive vector accesses (the branch is uniform over a run) ----
+__device__ __forceinline__ uint2 pack(const float* x) { return make_uint2(pack2(x[0], x[1]), pack2(x[2], x[3])); }
 
-__device__ __forceinline__ void ld8(const float* p, float (&x)[8])
+// 4 fp16 values from p (8-byte aligned: quads start on multiples of 4).
+__device__ __forceinline__ uint2 ld_hq(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+
+// Store 4 fp16 values with the widest accesses p's alignment allows (the
+// branch is uniform over a run).
+__device__ __forceinline__ void st_hq(uint16_t* p, const uint2 q)
 {
     const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 15u) == 0) {
-        const float4 lo = __ldcs(reinterpret_cast<const float4*>(p));
-        const float4 hi = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-        x[0] = lo.x; x[1] = lo.y; x[2] = lo.z; x[3] = lo.w;
-        x[4] = hi.x; x[5] = hi.y; x[6] = hi.z; x[7] = hi.w;
-    } else if ((a & 7u) == 0) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 t = __ldcs(reinterpret_cast<const float2*>(p) + k);
-            x[2 * k] = t.x;
-            x[2 * k + 1] = t.y;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = __ldcs(p + k);
-    }
-}
-
-__device__ __forceinline__ void st8(float* p, const float (&x)[8])
-{
-    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 15u) == 0) {
-        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
-        __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
-    } else if ((a & 7u) == 0) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            __stcs(reinterpret_cast<float2*>(p) + k, make_float2(x[2 * k], x[2 * k + 1]));
-    } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) __stcs(p + k, x[k]);
-    }
-}
-
-__device__ __forceinline__ void st_h8(uint16_t* p, const uint4 q)
-{
-    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 15u) == 0) {
-        __stcs(reinterpret_cast<uint4*>(p), q);
-    } else if ((a & 7u) == 0) {
-        __stcs(reinterpret_cast<uint2*>(p), make_uint2(q.x, q.y));
-        __stcs(reinterpret_cast<uint2*>(p) + 1, make_uint2(q.z, q.w));
+    if ((a & 7u) == 0) {
+        __stcs(reinterpret_cast<uint2*>(p), q);
     } else if ((a & 3u) == 0) {
         unsigned* u = reinterpret_cast<unsigned*>(p);
         __stcs(u, q.x);
         __stcs(u + 1, q.y);
-        __stcs(u + 2, q.z);
-        __stcs(u + 3, q.w);
     } else {
         unsigned short* h = reinterpret_cast<unsigned short*>(p);
-        const unsigned u[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            __stcs(h + 2 * k, (unsigned short)(u[k] & 0xffffu));
-            __stcs(h + 2 * k + 1, (unsigned short)(u[k] >> 16));
-        }
+        __stcs(h, (unsigned short)(q.x & 0xffffu));
+        __stcs(h + 1, (unsigned short)(q.x >> 16));
+        __stcs(h + 2, (unsigned short)(q.y & 0xffffu));
+        __stcs(h + 3, (unsigned short)(q.y >> 16));
     }
 }
 
-__device__ __forceinline__ uint4 ld_h8(const uint16_t* p)
+// 4 fp32 values, widest access the alignment allows.
+__device__ __forceinline__ void ldq(const float* p, float* x)
 {
-    return __ldcs(reinterpret_cast<const uint4*>(p));
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0) {
+        const float4 t = __ldcs(reinterpret_cast<const float4*>(p));
+        x[0] = t.x;
+        x[1] = t.y;
+        x[2] = t.z;
+        x[3] = t.w;
+    } else if ((a & 7u) == 0) {
+        const float2 t0 = __ldcs(reinterpret_cast<const float2*>(p));
+        const float2 t1 = __ldcs(reinterpret_cast<const float2*>(p) + 1);
+        x[0] = t0.x;
+        x[1] = t0.y;
+        x[2] = t1.x;
+        x[3] = t1.y;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = __ldcs(p + k);
+    }
+}
+
+__device__ __forceinline__ void stq(float* p, const float* x)
+{
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0) {
+        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+    } else if ((a & 7u) == 0) {
+        __stcs(reinterpret_cast<float2*>(p), make_float2(x[0], x[1]));
+        __stcs(reinterpret_cast<float2*>(p) + 1, make_float2(x[2], x[3]));
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) __stcs(p + k, x[k]);
+    }
+}
+
+// A lane's pair of quads: elements [ea, ea + 4) and, if hb, [eb, eb + 4) of
+// the run; values 0..3 belong to the first quad, 4..7 to the second.
+struct Pair {
+    long long ea, eb;
+    bool hb;
+};
+
+__device__ __forceinline__ void ld_pair(const float* base, long long ia, long long ib, bool hb,
+                                        float (&x)[8])
+{
+    ldq(base + ia, x);
+    if (hb)
+        ldq(base + ib, x + 4);
+    else
+        x[4] = x[5] = x[6] = x[7] = 0.0f;
+}
+
+__device__ __forceinline__ void st_pair(float* base, long long ia, long long ib, bool hb,
+                                        const float (&x)[8])
+{
+    stq(base + ia, x);
+    if (hb) stq(base + ib, x + 4);
 }
 
 // ---- the step's arithmetic ----
 
-// Rank-ordered binary32 sum of the Nd fp16 gradients of 8 consecutive
-// elements (16-byte aligned). Loads are issued 8 ranks at a time ahead of the
-// additions, so up to 8 x 16 bytes per lane are in flight.
-__device__ __forceinline__ void reduce8(const uint16_t* const* gp, int nd, long long gi,
-                                        float (&s)[8])
+// Rank-ordered binary32 sum of the Nd fp16 gradients of a lane's two quads.
+// Loads are issued 8 ranks at a time ahead of the additions.
+__device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, long long ga,
+                                            long long gb, bool hb, float (&s)[8])
 {
-    uint4 q[8];
+    uint2 qa[8], qb[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        if (j < nd) q[j] = ld_h8(gp[j] + gi);
-    unpack8(q[0], s);
+    for (int j = 0; j < 8; ++j) {
+        if (j < nd) {
+            qa[j] = ld_hq(gp[j] + ga);
+            qb[j] = hb ? ld_hq(gp[j] + gb) : make_uint2(0u, 0u);
+        }
+    }
+    unpack(qa[0], s);
+    unpack(qb[0], s + 4);
 #pragma unroll
     for (int j = 1; j < 8; ++j) {
         if (j < nd) {
             float x[8];
-            unpack8(q[j], x);
+            unpack(qa[j], x);
+            unpack(qb[j], x + 4);
 #pragma unroll
             for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
         }
     }
     for (int r0 = 8; r0 < nd; r0 += 8) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (r0 + j < nd) q[j] = ld_h8(gp[r0 + j] + gi);
+        for (int j = 0; j < 8; ++j) {
+            if (r0 + j < nd) {
+                qa[j] = ld_hq(gp[r0 + j] + ga);
+                qb[j] = hb ? ld_hq(gp[r0 + j] + gb) : make_uint2(0u, 0u);
+            }
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if (r0 + j < nd) {
                 float x[8];
-                unpack8(q[j], x);
+                unpack(qa[j], x);
+                unpack(qb[j], x + 4);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
             }
@@ -184,47 +217,53 @@ __device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, con
 
 template <int K>
 __device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* const* gp,
-                                         uint16_t* const* op, const SegDesc& d, long long e,
+                                         uint16_t* const* op, const SegDesc& d, const Pair& p,
                                          bool& bad)
 {
-    const long long gi = d.grad_begin + e, si = d.state_begin + e, oi = d.out_begin + e;
+    const long long ga = d.grad_begin + p.ea, gb = d.grad_begin + p.eb;
+    const long long sa = d.state_begin + p.ea, sb = d.state_begin + p.eb;
+    const long long oa = d.out_begin + p.ea, ob = d.out_begin + p.eb;
+    const bool hb = p.hb;
     float w[8], m[8], v[8], g[8];
     if (K == K_INIT) {
-        ld8(a.master_init + gi, w);
+        ld_pair(a.master_init, ga, gb, hb, w);
 #pragma unroll
         for (int j = 0; j < 8; ++j) m[j] = 0.0f;
-        st8(a.w_out + si, w);
-        st8(a.m_out + si, m);
-        st8(a.v_out + si, m);
+        st_pair(a.w_out, sa, sb, hb, w);
+        st_pair(a.m_out, sa, sb, hb, m);
+        st_pair(a.v_out, sa, sb, hb, m);
     } else if (K == K_CAST) {
-        ld8(a.w_in + si, w);
+        ld_pair(a.w_in, sa, sb, hb, w);
     } else {
         if (K == K_STEP_FUSED || K == K_UPDATE) {
-            ld8(a.w_in + si, w);
-            ld8(a.m_in + si, m);
-            ld8(a.v_in + si, v);
+            ld_pair(a.w_in, sa, sb, hb, w);
+            ld_pair(a.m_in, sa, sb, hb, m);
+            ld_pair(a.v_in, sa, sb, hb, v);
         }
         if (K == K_STEP_FUSED || K == K_REDUCE) {
-            reduce8(gp, a.nd, gi, g);
+            reduce_pair(gp, a.nd, ga, gb, hb, g);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 g[j] = __fmul_rn(g[j], a.c.inv_scale);
-                bad |= nonfinite(g[j]);
+                bad |= nonfinite(g[j]);  // an absent second quad holds zeros
             }
         }
         if (K == K_REDUCE) {
-            st8(a.red + si, g);
+            st_pair(a.red, sa, sb, hb, g);
             return;
         }
-        if (K == K_UPDATE) ld8(a.red + si, g);
+        if (K == K_UPDATE) ld_pair(a.red, sa, sb, hb, g);
 #pragma unroll
         for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], a.c);
-        st8(a.w_out + si, w);
-        st8(a.m_out + si, m);
-        st8(a.v_out + si, v);
+        st_pair(a.w_out, sa, sb, hb, w);
+        st_pair(a.m_out, sa, sb, hb, m);
+        st_pair(a.v_out, sa, sb, hb, v);
     }
-    const uint4 h = pack8(w);
-    for (int k = 0; k < a.n_out; ++k) st_h8(op[k] + oi, h);
+    const uint2 h0 = pack(w), h1 = pack(w + 4);
+    for (int k = 0; k < a.n_out; ++k) {
+        st_hq(op[k] + oa, h0);
+        if (hb) st_hq(op[k] + ob, h1);
+    }
 }
 
 template <int K>
@@ -279,8 +318,8 @@ __device__ __forceinline__ int find_run(const SegDesc* segs, int n, long long c)
     return lo;
 }
 
-// Walk the chunks of a run table; call vec(d, e) for each 8-element group at
-// run offset e and scal(d, e) for each head/tail element.
+// Walk the chunks of a run table; call vec(d, pair) for each lane's pair of
+// quads and scal(d, e) for each head/tail element (offsets within the run).
 template <class Vec, class Scal>
 __device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long n_chunks, Vec vec,
                                      Scal scal)
@@ -297,25 +336,34 @@ __device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long 
             lo = d.chunk_begin;
             hi = (s + 1 < n_segs) ? segs[s + 1].chunk_begin : n_chunks;
         }
-        const long long groups = (d.len - d.head - d.tail) >> 3;
-        const long long vec_chunks = (groups + kChunkGroups - 1) / kChunkGroups;
+        const long long quads = (d.len - d.head - d.tail) / kQuad;
+        const long long vec_chunks = (quads + kQuadsPerChunk - 1) / kQuadsPerChunk;
         const long long k = c - d.chunk_begin;
         if (k < vec_chunks) {
-            const long long gidx = k * kChunkGroups + lane;
-            if (gidx < groups) vec(d, (long long)d.head + gidx * kGroup);
+            const long long qa = k * kQuadsPerChunk + lane;
+            const long long qb = qa + 32;
+            if (qa < quads) {
+                Pair p;
+                p.ea = d.head + qa * kQuad;
+                p.hb = qb < quads;
+                p.eb = p.hb ? d.head + qb * kQuad : p.ea;
+                vec(d, p);
+            }
         } else {
+            // scalar chunks: head elements first, then the tail
+            const long long q = (k - vec_chunks) * 32 + lane;
             long long e = -1;
-            if (lane < d.head)
-                e = lane;
-            else if (lane >= 8 && lane - 8 < d.tail)
-                e = d.len - d.tail + (lane - 8);
+            if (q < d.head)
+                e = q;
+            else if (q < d.head + d.tail)
+                e = d.len - d.tail + (q - d.head);
             if (e >= 0) scal(d, e);
         }
     }
 }
 
 template <int K>
-__global__ void __launch_bounds__(kThreads) step_kernel(const StepArgs a)
+__global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const StepArgs a)
 {
     extern __shared__ uintptr_t s_ptr[];
     if (K == K_UPDATE) {
@@ -335,7 +383,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const StepArgs a)
     bool bad = false;
     walk(
         a.segs, a.n_segs, a.n_chunks,
-        [&](const SegDesc& d, long long e) { step_vec<K>(a, gp, op, d, e, bad); },
+        [&](const SegDesc& d, const Pair& p) { step_vec<K>(a, gp, op, d, p, bad); },
         [&](const SegDesc& d, long long e) { step_scalar<K>(a, gp, op, d, e, bad); });
 
     if (kGrads) {
@@ -348,8 +396,11 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const GatherArgs a)
 {
     walk(
         a.segs, a.n_segs, a.n_chunks,
-        [&](const SegDesc& d, long long e) {
-            st_h8(a.dst + d.out_begin + e, ld_h8(a.src + d.grad_begin + e));
+        [&](const SegDesc& d, const Pair& p) {
+            const uint2 qa = ld_hq(a.src + d.grad_begin + p.ea);
+            const uint2 qb = p.hb ? ld_hq(a.src + d.grad_begin + p.eb) : make_uint2(0u, 0u);
+            st_hq(a.dst + d.out_begin + p.ea, qa);
+            if (p.hb) st_hq(a.dst + d.out_begin + p.eb, qb);
         },
         [&](const SegDesc& d, long long e) {
             __stcs(reinterpret_cast<unsigned short*>(a.dst + d.out_begin + e),
