@@ -212,6 +212,43 @@ int zero_current_state(const zero_handle* h, float** master, float** m, float** 
  * 16-byte aligned) from src to dst with 16-byte streaming loads and stores. */
 int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);
 
+/* ---- allocation-free step (no counterpart on the pages) ----
+ *
+ * Some callers cannot allocate device memory for a workspace: code whose
+ * device memory belongs to another allocator it cannot reach from plain C (an
+ * embedding framework's caching allocator, say), or code that must not pay
+ * cudaMalloc's cost and its implicit device synchronisation in the middle of
+ * a training step. zero_step_static serves them: one two-pass stage 1/2 step
+ * (all Nd ranks emulated, flat parameter vector) whose scratch -- the fp32
+ * reduced gradients, the overflow word and the pointer and run tables -- lives
+ * in a fixed array inside the library, so the call allocates nothing. The
+ * caller still owns and passes every input and output:
+ *   grads      host array of nd device fp16 gradient buffers, psi values each
+ *   master, m, v  device fp32, psi values each, updated in place (the caller
+ *              initialises them: m = v = 0 before the first step)
+ *   replicas   host array of nd device fp16 parameter buffers, psi values each
+ *   t          host in/out step count (t-fold bias-correction products; it
+ *              advances by one on a step that is not skipped)
+ * The arithmetic and the result are those of zero_step with
+ * ZERO_VARIANT_TWO_PASS on the same state. Returns ZERO_OK or ZERO_SKIPPED
+ * (nothing changed), ZERO_ERR_ARG when psi > ZERO_STATIC_MAX_PSI or
+ * nd > ZERO_STATIC_MAX_ND (or for any other invalid argument), ZERO_ERR_ALIGN
+ * for a device pointer that is not 16-byte aligned, ZERO_ERR_CUDA otherwise.
+ *
+ * The scratch is one array of 8 KiB + 4 * ZERO_STATIC_MAX_PSI bytes (4 MiB +
+ * 8 KiB); every device that loads it holds it until the process exits. The
+ * first call on a device, with that device current, looks up the array's
+ * device address; make that first call before any stream capture. All calls
+ * on a device share the array and it keeps the last call's contents (the
+ * overflow word is cleared by each call): calls that overlap on the GPU, for
+ * example on two streams, race with each other and must not be issued. The
+ * call synchronises `stream` once to read the overflow word. */
+#define ZERO_STATIC_MAX_PSI 1048576
+#define ZERO_STATIC_MAX_ND 64
+int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* grads, float* master,
+                     float* m, float* v, uint16_t* const* replicas, float loss_scale,
+                     const zero_hyper* hp, int64_t* t, void* stream, int* skipped);
+
 /* The cudaError_t of the last failed CUDA call made through `h` (0 if none). */
 int zero_last_cuda_error(const zero_handle* h);
 

@@ -92,6 +92,9 @@ def lib():
             "zero_current_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                              C.POINTER(C.c_int64)]),
             "zero_stream_copy": (C.c_int, [P, P, C.c_size_t, P]),
+            "zero_step_static": (C.c_int, [C.c_int64, C.c_int32, C.POINTER(P), P, P, P, C.POINTER(P),
+                                           C.c_float, C.POINTER(zero_hyper),
+                                           C.POINTER(C.c_int64), P, C.POINTER(C.c_int)]),
             "zero_last_cuda_error": (C.c_int, [P]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
@@ -200,6 +203,23 @@ def zero_current_state(h: int) -> tuple[int, int, int, int]:
 
 def zero_stream_copy(dst: int, src: int, nbytes: int, stream: int) -> None:
     _check(lib().zero_stream_copy(dst, src, nbytes, stream), "zero_stream_copy")
+
+
+ZERO_STATIC_MAX_PSI = 1048576
+ZERO_STATIC_MAX_ND = 64
+
+
+def zero_step_static(psi: int, grads: Sequence[int], master: int, m: int, v: int,
+                     replicas: Sequence[int], loss_scale: float, hp: zero_hyper, t: int,
+                     stream: int) -> tuple[int, int]:
+    """Allocation-free two-pass step (scratch inside the library).
+    Returns (return code, new t)."""
+    tt = C.c_int64(t)
+    sk = C.c_int(0)
+    rc = _check(lib().zero_step_static(psi, len(grads), _ptr_array(grads), master, m, v,
+                                       _ptr_array(replicas), float(loss_scale), C.byref(hp),
+                                       C.byref(tt), stream, C.byref(sk)), "zero_step_static")
+    return rc, tt.value
 
 
 def zero_destroy(h: int) -> None:

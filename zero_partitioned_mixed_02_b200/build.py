@@ -28,7 +28,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-fmad=false", "-ftz=false",
           "-prec-div=true", "-prec-sqrt=true", "-Xcompiler", "-fPIC,-ffp-contract=off"]
 
-ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu")]
+ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu"),
+                os.path.join(CSRC, "zero_static.cu")]
 ZERO_DEPS = ZERO_SOURCES + [os.path.join(CSRC, "zero_internal.h"), os.path.join(INCLUDE, "zero.h")]
 SYNTH_SOURCES = [os.path.join(SYNTH, "zsynth.cu")]
 SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(SYNTH, "zsynth.h")]
