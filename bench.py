@@ -13,7 +13,7 @@ Prints ONE JSON line (rank 0). ``--impl reference`` times the plain CPU
 oracle on a bounded sample of the same workload instead.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--variant fused|two-pass] [--impl ours|reference]
+                    [--variant fused-tma|fused|two-pass] [--impl ours|reference]
 """
 from __future__ import annotations
 
@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "ZeRO Adam step Gparams/s and HBM GB/s (% of peak) on 1 B200 vs CPU oracle"
 UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "zero_partitioned_mixed_02_b200", "csrc", "zero_kernels.cu")
+CSRC = os.path.join(ROOT, "zero_partitioned_mixed_02_b200", "csrc")
 
 WORKLOADS = {
     "flat-1m": 1, "stress-16m": 2, "gpt2-1.5b": 3, "7.5b-rank-view": 4, "llama-2.7b": 5,
@@ -49,7 +49,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
-    p.add_argument("--variant", choices=["fused", "two-pass"], default="fused")
+    p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass"], default="fused-tma")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -82,7 +82,7 @@ def algorithmic_bytes(wl, variant):
     n_out = wl.nd if (wl.stage <= 2 and wl.rank_view < 0) else 1
     params = 2 * n * n_out                   # fp16 write-back to every replica / the shard
     floor = grads + state + params
-    if variant == "fused":
+    if variant in ("fused", "fused-tma"):
         per_launch = {"step_kernel<fused>": floor}
     else:
         per_launch = {"step_kernel<reduce>": grads + 4 * n,
@@ -103,8 +103,13 @@ def measured_peak():
 
 
 def kernel_sha():
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    """Hash of every device source the step kernels are built from."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
 
 
 def recorded_traffic(wl_name, variant):
@@ -305,7 +310,8 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     wl = workload(args.workload)
-    variant = A.ZERO_VARIANT_FUSED if args.variant == "fused" else A.ZERO_VARIANT_TWO_PASS
+    variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
+               "fused-tma": A.ZERO_VARIANT_FUSED_TMA}[args.variant]
     cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, variant=variant,
                    tensors=wl.tensors)
     L = A.zero_state_bytes(cfg)
@@ -373,7 +379,7 @@ def run_ours(args):
         dist.barrier()
 
     n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant)
-    launches_per_step = (1 if args.variant == "fused" else 2) + len(order)
+    launches_per_step = (2 if args.variant == "two-pass" else 1) + len(order)
     step_s = total_ms / 1e3 / args.steps
     value = world * n / step_s / 1e9
     peak, peak_src = measured_peak()
@@ -382,7 +388,12 @@ def run_ours(args):
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
     traffic = recorded_traffic(args.workload, args.variant)
-    kname = "step_kernel<fused>" if args.variant == "fused" else "step_kernel<reduce>+<update>"
+    if args.variant == "two-pass":
+        kname = "step_kernel<reduce>+<update>"
+    elif A.zero_uses_tma(h):
+        kname = "step_tma_kernel"
+    else:
+        kname = "step_kernel<fused>"
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -59,7 +59,9 @@ extern "C" {
 #define ZERO_ERR_STAGE (-3)     /* call not valid for this stage (gather on stage 1/2) */
 #define ZERO_ERR_WORKSPACE (-4) /* workspace smaller than zero_state_bytes says */
 #define ZERO_ERR_CUDA (-5)      /* a CUDA call failed; see zero_last_cuda_error */
-#define ZERO_ERR_INTERNAL (-6)  /* internal consistency check failed */
+#define ZERO_ERR_INTERNAL (-6)  /* internal consistency check failed, or a bounded
+                                   wait inside a kernel gave up; the step is then
+                                   rolled back like a skipped one */
 
 /* ---- step variants ---- */
 /* One pass: reads the gradients and the current master/m/v, writes the next
@@ -72,6 +74,14 @@ extern "C" {
  * every partition and the overflow flag; the update pass checks the flag and
  * runs Adam in place. One state buffer; 8 more bytes per element. */
 #define ZERO_VARIANT_TWO_PASS 1
+/* The fused pass with its loads and stores done by the Tensor Memory
+ * Accelerator: tiles of the Nd gradient slices and of master/m/v are staged
+ * into shared memory by bulk asynchronous copies while earlier tiles are
+ * computed, and results leave by bulk stores. Same arithmetic, bytes and
+ * workspace as ZERO_VARIANT_FUSED. Used when Nd <= 8 and every run's state
+ * and output indices are in 16-byte phase with its gradient index; otherwise
+ * the handle runs the ZERO_VARIANT_FUSED kernel. */
+#define ZERO_VARIANT_FUSED_TMA 2
 
 #define ZERO_MAX_ND 1024
 
@@ -90,7 +100,7 @@ typedef struct zero_config {
     int32_t stage;     /* ZeRO stage 1, 2 or 3 */
     int32_t rank_view; /* -1: emulate all Nd ranks; r >= 0 (stage 1/2 only):
                           act as rank r alone, owning partition r */
-    int32_t variant;   /* ZERO_VARIANT_FUSED or ZERO_VARIANT_TWO_PASS */
+    int32_t variant;   /* ZERO_VARIANT_FUSED, _TWO_PASS or _FUSED_TMA */
     int32_t n_tensors; /* 0 allowed for stage 1/2 (one flat tensor) */
     int32_t reserved;  /* must be 0 */
     const zero_tensor* tensors; /* host array of n_tensors; sum of numel == psi;
@@ -248,6 +258,10 @@ int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);
 int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* grads, float* master,
                      float* m, float* v, uint16_t* const* replicas, float loss_scale,
                      const zero_hyper* hp, int64_t* t, void* stream, int* skipped);
+
+/* 1 if the handle's steps run the TMA-staged kernel (ZERO_VARIANT_FUSED_TMA
+ * on an eligible configuration), 0 if not, ZERO_ERR_ARG for a NULL handle. */
+int zero_uses_tma(const zero_handle* h);
 
 /* The cudaError_t of the last failed CUDA call made through `h` (0 if none). */
 int zero_last_cuda_error(const zero_handle* h);

@@ -114,13 +114,13 @@ def test_unit_ranges_and_transient():
 
 
 def test_workspace_layout():
-    for variant in (0, 1):
+    for variant in (0, 1, 2):
         for stage in (1, 2, 3):
             tensors = [(1000, 0), (37, 1), (5000, 1)] if stage == 3 else None
             cfg = A.Config(6037, 8, stage, variant=variant, tensors=tensors)
             L = A.zero_state_bytes(cfg)
             offs = [L.off_master[0], L.off_m[0], L.off_v[0]]
-            if variant == 0:
+            if variant in (0, 2):
                 offs += [L.off_master[1], L.off_m[1], L.off_v[1]]
                 assert L.off_reduced == -1
             else:

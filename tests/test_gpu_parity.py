@@ -24,6 +24,8 @@ from gpu_common import (GuardedF16, GuardedWorkspace, SENTINEL16, compare_f16, c
 
 pytestmark = pytest.mark.gpu
 
+VARIANTS = [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA]
+
 if not torch.cuda.is_available():  # collected on CPU machines, never run there
     pytest.skip("needs a GPU", allow_module_level=True)
 
@@ -153,6 +155,9 @@ class Case:
             assert b.guards_intact(), f"param buffer guard band written {tag}"
         assert self.ws.guards_intact(), f"workspace guard band written {tag}"
 
+    def uses_tma(self):
+        return A.zero_uses_tma(self.h)
+
     def close(self):
         A.zero_destroy(self.h)
 
@@ -174,7 +179,7 @@ def _run(case: Case, steps: int, inject=()):
 PSIS = [1, 2, 3, 7, 8, 9, 15, 16, 17, 31, 33, 40, 255, 256, 257, 1000, 4099, 8197, 70001]
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("stage", [1, 2])
 @pytest.mark.parametrize("nd", [1, 2, 3, 4, 5, 8, 9])
 def test_stage12_grid(nd, stage, variant):
@@ -182,7 +187,7 @@ def test_stage12_grid(nd, stage, variant):
         _run(Case(psi, nd, stage, variant, hp=dict(lr=1e-2, weight_decay=0.01 * (psi % 2))), 2)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("nd", [1, 2, 3, 4, 5, 8, 9])
 def test_stage3_grid(nd, variant):
     rng = np.random.default_rng(nd * 10 + variant)
@@ -190,7 +195,7 @@ def test_stage3_grid(nd, variant):
         _run(Case(psi, nd, 3, variant, tensors=_tensor_list(rng, psi)), 2)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_single_rank_view_out_of_phase(variant):
     # partitions whose start is 2, 4 or 6 bytes off a 16-byte boundary in the
     # full parameter buffer, and a trailing rank that is short or empty
@@ -199,7 +204,7 @@ def test_single_rank_view_out_of_phase(variant):
             _run(Case(psi, nd, 1 + r % 2, variant, view=r), 2)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("bits", [0x7C00, 0xFC00, 0x7E00])
 def test_skip_is_global(variant, bits):
     # inf/-inf/NaN on the last rank at an element owned by rank 0, at step 1
@@ -215,7 +220,7 @@ def test_skip_is_global(variant, bits):
         assert skips == [True, False, True]
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_skip_when_unscale_overflows(variant):
     # finite fp16 gradients, but 1/loss_scale pushes their sum past FLT_MAX
     c = Case(300, 2, 2, variant, loss_scale=1e-36, grad_dist=S.normal(1.0, 10000.0))
@@ -236,7 +241,7 @@ def test_rank_order_of_the_sum():
     c.close()
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_zero_gradients_and_non_power_of_two_scale(variant):
     c = Case(4099, 5, 2, variant, loss_scale=3000.0, grad_dist=S.normal(0.0, 1.0))
     _run(c, 2)
@@ -244,7 +249,7 @@ def test_zero_gradients_and_non_power_of_two_scale(variant):
     _run(c, 3)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_workload_flat_1m(variant):
     wl = W.flat_1m()
     c = Case(wl.psi, wl.nd, wl.stage, variant, loss_scale=wl.loss_scale, hp=wl.hyper,
@@ -252,7 +257,7 @@ def test_workload_flat_1m(variant):
     assert _run(c, wl.steps) == [False] * wl.steps
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_workload_precision_stress(variant):
     wl = W.stress_16m()
     c = Case(wl.psi, wl.nd, wl.stage, variant, loss_scale=wl.loss_scale, hp=wl.hyper,
@@ -289,3 +294,34 @@ def test_workload_precision_stress(variant):
     p_after = c.bufs[0].bits()
     assert ((p_after != p_before) & lost).sum() > 0
     c.close()
+
+
+@pytest.mark.parametrize("nd", [1, 2, 3, 4, 8])
+def test_tma_path_runs_and_matches(nd):
+    # sizes with whole tiles, partial tiles, and heads/tails around them; every
+    # partition in 16-byte phase, so the TMA kernel is the one that runs
+    for psi in [64, 1024, 1024 * 3 + 8, 8 * 1024 * 5 + 200, 250_000, 1_000_003]:
+        c = Case(psi, nd, 2, A.ZERO_VARIANT_FUSED_TMA, hp=dict(weight_decay=0.01))
+        assert c.uses_tma()
+        assert _run(c, 2) == [False, False]
+    c = Case(4099, 9, 2, A.ZERO_VARIANT_FUSED_TMA)  # Nd > 8: the plain fused kernel
+    assert not c.uses_tma()
+    _run(c, 1)
+
+
+@pytest.mark.parametrize("nd", [2, 4, 8])
+def test_tma_stage3_eligible_tensors(nd):
+    # tensor sizes that keep every chunk in 16-byte phase: multiples of 8 * nd
+    rng = np.random.default_rng(nd)
+    for trial in range(4):
+        sizes = [int(x) * 8 * nd for x in rng.integers(1, 400, size=6)]
+        units = [0, 0, 1, 1, 1, 2]
+        c = Case(sum(sizes), nd, 3, A.ZERO_VARIANT_FUSED_TMA, tensors=list(zip(sizes, units)))
+        assert c.uses_tma()
+        assert _run(c, 2, inject=[(1, nd - 1, 5, 0x7C00)]) == [False, True]
+
+
+def test_tma_skip_restores_params():
+    c = Case(200_000, 8, 1, A.ZERO_VARIANT_FUSED_TMA)
+    assert c.uses_tma()
+    assert _run(c, 3, inject=[(1, 7, 123_456, 0x7E00)]) == [False, True, False]

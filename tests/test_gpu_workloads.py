@@ -160,16 +160,16 @@ def _run(wl: W.Workload, variant: int):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
 def test_gpt2_1p5b_stage2(variant):
     _run(W.gpt2_1p5b(), variant)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
 def test_running_example_7p5b_rank_view(variant):
     _run(W.running_example_7p5b(), variant)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
 def test_llama_2p7b_stage3(variant):
     _run(W.llama_2p7b(), variant)

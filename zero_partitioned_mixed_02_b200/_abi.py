@@ -25,6 +25,7 @@ ZERO_ERR_INTERNAL = -6
 
 ZERO_VARIANT_FUSED = 0
 ZERO_VARIANT_TWO_PASS = 1
+ZERO_VARIANT_FUSED_TMA = 2
 ZERO_MAX_ND = 1024
 
 
@@ -96,6 +97,7 @@ def lib():
                                            C.c_float, C.POINTER(zero_hyper),
                                            C.POINTER(C.c_int64), P, C.POINTER(C.c_int)]),
             "zero_last_cuda_error": (C.c_int, [P]),
+            "zero_uses_tma": (C.c_int, [P]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
         }
@@ -220,6 +222,10 @@ def zero_step_static(psi: int, grads: Sequence[int], master: int, m: int, v: int
                                        _ptr_array(replicas), float(loss_scale), C.byref(hp),
                                        C.byref(tt), stream, C.byref(sk)), "zero_step_static")
     return rc, tt.value
+
+
+def zero_uses_tma(h: int) -> bool:
+    return _check(lib().zero_uses_tma(h), "zero_uses_tma") == 1
 
 
 def zero_destroy(h: int) -> None:

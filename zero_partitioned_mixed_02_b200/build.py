@@ -29,8 +29,9 @@ COMMON = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-fmad=false", "-f
           "-prec-div=true", "-prec-sqrt=true", "-Xcompiler", "-fPIC,-ffp-contract=off"]
 
 ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu"),
-                os.path.join(CSRC, "zero_static.cu")]
-ZERO_DEPS = ZERO_SOURCES + [os.path.join(CSRC, "zero_internal.h"), os.path.join(INCLUDE, "zero.h")]
+                os.path.join(CSRC, "zero_static.cu"), os.path.join(CSRC, "zero_tma.cu")]
+ZERO_DEPS = ZERO_SOURCES + [os.path.join(CSRC, "zero_internal.h"), os.path.join(CSRC, "zero_device.cuh"),
+                            os.path.join(INCLUDE, "zero.h")]
 SYNTH_SOURCES = [os.path.join(SYNTH, "zsynth.cu")]
 SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(SYNTH, "zsynth.h")]
 

@@ -54,8 +54,12 @@ struct Layout {
     int64_t step_chunks = 0;
     std::vector<zk::SegDesc> gather_segs;
     std::vector<Unit> units;
+    std::vector<zk::TmaRun> tma_runs;  // TMA variant, when every run is eligible
+    bool tma_ok = false;
+    zk::TmaShape tma_shape = zk::kTmaDeep;
+    int64_t tma_tiles = 0, tma_scal = 0;
     int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
-            off_gather_segs = 0, off_reduced = -1, off_shard16 = -1, total = 0;
+            off_gather_segs = 0, off_tma_runs = -1, off_reduced = -1, off_shard16 = -1, total = 0;
     int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
     int64_t transient_elems = 0;
 };
@@ -87,7 +91,9 @@ int build_layout(const zero_config* cfg, Layout* L)
     if (cfg->psi < 1 || cfg->psi > kMaxPsi) return ZERO_ERR_ARG;
     if (cfg->nd < 1 || cfg->nd > ZERO_MAX_ND) return ZERO_ERR_ARG;
     if (cfg->stage < 1 || cfg->stage > 3) return ZERO_ERR_ARG;
-    if (cfg->variant != ZERO_VARIANT_FUSED && cfg->variant != ZERO_VARIANT_TWO_PASS) return ZERO_ERR_ARG;
+    if (cfg->variant != ZERO_VARIANT_FUSED && cfg->variant != ZERO_VARIANT_TWO_PASS &&
+        cfg->variant != ZERO_VARIANT_FUSED_TMA)
+        return ZERO_ERR_ARG;
     if (cfg->reserved != 0 || cfg->n_tensors < 0) return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
     if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
@@ -204,6 +210,34 @@ int build_layout(const zero_config* cfg, Layout* L)
         }
     }
 
+    // ---- TMA run table: the same runs, bodies cut at 8-element multiples ----
+    if (cfg->variant == ZERO_VARIANT_FUSED_TMA && nd <= zk::kTmaMaxNd) {
+        L->tma_shape = zk::tma_shape(L->n_out);
+        bool ok = true;
+        for (const zk::SegDesc& d : L->step_segs)
+            if ((d.state_begin - d.grad_begin) % 4 != 0 || (d.out_begin - d.grad_begin) % 8 != 0) ok = false;
+        if (ok) {
+            for (const zk::SegDesc& d : L->step_segs) {
+                zk::TmaRun t{};
+                t.grad_begin = d.grad_begin;
+                t.state_begin = d.state_begin;
+                t.out_begin = d.out_begin;
+                t.len = d.len;
+                int64_t head = (zk::kLineElems - d.grad_begin % zk::kLineElems) % zk::kLineElems;
+                if (head > d.len) head = d.len;
+                const int64_t body = (d.len - head) / 8 * 8;
+                t.head = (int)head;
+                t.tail = (int)(d.len - head - body);
+                t.tile_begin = L->tma_tiles;
+                t.scal_begin = L->tma_scal;
+                L->tma_tiles += (body + L->tma_shape.tile - 1) / L->tma_shape.tile;
+                L->tma_scal += t.head + t.tail;
+                L->tma_runs.push_back(t);
+            }
+            L->tma_ok = !L->tma_runs.empty();
+        }
+    }
+
     // ---- workspace layout ----
     int64_t off = 0;
     L->off_flag = off;
@@ -216,7 +250,11 @@ int build_layout(const zero_config* cfg, Layout* L)
     off += align_up((int64_t)std::max<size_t>(L->step_segs.size(), 1) * sizeof(zk::SegDesc));
     L->off_gather_segs = off;
     off += align_up((int64_t)L->gather_segs.size() * sizeof(zk::SegDesc));
-    const int n_buf = cfg->variant == ZERO_VARIANT_FUSED ? 2 : 1;
+    if (L->tma_ok) {
+        L->off_tma_runs = off;
+        off += align_up((int64_t)L->tma_runs.size() * sizeof(zk::TmaRun));
+    }
+    const int n_buf = cfg->variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
     for (int b = 0; b < n_buf; ++b)
         for (int k = 0; k < 3; ++k) {
             L->off_state[b][k] = off;
@@ -297,6 +335,9 @@ struct zero_handle {
     int occ[zk::K_COUNT] = {};
     zk::SegDesc* d_step_segs = nullptr;
     zk::SegDesc* d_gather_segs = nullptr;
+    zk::TmaRun* d_tma_runs = nullptr;
+    bool use_tma = false;  // TMA variant and its kernel fits on this device
+    int occ_tma = 0;
     const uint16_t** d_grad_tab = nullptr;
     uint16_t** d_out_tab = nullptr;
     unsigned* d_flag = nullptr;
@@ -306,7 +347,7 @@ struct zero_handle {
     int cur = 0;  // live state buffer (fused variant)
     int64_t t = 0;
     unsigned call_id = 0;
-    unsigned host_flag = 0;
+    unsigned host_flag[2] = {0, 0};  // overflow word, kernel error word
     int last_cuda = 0;
     bool pending = false;  // launched, not yet committed
     int64_t pending_t = 0;
@@ -443,6 +484,16 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     h->d_out_tab = reinterpret_cast<uint16_t**>(h->ws + L.off_out_tab);
     h->d_step_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_step_segs);
     h->d_gather_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_gather_segs);
+    if (L.tma_ok) {
+        h->d_tma_runs = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs);
+        e = zk::tma_prepare(L.tma_shape, L.nd, &h->occ_tma);
+        if (e != cudaSuccess) {
+            rc = cuda_fail(h, e);
+            delete h;
+            return rc;
+        }
+        h->use_tma = h->occ_tma >= 1;
+    }
     if (L.stage <= 2)
         h->out_tab.assign(param_bufs, param_bufs + L.n_out);
     else
@@ -454,6 +505,9 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && !L.step_segs.empty())
         e = cudaMemcpyAsync(h->d_step_segs, L.step_segs.data(), L.step_segs.size() * sizeof(zk::SegDesc),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && L.tma_ok)
+        e = cudaMemcpyAsync(h->d_tma_runs, L.tma_runs.data(), L.tma_runs.size() * sizeof(zk::TmaRun),
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && !L.gather_segs.empty())
         e = cudaMemcpyAsync(h->d_gather_segs, L.gather_segs.data(),
@@ -530,7 +584,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.c.wd = hp->weight_decay;
     bias_corrections(h, hp->beta1, hp->beta2, t_new, &a.c.bc1, &a.c.bc2);
 
-    const bool fused = L.variant == ZERO_VARIANT_FUSED;
+    const bool fused = L.variant != ZERO_VARIANT_TWO_PASS;
     const int nxt = fused ? 1 - h->cur : h->cur;
     a.w_in = h->state(h->cur, 0);
     a.m_in = h->state(h->cur, 1);
@@ -539,7 +593,18 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.m_out = h->state(nxt, 1);
     a.v_out = h->state(nxt, 2);
     if (L.step_chunks > 0) {
-        if (fused) {
+        if (h->use_tma) {
+            zk::TmaArgs ta{};
+            ta.b = a;
+            ta.runs = h->d_tma_runs;
+            ta.n_runs = (int)L.tma_runs.size();
+            ta.n_tiles = L.tma_tiles;
+            ta.n_scal = L.tma_scal;
+            ta.err = h->d_flag + 1;
+            const int64_t cap = (int64_t)h->sms * h->occ_tma;
+            const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
+            e = zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
+        } else if (fused) {
             e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
         } else {
             a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
@@ -563,19 +628,27 @@ ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
     const Layout& L = h->L;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // a copy into pageable host memory returns once the stream has reached it
-    cudaError_t e = cudaMemcpyAsync(&h->host_flag, h->d_flag, sizeof(unsigned),
+    cudaError_t e = cudaMemcpyAsync(h->host_flag, h->d_flag, 2 * sizeof(unsigned),
                                     cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(h, e);
-    if (h->host_flag == h->call_id) {
-        // Overflow: the state buffers do not switch (fused) or were never
-        // written (two-pass). The fused pass already wrote fp16 parameters,
-        // so rewrite them from the unchanged master.
-        if (L.variant == ZERO_VARIANT_FUSED && L.step_chunks > 0) {
+    const bool kernel_error = h->host_flag[1] != 0;
+    if (h->host_flag[0] == h->call_id || kernel_error) {
+        // Overflow (or a kernel that gave up a wait): the state buffers do not
+        // switch (fused) or were never written (two-pass). The fused pass
+        // already wrote fp16 parameters, so rewrite them from the unchanged
+        // master.
+        if (L.variant != ZERO_VARIANT_TWO_PASS && L.step_chunks > 0) {
             zk::StepArgs a = h->args;
             a.w_in = h->state(h->cur, 0);
             e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
             if (e != cudaSuccess) return cuda_fail(h, e);
+        }
+        if (kernel_error) {
+            e = cudaMemsetAsync(h->d_flag + 1, 0, sizeof(unsigned), s);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+            if (e != cudaSuccess) return cuda_fail(h, e);
+            return ZERO_ERR_INTERNAL;
         }
         if (skipped) *skipped = 1;
         return ZERO_SKIPPED;
@@ -636,6 +709,8 @@ ZERO_API int zero_stream_copy(void* dst, const void* src, size_t bytes, void* st
     const cudaError_t e = zk::launch_copy(dst, src, bytes, sms * 8, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA;
 }
+
+ZERO_API int zero_uses_tma(const zero_handle* h) { return h ? (h->use_tma ? 1 : 0) : ZERO_ERR_ARG; }
 
 ZERO_API int zero_last_cuda_error(const zero_handle* h) { return h ? h->last_cuda : 0; }
 

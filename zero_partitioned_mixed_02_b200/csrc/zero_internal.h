@@ -73,6 +73,48 @@ struct GatherArgs {
     uint16_t* dst;
 };
 
+// ---- the TMA-staged fused step ----
+// A run of the TMA path: its body [head, len - tail) starts on a line of the
+// gradient index and is a multiple of 8 elements, cut into tiles of the shape's
+// elements; head and tail elements are scalar items handled from global
+// memory. Every index space is in 16-byte phase with the gradient index.
+struct alignas(16) TmaRun {
+    long long grad_begin;
+    long long state_begin;
+    long long out_begin;
+    long long len;
+    long long tile_begin;  // first tile of the body in the launch's tile numbering
+    long long scal_begin;  // first scalar item in the launch's scalar numbering
+    int head;
+    int tail;
+    int pad[2];
+};
+static_assert(sizeof(TmaRun) == 64, "TmaRun layout");
+
+// Two shapes of the TMA kernel. Stage 1/2 with its Nd replica writes is
+// store-heavy: many consumer warps (one CTA of 32 warps per SM) and a single
+// stage, released as soon as the warps have read it, so the next tile's loads
+// overlap the arithmetic and the stores. Few output streams (stage 3, the rank
+// view): a deeper pipeline of two stages keeps more loads in flight.
+struct TmaShape {
+    int warps;   // consumer warps; one more warp produces
+    int stages;  // input stages
+    int tile;    // elements per tile: one quad per consumer thread
+};
+constexpr TmaShape kTmaWide{31, 1, 31 * 32 * 4};
+constexpr TmaShape kTmaDeep{20, 2, 20 * 32 * 4};
+inline TmaShape tma_shape(int n_out) { return n_out >= 4 ? kTmaWide : kTmaDeep; }
+constexpr int kTmaMaxNd = 8;  // ranks whose tiles fit the stages
+
+struct TmaArgs {
+    StepArgs b;             // pointers, tables, constants, flag (segs unused)
+    const TmaRun* runs;
+    int n_runs;
+    long long n_tiles;
+    long long n_scal;
+    unsigned* err;          // set when a bounded wait gives up
+};
+
 enum Kernel : int {
     K_STEP_FUSED = 0,  // reduce + unscale + flag + Adam into the next buffer + fp16 write-back
     K_REDUCE = 1,      // two-pass, pass 1: reduce + unscale + flag into red
@@ -88,6 +130,10 @@ cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm);
 cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cudaStream_t s);
+// TMA-staged fused step: one-time attribute set-up and blocks per SM for the
+// shape and nd ranks, launch.
+cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);
+cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s);
 int step_smem_bytes(int nd, int n_out);
 
 }  // namespace zk

@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "zero_device.cuh"
 #include "zero_internal.h"
 
 // Minimum resident blocks per SM the step kernels are compiled for (caps
@@ -32,186 +33,6 @@
 
 namespace zk {
 namespace {
-
-__device__ __forceinline__ bool nonfinite(float x)
-{
-    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
-}
-
-__device__ __forceinline__ float h2f(unsigned short b) { return __half2float(__ushort_as_half(b)); }
-
-__device__ __forceinline__ unsigned short f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
-
-// ---- quads: 4 fp16 values packed in a uint2, 4 fp32 values ----
-
-__device__ __forceinline__ void unpack(const uint2 q, float* x)
-{
-    x[0] = h2f((unsigned short)(q.x & 0xffffu));
-    x[1] = h2f((unsigned short)(q.x >> 16));
-    x[2] = h2f((unsigned short)(q.y & 0xffffu));
-    x[3] = h2f((unsigned short)(q.y >> 16));
-}
-
-__device__ __forceinline__ unsigned pack2(float lo, float hi)
-{
-    return (unsigned)f2h(lo) | ((unsigned)f2h(hi) << 16);
-}
-
-__device__ __forceinline__ uint2 pack(const float* x) { return make_uint2(pack2(x[0], x[1]), pack2(x[2], x[3])); }
-
-// 4 fp16 values from p (8-byte aligned: quads start on multiples of 4).
-__device__ __forceinline__ uint2 ld_hq(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
-
-// Store 4 fp16 values with the widest accesses p's alignment allows (the
-// branch is uniform over a run).
-__device__ __forceinline__ void st_hq(uint16_t* p, const uint2 q)
-{
-    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 7u) == 0) {
-        __stcs(reinterpret_cast<uint2*>(p), q);
-    } else if ((a & 3u) == 0) {
-        unsigned* u = reinterpret_cast<unsigned*>(p);
-        __stcs(u, q.x);
-        __stcs(u + 1, q.y);
-    } else {
-        unsigned short* h = reinterpret_cast<unsigned short*>(p);
-        __stcs(h, (unsigned short)(q.x & 0xffffu));
-        __stcs(h + 1, (unsigned short)(q.x >> 16));
-        __stcs(h + 2, (unsigned short)(q.y & 0xffffu));
-        __stcs(h + 3, (unsigned short)(q.y >> 16));
-    }
-}
-
-// 4 fp32 values, widest access the alignment allows.
-__device__ __forceinline__ void ldq(const float* p, float* x)
-{
-    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 15u) == 0) {
-        const float4 t = __ldcs(reinterpret_cast<const float4*>(p));
-        x[0] = t.x;
-        x[1] = t.y;
-        x[2] = t.z;
-        x[3] = t.w;
-    } else if ((a & 7u) == 0) {
-        const float2 t0 = __ldcs(reinterpret_cast<const float2*>(p));
-        const float2 t1 = __ldcs(reinterpret_cast<const float2*>(p) + 1);
-        x[0] = t0.x;
-        x[1] = t0.y;
-        x[2] = t1.x;
-        x[3] = t1.y;
-    } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = __ldcs(p + k);
-    }
-}
-
-__device__ __forceinline__ void stq(float* p, const float* x)
-{
-    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
-    if ((a & 15u) == 0) {
-        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
-    } else if ((a & 7u) == 0) {
-        __stcs(reinterpret_cast<float2*>(p), make_float2(x[0], x[1]));
-        __stcs(reinterpret_cast<float2*>(p) + 1, make_float2(x[2], x[3]));
-    } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) __stcs(p + k, x[k]);
-    }
-}
-
-// A lane's pair of quads: elements [ea, ea + 4) and, if hb, [eb, eb + 4) of
-// the run; values 0..3 belong to the first quad, 4..7 to the second.
-struct Pair {
-    long long ea, eb;
-    bool hb;
-};
-
-__device__ __forceinline__ void ld_pair(const float* base, long long ia, long long ib, bool hb,
-                                        float (&x)[8])
-{
-    ldq(base + ia, x);
-    if (hb)
-        ldq(base + ib, x + 4);
-    else
-        x[4] = x[5] = x[6] = x[7] = 0.0f;
-}
-
-__device__ __forceinline__ void st_pair(float* base, long long ia, long long ib, bool hb,
-                                        const float (&x)[8])
-{
-    stq(base + ia, x);
-    if (hb) stq(base + ib, x + 4);
-}
-
-// ---- the step's arithmetic ----
-
-// Rank-ordered binary32 sum of the Nd fp16 gradients of a lane's two quads.
-// Loads are issued 8 ranks at a time ahead of the additions.
-__device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, long long ga,
-                                            long long gb, bool hb, float (&s)[8])
-{
-    uint2 qa[8], qb[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j < nd) {
-            qa[j] = ld_hq(gp[j] + ga);
-            qb[j] = hb ? ld_hq(gp[j] + gb) : make_uint2(0u, 0u);
-        }
-    }
-    unpack(qa[0], s);
-    unpack(qb[0], s + 4);
-#pragma unroll
-    for (int j = 1; j < 8; ++j) {
-        if (j < nd) {
-            float x[8];
-            unpack(qa[j], x);
-            unpack(qb[j], x + 4);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
-        }
-    }
-    for (int r0 = 8; r0 < nd; r0 += 8) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (r0 + j < nd) {
-                qa[j] = ld_hq(gp[r0 + j] + ga);
-                qb[j] = hb ? ld_hq(gp[r0 + j] + gb) : make_uint2(0u, 0u);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (r0 + j < nd) {
-                float x[8];
-                unpack(qa[j], x);
-                unpack(qb[j], x + 4);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ float reduce1(const uint16_t* const* gp, int nd, long long gi)
-{
-    float s = h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[0] + gi)));
-    for (int r = 1; r < nd; ++r)
-        s = __fadd_rn(s, h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[r] + gi))));
-    return s;
-}
-
-// One element of mixed-precision Adam (bias-corrected, decoupled weight decay
-// scaled by lr), binary32, in the order of the step's definition.
-__device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, const Coef& c)
-{
-    const float m1 = __fadd_rn(__fmul_rn(c.b1, m), __fmul_rn(c.omb1, g));
-    const float v1 = __fadd_rn(__fmul_rn(c.b2, v), __fmul_rn(c.omb2, __fmul_rn(g, g)));
-    const float mh = __fdiv_rn(m1, c.bc1);
-    const float vh = __fdiv_rn(v1, c.bc2);
-    const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), c.eps));
-    w = __fsub_rn(w, __fmul_rn(c.lr, __fadd_rn(u, __fmul_rn(c.wd, w))));
-    m = m1;
-    v = v1;
-}
 
 // ---- per-item bodies of the step kernels ----
 
@@ -264,58 +85,6 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* cons
         st_hq(op[k] + oa, h0);
         if (hb) st_hq(op[k] + ob, h1);
     }
-}
-
-template <int K>
-__device__ __forceinline__ void step_scalar(const StepArgs& a, const uint16_t* const* gp,
-                                            uint16_t* const* op, const SegDesc& d, long long e,
-                                            bool& bad)
-{
-    const long long gi = d.grad_begin + e, si = d.state_begin + e, oi = d.out_begin + e;
-    float w = 0.0f, m = 0.0f, v = 0.0f, g = 0.0f;
-    if (K == K_INIT) {
-        w = __ldcs(a.master_init + gi);
-        __stcs(a.w_out + si, w);
-        __stcs(a.m_out + si, 0.0f);
-        __stcs(a.v_out + si, 0.0f);
-    } else if (K == K_CAST) {
-        w = __ldcs(a.w_in + si);
-    } else {
-        if (K == K_STEP_FUSED || K == K_UPDATE) {
-            w = __ldcs(a.w_in + si);
-            m = __ldcs(a.m_in + si);
-            v = __ldcs(a.v_in + si);
-        }
-        if (K == K_STEP_FUSED || K == K_REDUCE) {
-            g = __fmul_rn(reduce1(gp, a.nd, gi), a.c.inv_scale);
-            bad |= nonfinite(g);
-        }
-        if (K == K_REDUCE) {
-            __stcs(a.red + si, g);
-            return;
-        }
-        if (K == K_UPDATE) g = __ldcs(a.red + si);
-        adam1(g, w, m, v, a.c);
-        __stcs(a.w_out + si, w);
-        __stcs(a.m_out + si, m);
-        __stcs(a.v_out + si, v);
-    }
-    const unsigned short h = f2h(w);
-    for (int k = 0; k < a.n_out; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);
-}
-
-// Largest run index whose first chunk is <= c.
-__device__ __forceinline__ int find_run(const SegDesc* segs, int n, long long c)
-{
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (segs[mid].chunk_begin <= c)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
 }
 
 // Walk the chunks of a run table; call vec(d, pair) for each lane's pair of

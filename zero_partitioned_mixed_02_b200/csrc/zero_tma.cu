@@ -1,0 +1,289 @@
+// The fused step with TMA staging (sm_100a).
+//
+// Persistent CTAs: the last warp is the producer, the others consume. The
+// kernel is instantiated for the two shapes of zero_internal.h (consumer
+// warps x input stages). The producer's lane 0 stages each tile -- the Nd fp16 gradient
+// slices and the fp32 master/m/v of TILE elements -- into one of
+// STAGES shared-memory stages with 1D bulk asynchronous copies
+// (cp.async.bulk; completion counted in bytes on the stage's "full" mbarrier),
+// running up to STAGES tiles ahead of the consumers; a stage is released as
+// soon as every consumer warp has read it, before the arithmetic and stores. Each consumer warp
+// waits for the tile on its own, reduces, unscales, checks and runs Adam on
+// its 32 quads straight out of shared memory, writes the new master/m/v and
+// the fp16 parameters to global memory with streaming stores, and releases the
+// stage with one arrival on its "empty" mbarrier. Warps never wait on each
+// other: there is no CTA-wide barrier after set-up.
+//
+// Every wait is bounded. A warp that gives up sets the error word and leaves
+// its loop (the producer then gives up on that stage too); the producer drains
+// its own copies in flight before it returns. No cluster multicast.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zero_device.cuh"
+#include "zero_internal.h"
+
+namespace zk {
+namespace {
+
+constexpr unsigned kWaitLimit = 1u << 22;  // try_wait rounds (each may suspend ~1 us)
+constexpr int kHdrBytes = 1024;             // barriers and tile descriptors
+
+struct TileDesc {
+    long long gi, si, oi;
+    int n;
+    int pad;
+};
+constexpr int kMaxStages = 8;
+static_assert(16 * kMaxStages + sizeof(TileDesc) * kMaxStages <= kHdrBytes, "header overflow");
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(unsigned bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned bar, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity)
+{
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000u)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity` to complete.
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity)
+{
+    for (unsigned i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(unsigned dst, const void* src, unsigned bytes, unsigned bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Largest index whose begin field is <= x.
+template <long long TmaRun::*F>
+__device__ __forceinline__ int find_tma_run(const TmaRun* runs, int n, long long x)
+{
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (runs[mid].*F <= x)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+template <int WARPS, int STAGES>
+__global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const TmaArgs a)
+{
+    static_assert(STAGES <= kMaxStages, "too many stages");
+    constexpr int kTmaConsumerWarps = WARPS;
+    constexpr int kTmaStages = STAGES;
+    constexpr int kTmaTile = WARPS * 32 * kQuad;
+    extern __shared__ __align__(128) char smem[];
+    const StepArgs& b = a.b;
+    const int nd = b.nd;
+    const unsigned full0 = smem_u32(smem);
+    const unsigned empty0 = full0 + 8 * kTmaStages;
+    TileDesc* desc = reinterpret_cast<TileDesc*>(smem + 16 * kTmaStages);
+    const int stage_bytes = nd * kTmaTile * 2 + 3 * kTmaTile * 4;
+    char* stage0 = smem + kHdrBytes;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);                   // the producer's expect_tx arrival
+            mbar_init(empty0 + 8 * s, kTmaConsumerWarps);  // one arrival per consumer warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == kTmaConsumerWarps) {
+        // ---------------- producer ----------------
+        if (lane != 0) return;
+        int it = 0, r = 0;
+        long long lo = 0, hi = 0;  // tile range of run r
+        for (long long t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
+            const int st = it % kTmaStages;
+            const unsigned ph = (unsigned)(it / kTmaStages) & 1u;
+            if (it >= kTmaStages && !mbar_wait(empty0 + 8 * st, ph ^ 1u)) {
+                atomicOr(a.err, 1u);
+                break;
+            }
+            if (t < lo || t >= hi) {
+                r = find_tma_run<&TmaRun::tile_begin>(a.runs, a.n_runs, t);
+                lo = a.runs[r].tile_begin;
+                hi = (r + 1 < a.n_runs) ? a.runs[r + 1].tile_begin : a.n_tiles;
+            }
+            const TmaRun& run = a.runs[r];
+            const long long body = run.len - run.head - run.tail;
+            const long long e0 = run.head + (t - run.tile_begin) * kTmaTile;
+            const long long rem = run.head + body - e0;
+            const int n = (int)(rem < kTmaTile ? rem : kTmaTile);
+            TileDesc& d = desc[st];
+            d.gi = run.grad_begin + e0;
+            d.si = run.state_begin + e0;
+            d.oi = run.out_begin + e0;
+            d.n = n;
+            char* sp = stage0 + st * stage_bytes;
+            const unsigned full = full0 + 8 * st;
+            mbar_expect_tx(full, (unsigned)n * (unsigned)(2 * nd + 12));
+            for (int k = 0; k < nd; ++k)
+                bulk_g2s(smem_u32(sp + k * kTmaTile * 2), b.grads[k] + d.gi, 2u * n, full);
+            char* sw = sp + nd * kTmaTile * 2;
+            bulk_g2s(smem_u32(sw), b.w_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw + kTmaTile * 4), b.m_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw + 2 * kTmaTile * 4), b.v_in + d.si, 4u * n, full);
+        }
+        // drain: every stage's last armed phase must have landed before exit
+        for (int k = 0; k < kTmaStages && k < it; ++k) {
+            const int i = it - 1 - k;
+            if (!mbar_wait(full0 + 8 * (i % kTmaStages), (unsigned)(i / kTmaStages) & 1u)) atomicOr(a.err, 2u);
+        }
+        return;
+    }
+
+    // ---------------- consumer warps ----------------
+    bool bad = false;
+    const int q4 = (warp * 32 + lane) * kQuad;  // this lane's quad in every tile
+    int it = 0;
+    for (long long t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
+        const int st = it % kTmaStages;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (unsigned)(it / kTmaStages) & 1u));
+        if (!ok) {
+            if (lane == 0) atomicOr(a.err, 4u);
+            break;
+        }
+        const TileDesc d = desc[st];
+        const bool active = q4 < d.n;
+        float g[4], w[4], m[4], v[4];
+        if (active) {
+            const char* sp = stage0 + st * stage_bytes;
+            const uint16_t* sg = reinterpret_cast<const uint16_t*>(sp);
+            const float* sw = reinterpret_cast<const float*>(sp + nd * kTmaTile * 2);
+            float x[4];
+            unpack(*reinterpret_cast<const uint2*>(sg + q4), g);
+            for (int k = 1; k < nd; ++k) {
+                unpack(*reinterpret_cast<const uint2*>(sg + k * kTmaTile + q4), x);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) g[j] = __fadd_rn(g[j], x[j]);
+            }
+            const float4 w4 = *reinterpret_cast<const float4*>(sw + q4);
+            const float4 m4 = *reinterpret_cast<const float4*>(sw + kTmaTile + q4);
+            const float4 v4 = *reinterpret_cast<const float4*>(sw + 2 * kTmaTile + q4);
+            w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
+            m[0] = m4.x; m[1] = m4.y; m[2] = m4.z; m[3] = m4.w;
+            v[0] = v4.x; v[1] = v4.y; v[2] = v4.z; v[3] = v4.w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);  // the warp is done reading the stage
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                g[j] = __fmul_rn(g[j], b.c.inv_scale);
+                bad |= nonfinite(g[j]);
+                adam1(g[j], w[j], m[j], v[j], b.c);
+            }
+            // state indices are 4-element and output indices 8-element aligned
+            // with the gradient index (the host's eligibility rule)
+            __stcs(reinterpret_cast<float4*>(b.w_out + d.si + q4), make_float4(w[0], w[1], w[2], w[3]));
+            __stcs(reinterpret_cast<float4*>(b.m_out + d.si + q4), make_float4(m[0], m[1], m[2], m[3]));
+            __stcs(reinterpret_cast<float4*>(b.v_out + d.si + q4), make_float4(v[0], v[1], v[2], v[3]));
+            const uint2 h = pack(w);
+            for (int k = 0; k < b.n_out; ++k) __stcs(reinterpret_cast<uint2*>(b.outs[k] + d.oi + q4), h);
+        }
+    }
+
+    // scalar items (heads and tails of the runs), straight from global memory
+    constexpr int n_cons_cta = kTmaConsumerWarps * 32;
+    const long long n_cons = (long long)gridDim.x * n_cons_cta;
+    int r = 0;
+    long long lo = 0, hi = 0;
+    for (long long j = (long long)blockIdx.x * n_cons_cta + tid; j < a.n_scal; j += n_cons) {
+        if (j < lo || j >= hi) {
+            r = find_tma_run<&TmaRun::scal_begin>(a.runs, a.n_runs, j);
+            lo = a.runs[r].scal_begin;
+            hi = (r + 1 < a.n_runs) ? a.runs[r + 1].scal_begin : a.n_scal;
+        }
+        const TmaRun& run = a.runs[r];
+        const long long q = j - run.scal_begin;
+        SegDesc sd;
+        sd.grad_begin = run.grad_begin;
+        sd.state_begin = run.state_begin;
+        sd.out_begin = run.out_begin;
+        sd.len = run.len;
+        sd.chunk_begin = 0;
+        sd.head = run.head;
+        sd.tail = run.tail;
+        const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
+        step_scalar<K_STEP_FUSED>(b, b.grads, b.outs, sd, e, bad);
+    }
+
+    // one atomic per consumer warp that saw a non-finite unscaled gradient
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicMax(b.flag, b.call_id);
+}
+
+int smem_bytes(TmaShape sh, int nd) { return kHdrBytes + sh.stages * (nd * sh.tile * 2 + 3 * sh.tile * 4); }
+
+const void* kernel_for(TmaShape sh)
+{
+    if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages)
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaWide.warps, kTmaWide.stages>);
+    if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages)
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages>);
+    return nullptr;
+}
+
+}  // namespace
+
+cudaError_t tma_prepare(TmaShape sh, int nd, int* blocks_per_sm)
+{
+    const void* f = kernel_for(sh);
+    if (!f) return cudaErrorInvalidValue;
+    const int smem = smem_bytes(sh, nd);
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, f, (sh.warps + 1) * 32, smem);
+}
+
+cudaError_t launch_step_tma(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s)
+{
+    const int smem = smem_bytes(sh, a.b.nd);
+    if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages)
+        step_tma_kernel<kTmaWide.warps, kTmaWide.stages><<<grid, (sh.warps + 1) * 32, smem, s>>>(a);
+    else if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages)
+        step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages><<<grid, (sh.warps + 1) * 32, smem, s>>>(a);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace zk
