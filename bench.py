@@ -177,6 +177,25 @@ def cpu_info():
     return model, os.cpu_count()
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device: str) -> float:
+    """The largest x over all ranks (the device time of the slowest rank);
+    x itself without a multi-rank process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(elements_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Gparams/s of the whole job: every rank updates elements_per_rank per
+    step (weak scaling), timed by the slowest rank."""
+    return world * elements_per_rank * steps / (max_ms / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------- oracle leg
 def oracle_sample_step(wl, n_s, step, state):
     """One oracle step over the first n_s owned elements of the workload (the
@@ -370,18 +389,15 @@ def run_ours(args):
     t1.record(stream)
     torch.cuda.synchronize()
     clock_info = clocks.stop() if clocks else None
-    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
     kern_ms = [a.elapsed_time(b) for a, b in kernel_events]
     if world > 1:
-        tt = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
         dist.barrier()
 
     n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant)
     launches_per_step = (2 if args.variant == "two-pass" else 1) + len(order)
     step_s = total_ms / 1e3 / args.steps
-    value = world * n / step_s / 1e9
+    value = whole_job_value(n, args.steps, world, total_ms)
     peak, peak_src = measured_peak()
     # dominant kernel: the step kernel (both kernels of the two-pass variant timed together)
     k_s = statistics.mean(kern_ms) / 1e3
@@ -466,13 +482,9 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
         step()
     b.record(s)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(a.elapsed_time(b), "cuda")
     n = L.state_elems
-    return {"value": world * n * args.e2e_steps / (ms / 1e3) / 1e9, "unit": UNIT,
+    return {"value": whole_job_value(n, args.e2e_steps, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": len(grads) * n_own * 2, "d2h_bytes_per_step": result.numel() * 2,
             "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
 

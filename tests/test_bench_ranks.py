@@ -1,0 +1,60 @@
+"""The benchmark's multi-rank logic on CPU: two gloo ranks (world size 2)
+take the device time of the slowest rank and report the whole job's
+throughput; without a process group the same helpers are identities."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, out):
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        ms = bench.max_over_ranks(times[rank], "cpu")
+        value = bench.whole_job_value(1_000_000, 10, world, ms)
+        out.put((rank, ms, value))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_max_over_ranks_and_value_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    times = [100.0, 150.0]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, times, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, ms, value in got:
+        assert ms == 150.0  # every rank sees the slowest rank's time
+        assert value == pytest.approx(world * 1_000_000 * 10 / 0.150 / 1e9)
+
+
+def test_single_process_identity():
+    assert bench.max_over_ranks(12.5, "cpu") == 12.5
+    assert bench.whole_job_value(2_000_000_000, 4, 1, 1000.0) == pytest.approx(8.0)
+
+
+def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    class A:  # the arguments run_reference reads
+        workload, steps, warmup, gpus, variant = "flat-1m", 1, 0, 2, "fused-tma"
+    bench.run_reference(A)
+    assert capsys.readouterr().out == ""
