@@ -359,6 +359,7 @@ def run_ours(args):
     order = (list(range(L.n_units)) + list(reversed(range(L.n_units)))) if wl.stage == 3 else []
 
     kernel_events = []
+    gather_events = []
 
     def one_step(timed):
         if timed:
@@ -371,8 +372,15 @@ def run_ours(args):
         rc = A.zero_step_commit(h, s)
         if rc != A.ZERO_OK:
             raise RuntimeError("unexpected skip in the benchmark workload")
-        for u in order:
-            A.zero_gather_layer(h, u, gather_out.data_ptr(), s)
+        if order:
+            if timed:
+                c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                c.record(stream)
+            for u in order:
+                A.zero_gather_layer(h, u, gather_out.data_ptr(), s)
+            if timed:
+                d.record(stream)
+                gather_events.append((c, d))
 
     for _ in range(args.warmup):
         one_step(False)
@@ -424,6 +432,11 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
     }
+    if gather_events:
+        g_ms = statistics.mean(a.elapsed_time(b) for a, b in gather_events)
+        line["gathers"] = {"per_step_ms": g_ms, "launches_per_step": len(order),
+                           "bytes_per_step": gathers, "achieved_gbs": gathers / (g_ms / 1e3) / 1e9,
+                           "frac": gathers / (g_ms / 1e3) / 1e9 / peak}
 
     # ---- end to end through the public API from pinned host buffers ----
     if not args.no_e2e and args.e2e_steps > 0:

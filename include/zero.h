@@ -80,7 +80,10 @@ extern "C" {
  * computed, and results leave by bulk stores. Same arithmetic, bytes and
  * workspace as ZERO_VARIANT_FUSED. Used when Nd <= 8 and every run's state
  * and output indices are in 16-byte phase with its gradient index; otherwise
- * the handle runs the ZERO_VARIANT_FUSED kernel. */
+ * the handle runs the ZERO_VARIANT_FUSED kernel. Its stage-3 layer gathers
+ * copy through shared memory with bulk copies too (for units whose chunks are
+ * in 16-byte phase with their place in the output); a gather whose bounded
+ * wait gave up is reported by the next zero_step as ZERO_ERR_INTERNAL. */
 #define ZERO_VARIANT_FUSED_TMA 2
 
 #define ZERO_MAX_ND 1024

@@ -38,6 +38,11 @@ struct Unit {
     int64_t n_chunks = 0;
     int64_t flat_begin = 0;
     int64_t numel = 0;
+    bool tma_ok = false;  // bulk-copy gather table built (TMA variant, runs in 16-byte phase)
+    int64_t tma_run0 = 0;
+    int64_t tma_n_runs = 0;
+    int64_t tma_tiles = 0;
+    int64_t tma_scal = 0;
 };
 
 // Everything that follows from a configuration: partitions, run tables,
@@ -53,13 +58,15 @@ struct Layout {
     std::vector<zk::SegDesc> step_segs;
     int64_t step_chunks = 0;
     std::vector<zk::SegDesc> gather_segs;
+    std::vector<zk::TmaRun> tma_gather;  // TMA variant: bulk-copy gather runs of all units
     std::vector<Unit> units;
     std::vector<zk::TmaRun> tma_runs;  // TMA variant, when every run is eligible
     bool tma_ok = false;
     zk::TmaShape tma_shape = zk::kTmaDeep;
     int64_t tma_tiles = 0, tma_scal = 0;
     int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
-            off_gather_segs = 0, off_tma_runs = -1, off_reduced = -1, off_shard16 = -1, total = 0;
+            off_gather_segs = 0, off_tma_runs = -1, off_tma_gather = -1, off_reduced = -1, off_shard16 = -1,
+            total = 0;
     int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
     int64_t transient_elems = 0;
 };
@@ -207,6 +214,35 @@ int build_layout(const zero_config* cfg, Layout* L)
             U.n_segs = (int64_t)L->gather_segs.size() - U.seg0;
             U.n_chunks = chunks;
             L->transient_elems = std::max(L->transient_elems, U.numel);
+            if (cfg->variant == ZERO_VARIANT_FUSED_TMA) {
+                bool ok = U.n_segs > 0;
+                for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
+                    const zk::SegDesc& g = L->gather_segs[i];
+                    if ((g.out_begin - g.grad_begin) % 8 != 0) ok = false;
+                }
+                if (ok) {
+                    U.tma_ok = true;
+                    U.tma_run0 = (int64_t)L->tma_gather.size();
+                    for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
+                        const zk::SegDesc& g = L->gather_segs[i];
+                        zk::TmaRun t{};
+                        t.grad_begin = g.grad_begin;
+                        t.out_begin = g.out_begin;
+                        t.len = g.len;
+                        int64_t head = (zk::kLineElems - g.grad_begin % zk::kLineElems) % zk::kLineElems;
+                        if (head > g.len) head = g.len;
+                        const int64_t body = (g.len - head) / 8 * 8;
+                        t.head = (int)head;
+                        t.tail = (int)(g.len - head - body);
+                        t.tile_begin = U.tma_tiles;
+                        t.scal_begin = U.tma_scal;
+                        U.tma_tiles += (body + zk::kGatherTile - 1) / zk::kGatherTile;
+                        U.tma_scal += t.head + t.tail;
+                        L->tma_gather.push_back(t);
+                    }
+                    U.tma_n_runs = (int64_t)L->tma_gather.size() - U.tma_run0;
+                }
+            }
         }
     }
 
@@ -253,6 +289,10 @@ int build_layout(const zero_config* cfg, Layout* L)
     if (L->tma_ok) {
         L->off_tma_runs = off;
         off += align_up((int64_t)L->tma_runs.size() * sizeof(zk::TmaRun));
+    }
+    if (!L->tma_gather.empty()) {
+        L->off_tma_gather = off;
+        off += align_up((int64_t)L->tma_gather.size() * sizeof(zk::TmaRun));
     }
     const int n_buf = cfg->variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
     for (int b = 0; b < n_buf; ++b)
@@ -338,6 +378,8 @@ struct zero_handle {
     zk::TmaRun* d_tma_runs = nullptr;
     bool use_tma = false;  // TMA variant and its kernel fits on this device
     int occ_tma = 0;
+    zk::TmaRun* d_tma_gather = nullptr;
+    int occ_gather_tma = 0;
     const uint16_t** d_grad_tab = nullptr;
     uint16_t** d_out_tab = nullptr;
     unsigned* d_flag = nullptr;
@@ -494,6 +536,15 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
         }
         h->use_tma = h->occ_tma >= 1;
     }
+    if (!L.tma_gather.empty()) {
+        h->d_tma_gather = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_gather);
+        e = zk::tma_gather_prepare(&h->occ_gather_tma);
+        if (e != cudaSuccess) {
+            rc = cuda_fail(h, e);
+            delete h;
+            return rc;
+        }
+    }
     if (L.stage <= 2)
         h->out_tab.assign(param_bufs, param_bufs + L.n_out);
     else
@@ -508,6 +559,9 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && L.tma_ok)
         e = cudaMemcpyAsync(h->d_tma_runs, L.tma_runs.data(), L.tma_runs.size() * sizeof(zk::TmaRun),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !L.tma_gather.empty())
+        e = cudaMemcpyAsync(h->d_tma_gather, L.tma_gather.data(), L.tma_gather.size() * sizeof(zk::TmaRun),
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && !L.gather_segs.empty())
         e = cudaMemcpyAsync(h->d_gather_segs, L.gather_segs.data(),
@@ -676,6 +730,20 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     if (!aligned16(out)) return ZERO_ERR_ALIGN;
     const Unit& U = L.units[unit];
     if (U.n_chunks == 0) return ZERO_OK;
+    if (U.tma_ok && h->occ_gather_tma >= 1) {
+        zk::TmaGatherArgs g{};
+        g.runs = h->d_tma_gather + U.tma_run0;
+        g.n_runs = (int)U.tma_n_runs;
+        g.n_tiles = U.tma_tiles;
+        g.n_scal = U.tma_scal;
+        g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
+        g.dst = out;
+        g.err = h->d_flag + 1;
+        const int64_t want = std::max<int64_t>(1, std::max(U.tma_tiles, (U.tma_scal + 31) / 32));
+        const int64_t cap = (int64_t)h->sms * h->occ_gather_tma;
+        const cudaError_t e = zk::launch_gather_tma(g, (int)std::min(want, cap), static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+    }
     zk::GatherArgs g{};
     g.segs = h->d_gather_segs + U.seg0;
     g.n_segs = (int)U.n_segs;

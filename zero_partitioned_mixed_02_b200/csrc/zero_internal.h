@@ -115,6 +115,23 @@ struct TmaArgs {
     unsigned* err;          // set when a bounded wait gives up
 };
 
+// The stage-3 layer gather with bulk copies: each run (one rank's chunk of one
+// tensor) is copied shard -> output through shared memory in tiles of
+// kGatherTile elements, kGatherStages tiles in flight per CTA. TmaRun fields:
+// grad_begin = source (shard) index, out_begin = destination index.
+constexpr int kGatherTile = 8192;
+constexpr int kGatherStages = 4;
+
+struct TmaGatherArgs {
+    const TmaRun* runs;
+    int n_runs;
+    long long n_tiles;
+    long long n_scal;
+    const uint16_t* src;
+    uint16_t* dst;
+    unsigned* err;
+};
+
 enum Kernel : int {
     K_STEP_FUSED = 0,  // reduce + unscale + flag + Adam into the next buffer + fp16 write-back
     K_REDUCE = 1,      // two-pass, pass 1: reduce + unscale + flag into red
@@ -134,6 +151,8 @@ cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cuda
 // shape and nd ranks, launch.
 cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);
 cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s);
+cudaError_t tma_gather_prepare(int* blocks_per_sm);
+cudaError_t launch_gather_tma(const TmaGatherArgs& a, int grid, cudaStream_t s);
 int step_smem_bytes(int nd, int n_out);
 
 }  // namespace zk
