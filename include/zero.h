@@ -266,6 +266,16 @@ int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* grads, floa
  * on an eligible configuration), 0 if not, ZERO_ERR_ARG for a NULL handle. */
 int zero_uses_tma(const zero_handle* h);
 
+/* Test hook for the bounded waits of the TMA kernels, which fail without any
+ * GPU fault: the next TMA step or TMA layer gather on this handle leaves its
+ * tile number `tile` unarmed, so the waits on it give up after `wait_rounds`
+ * try_wait rounds (each suspends about a microsecond). The kernel sets its
+ * error word and drains its own copies; the step is rolled back like a
+ * skipped one and returns ZERO_ERR_INTERNAL (a gather's failure is reported,
+ * and its step rolled back, by the next zero_step). The hook applies once.
+ * Has no effect on handles that do not run the TMA kernels. */
+int zero_test_hold_tile(zero_handle* h, int64_t tile, uint32_t wait_rounds);
+
 /* The cudaError_t of the last failed CUDA call made through `h` (0 if none). */
 int zero_last_cuda_error(const zero_handle* h);
 

@@ -325,3 +325,51 @@ def test_tma_skip_restores_params():
     c = Case(200_000, 8, 1, A.ZERO_VARIANT_FUSED_TMA)
     assert c.uses_tma()
     assert _run(c, 3, inject=[(1, 7, 123_456, 0x7E00)]) == [False, True, False]
+
+
+def test_tma_wait_that_gives_up_is_reported_and_rolled_back():
+    # A tile left unarmed makes the kernel's bounded waits run out (no fault):
+    # the step returns ZERO_ERR_INTERNAL, nothing changes, and the next step
+    # is exactly the oracle's next step.
+    for psi, nd, stage in [(200_000, 8, 1), (50_000, 2, 2)]:
+        c = Case(psi, nd, stage, A.ZERO_VARIANT_FUSED_TMA)
+        assert c.uses_tma()
+        c.check("after init")
+        c.step(c.grads(0))
+        c.check("after step 0")
+        A.zero_test_hold_tile(c.h, 3, 1 << 14)
+        n = c.e0 - c.b0
+        gs = c.grads(1)
+        for k in range(c.nd):
+            c.g_dev[k][:n].copy_(torch.from_numpy(gs[k].view(np.int16)))
+        with pytest.raises(A.ZeroError) as ei:
+            A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], c.loss_scale, hyper(), c.stream)
+        assert ei.value.code == A.ZERO_ERR_INTERNAL
+        c.check("after the failed step: unchanged")
+        assert c.step(c.grads(2)) is False
+        c.check("after the next step")
+        c.close()
+
+
+def test_tma_gather_wait_that_gives_up_is_reported():
+    nd = 4
+    sizes = [8 * nd * 700, 8 * nd * 300, 8 * nd * 1200]
+    c = Case(sum(sizes), nd, 3, A.ZERO_VARIANT_FUSED_TMA, tensors=list(zip(sizes, [0, 1, 1])))
+    assert c.uses_tma()
+    c.step(c.grads(0))
+    c.check("after step 0")
+    A.zero_test_hold_tile(c.h, 0, 1 << 14)
+    fb, cnt = A.zero_unit_range(c.cfg, 1)
+    out = GuardedF16(cnt)
+    A.zero_gather_layer(c.h, 1, out.ptr(), c.stream)  # its failure shows at the next step
+    n = c.e0 - c.b0
+    gs = c.grads(1)
+    for k in range(c.nd):
+        c.g_dev[k][:n].copy_(torch.from_numpy(gs[k].view(np.int16)))
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], c.loss_scale, hyper(), c.stream)
+    assert ei.value.code == A.ZERO_ERR_INTERNAL
+    c.check("after the reported failure: unchanged")  # gathers re-checked inside
+    assert c.step(c.grads(2)) is False
+    c.check("after the next step")
+    c.close()

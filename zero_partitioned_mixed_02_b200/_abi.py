@@ -98,6 +98,7 @@ def lib():
                                            C.POINTER(C.c_int64), P, C.POINTER(C.c_int)]),
             "zero_last_cuda_error": (C.c_int, [P]),
             "zero_uses_tma": (C.c_int, [P]),
+            "zero_test_hold_tile": (C.c_int, [P, C.c_int64, C.c_uint32]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
         }
@@ -222,6 +223,10 @@ def zero_step_static(psi: int, grads: Sequence[int], master: int, m: int, v: int
                                        _ptr_array(replicas), float(loss_scale), C.byref(hp),
                                        C.byref(tt), stream, C.byref(sk)), "zero_step_static")
     return rc, tt.value
+
+
+def zero_test_hold_tile(h: int, tile: int, wait_rounds: int) -> None:
+    _check(lib().zero_test_hold_tile(h, tile, wait_rounds), "zero_test_hold_tile")
 
 
 def zero_uses_tma(h: int) -> bool:

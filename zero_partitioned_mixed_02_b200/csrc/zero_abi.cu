@@ -380,6 +380,8 @@ struct zero_handle {
     int occ_tma = 0;
     zk::TmaRun* d_tma_gather = nullptr;
     int occ_gather_tma = 0;
+    int64_t hold_tile = -1;  // test hook for the bounded waits (zero_test_hold_tile)
+    unsigned hold_rounds = 0;
     const uint16_t** d_grad_tab = nullptr;
     uint16_t** d_out_tab = nullptr;
     unsigned* d_flag = nullptr;
@@ -655,6 +657,9 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
             ta.n_tiles = L.tma_tiles;
             ta.n_scal = L.tma_scal;
             ta.err = h->d_flag + 1;
+            ta.wait_rounds = h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds;
+            ta.hold_tile = h->hold_tile;
+            h->hold_tile = -1;
             const int64_t cap = (int64_t)h->sms * h->occ_tma;
             const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
             e = zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
@@ -739,6 +744,9 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
         g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
         g.dst = out;
         g.err = h->d_flag + 1;
+        g.wait_rounds = h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds;
+        g.hold_tile = h->hold_tile;
+        h->hold_tile = -1;
         const int64_t want = std::max<int64_t>(1, std::max(U.tma_tiles, (U.tma_scal + 31) / 32));
         const int64_t cap = (int64_t)h->sms * h->occ_gather_tma;
         const cudaError_t e = zk::launch_gather_tma(g, (int)std::min(want, cap), static_cast<cudaStream_t>(stream));
@@ -776,6 +784,14 @@ ZERO_API int zero_stream_copy(void* dst, const void* src, size_t bytes, void* st
         return ZERO_ERR_CUDA;
     const cudaError_t e = zk::launch_copy(dst, src, bytes, sms * 8, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA;
+}
+
+ZERO_API int zero_test_hold_tile(zero_handle* h, int64_t tile, uint32_t wait_rounds)
+{
+    if (!h || tile < 0 || wait_rounds == 0) return ZERO_ERR_ARG;
+    h->hold_tile = tile;
+    h->hold_rounds = wait_rounds;
+    return ZERO_OK;
 }
 
 ZERO_API int zero_uses_tma(const zero_handle* h) { return h ? (h->use_tma ? 1 : 0) : ZERO_ERR_ARG; }

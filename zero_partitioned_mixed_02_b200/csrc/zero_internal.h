@@ -113,6 +113,8 @@ struct TmaArgs {
     long long n_tiles;
     long long n_scal;
     unsigned* err;          // set when a bounded wait gives up
+    unsigned wait_rounds;   // try_wait rounds before a wait gives up
+    long long hold_tile;    // test hook: this tile is never armed (-1: none)
 };
 
 // The stage-3 layer gather with bulk copies: each run (one rank's chunk of one
@@ -130,7 +132,13 @@ struct TmaGatherArgs {
     const uint16_t* src;
     uint16_t* dst;
     unsigned* err;
+    unsigned wait_rounds;
+    long long hold_tile;
 };
+
+// try_wait rounds (each may suspend about a microsecond) before a wait of the
+// TMA kernels gives up: a few seconds, far beyond any legitimate wait.
+constexpr unsigned kTmaWaitRounds = 1u << 22;
 
 enum Kernel : int {
     K_STEP_FUSED = 0,  // reduce + unscale + flag + Adam into the next buffer + fp16 write-back

@@ -27,7 +27,6 @@
 namespace zk {
 namespace {
 
-constexpr unsigned kWaitLimit = 1u << 22;  // try_wait rounds (each may suspend ~1 us)
 constexpr int kHdrBytes = 1024;             // barriers and tile descriptors
 
 struct TileDesc {
@@ -69,9 +68,9 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity)
 }
 
 // Bounded wait for the phase of parity `parity` to complete.
-__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity)
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, unsigned rounds)
 {
-    for (unsigned i = 0; i < kWaitLimit; ++i)
+    for (unsigned i = 0; i < rounds; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
@@ -134,7 +133,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         for (long long t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
             const int st = it % kTmaStages;
             const unsigned ph = (unsigned)(it / kTmaStages) & 1u;
-            if (it >= kTmaStages && !mbar_wait(empty0 + 8 * st, ph ^ 1u)) {
+            if (it >= kTmaStages && !mbar_wait(empty0 + 8 * st, ph ^ 1u, a.wait_rounds)) {
                 atomicOr(a.err, 1u);
                 break;
             }
@@ -148,6 +147,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
             const long long e0 = run.head + (t - run.tile_begin) * kTmaTile;
             const long long rem = run.head + body - e0;
             const int n = (int)(rem < kTmaTile ? rem : kTmaTile);
+            if (t == a.hold_tile) continue;  // test hook: leave this stage unarmed
             TileDesc& d = desc[st];
             d.gi = run.grad_begin + e0;
             d.si = run.state_begin + e0;
@@ -166,7 +166,8 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         // drain: every stage's last armed phase must have landed before exit
         for (int k = 0; k < kTmaStages && k < it; ++k) {
             const int i = it - 1 - k;
-            if (!mbar_wait(full0 + 8 * (i % kTmaStages), (unsigned)(i / kTmaStages) & 1u)) atomicOr(a.err, 2u);
+            if (!mbar_wait(full0 + 8 * (i % kTmaStages), (unsigned)(i / kTmaStages) & 1u, a.wait_rounds))
+                atomicOr(a.err, 2u);
         }
         return;
     }
@@ -177,7 +178,8 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
     int it = 0;
     for (long long t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
         const int st = it % kTmaStages;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (unsigned)(it / kTmaStages) & 1u));
+        const bool ok =
+            __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (unsigned)(it / kTmaStages) & 1u, a.wait_rounds));
         if (!ok) {
             if (lane == 0) atomicOr(a.err, 4u);
             break;
@@ -309,12 +311,14 @@ __global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
                 tiles[st].d = run.out_begin + e0;
                 tiles[st].bytes = 2u * n;
                 const unsigned full = full0 + 8 * st;
-                mbar_expect_tx(full, 2u * n);
-                bulk_g2s(smem_u32(stage0 + st * kGatherTile * 2), a.src + tiles[st].s, 2u * n, full);
+                if (t != a.hold_tile) {  // test hook: leave this stage unarmed
+                    mbar_expect_tx(full, 2u * n);
+                    bulk_g2s(smem_u32(stage0 + st * kGatherTile * 2), a.src + tiles[st].s, 2u * n, full);
+                }
                 ++issued;
             }
             const int st = (int)(i % S);
-            if (!mbar_wait(full0 + 8 * st, (unsigned)(i / S) & 1u)) {
+            if (!mbar_wait(full0 + 8 * st, (unsigned)(i / S) & 1u, a.wait_rounds)) {
                 atomicOr(a.err, 8u);
                 failed = true;
                 break;
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
         }
         // drain: issued loads must land, issued stores must finish, before exit
         for (long long i = issued - 1; i >= 0 && i >= issued - S; --i)
-            if (!mbar_wait(full0 + 8 * (int)(i % S), (unsigned)(i / S) & 1u)) atomicOr(a.err, 16u);
+            if (!mbar_wait(full0 + 8 * (int)(i % S), (unsigned)(i / S) & 1u, a.wait_rounds)) atomicOr(a.err, 16u);
         bulk_wait_all();
     }
     __syncwarp();
