@@ -334,6 +334,27 @@ int64_t zr_zero3_gather(int32_t n_tensors, const int64_t* numel, const int32_t* 
 }
 
 /* ======================================================================
+ * Dynamic loss scaling: multiplicative back-off on overflow, growth after a
+ * run of good steps.
+ * ==================================================================== */
+
+void zr_scaler_update(float* scale, int32_t* good, int overflow, float growth, float backoff,
+                      int32_t interval)
+{
+    if (overflow) {
+        *scale = *scale * backoff;
+        *good = 0;
+        return;
+    }
+    *good = *good + 1;
+    if (*good >= interval) {
+        const float grown = *scale * growth;
+        if (isfinite(grown)) *scale = grown;
+        *good = 0;
+    }
+}
+
+/* ======================================================================
  * Ledger.  [P1] "Where 16 bytes per parameter comes from" (2 + 2 + K, K = 12)
  * and the stage table in "The replication nobody questioned"; [P2] "The
  * Mathematics", M_states(p, Nd); [P3] "What each ZeRO stage partitions".

@@ -95,6 +95,13 @@ int64_t zr_zero3_gather(int32_t n_tensors, const int64_t* numel, const int32_t* 
                         int32_t nd, int32_t unit, const uint16_t* const* p_sh,
                         uint16_t* out);
 
+/* ---- dynamic loss scaling (not on the pages; the usual reading) ----
+ * After a skipped (overflowing) step the scale is multiplied by `backoff` and
+ * the run of good steps restarts; after `interval` consecutive good steps it
+ * is multiplied by `growth` (kept if that would overflow binary32). */
+void zr_scaler_update(float* scale, int32_t* good, int overflow, float growth, float backoff,
+                      int32_t interval);
+
 /* ---- memory and communication ledger ---- */
 /* Per-rank model-state bytes from the pages' formulas:
  * out = {16 psi, 4 psi + 12 psi/nd, 2 psi + 14 psi/nd, 16 psi/nd}. */

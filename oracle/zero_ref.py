@@ -55,6 +55,7 @@ _z3_gather = _sig("zr_zero3_gather", _i64, _i32, _p, _p, _i32, _i32, _pp, _p)
 _formula = _sig("zr_ledger_formula", None, C.c_double, C.c_double, C.POINTER(C.c_double))
 _exact = _sig("zr_ledger_exact", None, _i64, _i32, _i32, _p, C.POINTER(_i64))
 _comm = _sig("zr_comm_elements", None, _i64, _i32, C.POINTER(_i64))
+_scaler = _sig("zr_scaler_update", None, C.POINTER(_f32), C.POINTER(_i32), C.c_int, _f32, _f32, _i32)
 
 
 def _ptr(a: np.ndarray) -> int:
@@ -194,3 +195,10 @@ def comm_elements(psi: int, nd: int) -> dict:
     _comm(psi, nd, out)
     keys = ["reduce_scatter", "all_gather", "dp", "stage1", "stage2", "stage3"]
     return dict(zip(keys, out[:]))
+
+
+def scaler_update(scale: float, good: int, overflow: bool, growth: float, backoff: float,
+                  interval: int) -> tuple[float, int]:
+    sc, g = _f32(scale), _i32(good)
+    _scaler(C.byref(sc), C.byref(g), int(overflow), growth, backoff, interval)
+    return float(np.float32(sc.value)), g.value
