@@ -209,6 +209,46 @@ int zero_step_launch(zero_handle* h, const uint16_t* const* grads, float loss_sc
                      const zero_hyper* hp, void* stream);
 int zero_step_commit(zero_handle* h, void* stream, int* skipped);
 
+/* ---- asynchronous steps ([P1]-[P3] do not cover loss scaling; the usual
+ * dynamic loss scaling is the reading) ----
+ * Between zero_async_begin and zero_async_end the step count, the bias-
+ * correction products, the live state buffer and a dynamic loss scale live on
+ * the device, and zero_step_async only enqueues work: it reads nothing back
+ * and calls nothing that synchronises, so a caller can issue steps back to
+ * back or capture one in a CUDA graph and replay it. Each step computes what
+ * zero_step computes with the current loss scale; then, on the device, an
+ * overflowing step is rolled back (as with ZERO_SKIPPED) and the scale is
+ * multiplied by backoff_factor, while a good step commits and, after
+ * growth_interval good steps in a row, multiplies the scale by growth_factor
+ * (kept if that would overflow binary32). */
+typedef struct zero_scaler {
+    float init_scale;        /* > 0 and finite */
+    float growth_factor;     /* >= 1 */
+    float backoff_factor;    /* in (0, 1] */
+    int32_t growth_interval; /* >= 1 */
+} zero_scaler;
+
+typedef struct zero_async_state {
+    int64_t t;          /* steps committed (all time) */
+    int64_t skipped;    /* steps skipped during this run */
+    float loss_scale;   /* the scale the next step would use */
+    int32_t good_steps; /* good steps since the last growth or back-off */
+} zero_async_state;
+
+/* Open an asynchronous run: grads (host array of Nd device pointers, as for
+ * zero_step) are bound for the whole run -- refill the same buffers between
+ * steps -- and beta1/beta2 are fixed. Synchronises `stream` once. Every later
+ * zero_step_async must pass the same betas. zero_step, zero_step_launch and
+ * zero_current_state return ZERO_ERR_ARG until zero_async_end. */
+int zero_async_begin(zero_handle* h, const uint16_t* const* grads, const zero_scaler* sc,
+                     float beta1, float beta2, void* stream);
+/* Enqueue one step (no host synchronisation, no host-side reads). */
+int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream);
+/* Close the run: synchronise `stream`, return the device-side counters and
+ * hand t and the live buffer back to the host. Returns ZERO_ERR_INTERNAL if a
+ * kernel gave up a bounded wait during the run (those steps were skipped). */
+int zero_async_end(zero_handle* h, void* stream, zero_async_state* out);
+
 /* Stage 3: write layer unit `unit`'s full fp16 weights into `out` (device,
  * >= the numel zero_unit_range reports): its tensors in tensor order, each whole
  * and contiguous, back to back. Call it per unit in forward order and again in
@@ -218,7 +258,7 @@ int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
 
 /* Current state: device pointers to the live master/m/v arrays (the fused
  * variant alternates between two buffers) and the step count t. Any output
- * pointer may be NULL. */
+ * pointer may be NULL. ZERO_ERR_ARG while an asynchronous run is open. */
 int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t);
 
 /* Memory bandwidth reference: copy `bytes` (a multiple of 16, both pointers

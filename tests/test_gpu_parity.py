@@ -104,22 +104,29 @@ class Case:
         return [S.host_f16_bits(n, self.b0, S.key(self.seed, S.STREAM_GRAD, step, k),
                                 self.grad_dist) for k in range(self.nd)]
 
-    def step(self, gs):
+    def upload(self, gs):
         n = self.e0 - self.b0
         for k in range(self.nd):
             if n:
                 self.g_dev[k][:n].copy_(torch.from_numpy(gs[k].view(np.int16)))
-        rc = A.zero_step(self.h, [g.data_ptr() for g in self.g_dev], self.loss_scale,
-                         hyper(**self.hp), self.stream)
+
+    def oracle_step(self, gs, loss_scale):
         hp = Z.hyper(**self.hp)
         if self.stage <= 2 and self.view < 0:
             sk, self.t = Z.zero12_step(self.psi, gs, self.w_sh, self.m_sh, self.v_sh, self.reps,
-                                       self.loss_scale, hp, self.t)
+                                       loss_scale, hp, self.t)
         elif self.view >= 0:
-            sk, self.t = Z.dp_step(gs, self.w, self.m, self.v, self.p16, self.loss_scale, hp, self.t)
+            sk, self.t = Z.dp_step(gs, self.w, self.m, self.v, self.p16, loss_scale, hp, self.t)
         else:
             sk, self.t = Z.zero3_step(self.numel, gs, self.w_sh, self.m_sh, self.v_sh, self.p_sh,
-                                      self.loss_scale, hp, self.t)
+                                      loss_scale, hp, self.t)
+        return sk
+
+    def step(self, gs):
+        self.upload(gs)
+        rc = A.zero_step(self.h, [g.data_ptr() for g in self.g_dev], self.loss_scale,
+                         hyper(**self.hp), self.stream)
+        sk = self.oracle_step(gs, self.loss_scale)
         assert (rc == A.ZERO_SKIPPED) == sk, (rc, sk)
         return sk
 
@@ -372,4 +379,81 @@ def test_tma_gather_wait_that_gives_up_is_reported():
     c.check("after the reported failure: unchanged")  # gathers re-checked inside
     assert c.step(c.grads(2)) is False
     c.check("after the next step")
+    c.close()
+
+
+def _async_case(stage, variant, nd=4):
+    if stage == 3:
+        sizes = [8 * nd * 500, 8 * nd * 37, 8 * nd * 900]
+        return Case(sum(sizes), nd, 3, variant, tensors=list(zip(sizes, [0, 1, 1])),
+                    grad_dist=S.normal(1e-3, 1.0), hp=dict(weight_decay=0.01))
+    return Case(70_001, nd, stage, variant, grad_dist=S.normal(1e-3, 1.0),
+                hp=dict(weight_decay=0.01))
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("stage", [2, 3])
+def test_async_steps_with_dynamic_loss_scaling(stage, variant):
+    # 8 steps enqueued back to back; infs at steps 2 and 3 back the scale off
+    # twice, runs of 2 good steps grow it; the oracle follows the same rule
+    c = _async_case(stage, variant)
+    c.check("after init")
+    sc = A.zero_scaler(1024.0, 2.0, 0.5, 2)
+    A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], sc, 0.9, 0.999, c.stream)
+    scale, good, skipped = 1024.0, 0, 0
+    for s in range(8):
+        gs = c.grads(s)
+        if s in (2, 3):
+            gs[1][c.e0 - c.b0 - 1] = 0x7C00
+        c.upload(gs)
+        A.zero_step_async(c.h, hyper(**c.hp), c.stream)
+        sk = c.oracle_step(gs, scale)
+        skipped += int(sk)
+        scale, good = Z.scaler_update(scale, good, sk, 2.0, 0.5, 2)
+    st = A.zero_async_end(c.h, c.stream)
+    assert (st.t, st.skipped, st.good_steps) == (c.t, skipped, good) == (6, 2, good)
+    assert st.loss_scale == np.float32(scale)
+    c.check("after the asynchronous run")
+    assert c.step(c.grads(9)) is False  # the synchronous path continues from there
+    c.check("after a synchronous step")
+    c.close()
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_async_step_captured_in_a_cuda_graph(variant):
+    c = _async_case(2, variant, nd=8)
+    cap = torch.cuda.Stream()
+    sc = A.zero_scaler(4096.0, 2.0, 0.5, 3)
+    with torch.cuda.stream(cap):
+        A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], sc, 0.9, 0.999, cap.cuda_stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            A.zero_step_async(c.h, hyper(**c.hp), cap.cuda_stream)
+        scale, good = 4096.0, 0
+        for s in range(5):
+            gs = c.grads(s)
+            if s == 1:
+                gs[3][7] = 0x7E00
+            c.upload(gs)
+            graph.replay()
+            sk = c.oracle_step(gs, scale)
+            scale, good = Z.scaler_update(scale, good, sk, 2.0, 0.5, 3)
+        st = A.zero_async_end(c.h, cap.cuda_stream)
+    torch.cuda.synchronize()
+    assert (st.t, st.skipped) == (c.t, 1) and st.loss_scale == np.float32(scale)
+    c.check("after graph replays")
+    del graph
+    c.close()
+
+
+def test_async_rejects_mismatched_betas_and_sync_calls():
+    c = _async_case(2, A.ZERO_VARIANT_FUSED)
+    A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], A.zero_scaler(8.0, 2.0, 0.5, 1),
+                       0.9, 0.999, c.stream)
+    with pytest.raises(A.ZeroError):
+        A.zero_step_async(c.h, hyper(beta1=0.8), c.stream)
+    with pytest.raises(A.ZeroError):
+        A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], 1.0, hyper(), c.stream)
+    st = A.zero_async_end(c.h, c.stream)
+    assert st.t == 0
     c.close()

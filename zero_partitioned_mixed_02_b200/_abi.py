@@ -53,6 +53,16 @@ class zero_hyper(C.Structure):
                 ("eps", C.c_float), ("weight_decay", C.c_float)]
 
 
+class zero_scaler(C.Structure):
+    _fields_ = [("init_scale", C.c_float), ("growth_factor", C.c_float),
+                ("backoff_factor", C.c_float), ("growth_interval", C.c_int32)]
+
+
+class zero_async_state(C.Structure):
+    _fields_ = [("t", C.c_int64), ("skipped", C.c_int64), ("loss_scale", C.c_float),
+                ("good_steps", C.c_int32)]
+
+
 class zero_ledger(C.Structure):
     _fields_ = [("formula_bytes", C.c_double * 4), ("exact_bytes", C.c_int64 * 4),
                 ("comm_elements", C.c_int64 * 6), ("allreduce_buffer_bytes", C.c_int64),
@@ -90,6 +100,10 @@ def lib():
             "zero_step_launch": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P]),
             "zero_step_commit": (C.c_int, [P, P, C.POINTER(C.c_int)]),
             "zero_gather_layer": (C.c_int, [P, C.c_int32, P, P]),
+            "zero_async_begin": (C.c_int, [P, C.POINTER(P), C.POINTER(zero_scaler), C.c_float,
+                                           C.c_float, P]),
+            "zero_step_async": (C.c_int, [P, C.POINTER(zero_hyper), P]),
+            "zero_async_end": (C.c_int, [P, P, C.POINTER(zero_async_state)]),
             "zero_current_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                              C.POINTER(C.c_int64)]),
             "zero_stream_copy": (C.c_int, [P, P, C.c_size_t, P]),
@@ -190,6 +204,22 @@ def zero_step_launch(h: int, grads: Sequence[int], loss_scale: float, hp: zero_h
 def zero_step_commit(h: int, stream: int) -> int:
     sk = C.c_int(0)
     return _check(lib().zero_step_commit(h, stream, C.byref(sk)), "zero_step_commit", h)
+
+
+def zero_async_begin(h: int, grads: Sequence[int], sc: zero_scaler, beta1: float, beta2: float,
+                     stream: int) -> None:
+    _check(lib().zero_async_begin(h, _ptr_array(grads), C.byref(sc), beta1, beta2, stream),
+           "zero_async_begin", h)
+
+
+def zero_step_async(h: int, hp: zero_hyper, stream: int) -> None:
+    _check(lib().zero_step_async(h, C.byref(hp), stream), "zero_step_async", h)
+
+
+def zero_async_end(h: int, stream: int) -> zero_async_state:
+    out = zero_async_state()
+    _check(lib().zero_async_end(h, stream, C.byref(out)), "zero_async_end", h)
+    return out
 
 
 def zero_gather_layer(h: int, unit: int, out: int, stream: int) -> None:

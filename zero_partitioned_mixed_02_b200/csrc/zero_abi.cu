@@ -382,6 +382,10 @@ struct zero_handle {
     int occ_gather_tma = 0;
     int64_t hold_tile = -1;  // test hook for the bounded waits (zero_test_hold_tile)
     unsigned hold_rounds = 0;
+    bool async = false;      // between zero_async_begin and zero_async_end
+    float async_b1 = 0.0f, async_b2 = 0.0f;
+    zk::Ctrl ctrl_host{};    // staging copy of the control block
+    zk::Ctrl* d_ctrl = nullptr;
     const uint16_t** d_grad_tab = nullptr;
     uint16_t** d_out_tab = nullptr;
     unsigned* d_flag = nullptr;
@@ -524,6 +528,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
         return rc;
     }
     h->d_flag = reinterpret_cast<unsigned*>(h->ws + L.off_flag);
+    h->d_ctrl = reinterpret_cast<zk::Ctrl*>(h->ws + L.off_flag + 64);
     h->d_grad_tab = reinterpret_cast<const uint16_t**>(h->ws + L.off_grad_tab);
     h->d_out_tab = reinterpret_cast<uint16_t**>(h->ws + L.off_out_tab);
     h->d_step_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_step_segs);
@@ -597,7 +602,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
                               const zero_hyper* hp, void* stream)
 {
     if (!h || !grads || !hp) return ZERO_ERR_ARG;
-    if (h->pending) return ZERO_ERR_ARG;  // the previous launch was not committed
+    if (h->pending || h->async) return ZERO_ERR_ARG;  // uncommitted launch, or an asynchronous run is open
     if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale)) return ZERO_ERR_ARG;
     if (!std::isfinite(hp->lr) || !std::isfinite(hp->beta1) || !std::isfinite(hp->beta2) ||
         !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
@@ -726,6 +731,146 @@ ZERO_API int zero_step(zero_handle* h, const uint16_t* const* grads, float loss_
     return zero_step_commit(h, stream, skipped);
 }
 
+ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, const zero_scaler* sc,
+                              float beta1, float beta2, void* stream)
+{
+    if (!h || !grads || !sc || h->pending || h->async) return ZERO_ERR_ARG;
+    if (!(sc->init_scale > 0.0f) || !std::isfinite(sc->init_scale) || !(sc->growth_factor >= 1.0f) ||
+        !std::isfinite(sc->growth_factor) || !(sc->backoff_factor > 0.0f) || !(sc->backoff_factor <= 1.0f) ||
+        sc->growth_interval < 1 || !std::isfinite(beta1) || !std::isfinite(beta2))
+        return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    for (int k = 0; k < L.nd; ++k) {
+        if (!grads[k]) return ZERO_ERR_ARG;
+        if (!aligned16(grads[k])) return ZERO_ERR_ALIGN;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    h->grad_tab.assign(grads, grads + L.nd);
+    cudaError_t e = cudaMemcpyAsync(h->d_grad_tab, h->grad_tab.data(), L.nd * sizeof(uint16_t*),
+                                    cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    h->grad_tab_valid = true;
+    zk::Ctrl& c = h->ctrl_host;
+    c = zk::Ctrl{};
+    c.p1 = 1.0;
+    c.p2 = 1.0;
+    for (int64_t k = 0; k < h->t; ++k) {  // the t-fold products
+        c.p1 = c.p1 * (double)beta1;
+        c.p2 = c.p2 * (double)beta2;
+    }
+    c.t = h->t;
+    c.scale = sc->init_scale;
+    c.growth = sc->growth_factor;
+    c.backoff = sc->backoff_factor;
+    c.b1 = beta1;
+    c.b2 = beta2;
+    c.interval = sc->growth_interval;
+    c.cur = h->cur;
+    c.fused = L.variant != ZERO_VARIANT_TWO_PASS;
+    e = cudaMemcpyAsync(h->d_ctrl, &c, sizeof(zk::Ctrl), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->d_flag, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    h->async = true;
+    h->async_b1 = beta1;
+    h->async_b2 = beta2;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
+{
+    if (!h || !hp || !h->async) return ZERO_ERR_ARG;
+    if (hp->beta1 != h->async_b1 || hp->beta2 != h->async_b2) return ZERO_ERR_ARG;
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
+        return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    if (L.step_chunks == 0) return ZERO_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    zk::StepArgs a{};
+    a.segs = h->d_step_segs;
+    a.n_segs = (int)L.step_segs.size();
+    a.n_chunks = L.step_chunks;
+    a.grads = h->d_grad_tab;
+    a.outs = h->d_out_tab;
+    a.nd = L.nd;
+    a.n_out = (int)h->out_tab.size();
+    a.flag = h->d_flag;
+    a.err = h->d_flag + 1;
+    a.call_id = 1;  // the commit kernel clears the word after every step
+    a.c.lr = hp->lr;
+    a.c.b1 = hp->beta1;
+    a.c.b2 = hp->beta2;
+    a.c.omb1 = 1.0f - hp->beta1;
+    a.c.omb2 = 1.0f - hp->beta2;
+    a.c.eps = hp->eps;
+    a.c.wd = hp->weight_decay;
+    a.ctrl = h->d_ctrl;
+    const int nb = L.variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
+    for (int b = 0; b < 2; ++b)
+        for (int k = 0; k < 3; ++k) a.st[b][k] = h->state(b < nb ? b : 0, k);
+    const bool fused = L.variant != ZERO_VARIANT_TWO_PASS;
+    cudaError_t e;
+    if (h->use_tma) {
+        zk::TmaArgs ta{};
+        ta.b = a;
+        ta.runs = h->d_tma_runs;
+        ta.n_runs = (int)L.tma_runs.size();
+        ta.n_tiles = L.tma_tiles;
+        ta.n_scal = L.tma_scal;
+        ta.err = h->d_flag + 1;
+        ta.wait_rounds = zk::kTmaWaitRounds;
+        ta.hold_tile = -1;
+        const int64_t cap = (int64_t)h->sms * h->occ_tma;
+        const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
+        e = zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
+    } else if (fused) {
+        e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
+    } else {
+        a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
+        e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s);
+        if (e == cudaSuccess) e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s);
+    }
+    // the fused passes wrote fp16 parameters: rewrite them from the unchanged
+    // master if the step overflowed (the kernel returns at once otherwise)
+    if (e == cudaSuccess && fused)
+        e = zk::launch_step(zk::K_CAST_IF, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
+    if (e == cudaSuccess) e = zk::launch_commit(h->d_ctrl, h->d_flag, h->d_flag + 1, s);
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+}
+
+ZERO_API int zero_async_end(zero_handle* h, void* stream, zero_async_state* out)
+{
+    if (!h || !h->async) return ZERO_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    zk::Ctrl c{};
+    unsigned err = 0;
+    cudaError_t e = cudaMemcpyAsync(&c, h->d_ctrl, sizeof(zk::Ctrl), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&err, h->d_flag + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    h->async = false;
+    h->t = c.t;
+    h->cur = c.cur;
+    h->bc_b1 = h->async_b1;  // continue the host's products where the device left them
+    h->bc_b2 = h->async_b2;
+    h->bc_t = c.t;
+    h->bc_p1 = c.p1;
+    h->bc_p2 = c.p2;
+    if (out) {
+        out->t = c.t;
+        out->skipped = c.skipped;
+        out->loss_scale = c.scale;
+        out->good_steps = c.good;
+    }
+    if (err != 0) {
+        e = cudaMemsetAsync(h->d_flag + 1, 0, sizeof(unsigned), s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+        return ZERO_ERR_INTERNAL;
+    }
+    return ZERO_OK;
+}
+
 ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
 {
     if (!h || h->pending) return ZERO_ERR_ARG;
@@ -765,7 +910,7 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
 
 ZERO_API int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t)
 {
-    if (!h) return ZERO_ERR_ARG;
+    if (!h || h->async) return ZERO_ERR_ARG;
     if (master) *master = h->state(h->cur, 0);
     if (m) *m = h->state(h->cur, 1);
     if (v) *v = h->state(h->cur, 2);

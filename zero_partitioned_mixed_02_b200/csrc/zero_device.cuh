@@ -192,8 +192,54 @@ __device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, con
     v = v1;
 }
 
+// What a launch's items use: the state buffers and the step constants. For
+// the synchronous step they come from the kernel arguments; for the
+// asynchronous step from the control block: the bias corrections for t + 1
+// (one more factor on the t-fold products) and 1 / loss scale, with the host
+// path's roundings, and the buffers picked by the live index (by selects, so
+// nothing is indexed at run time).
+struct Live {
+    const float* w_in;
+    const float* m_in;
+    const float* v_in;
+    float* w_out;
+    float* m_out;
+    float* v_out;
+    Coef c;
+};
+
+__device__ __forceinline__ Live live_of(const StepArgs& a)
+{
+    Live L;
+    L.c = a.c;
+    if (!a.ctrl) {
+        L.w_in = a.w_in;
+        L.m_in = a.m_in;
+        L.v_in = a.v_in;
+        L.w_out = a.w_out;
+        L.m_out = a.m_out;
+        L.v_out = a.v_out;
+        return L;
+    }
+    const Ctrl* c = a.ctrl;
+    const double p1 = c->p1 * (double)c->b1;
+    const double p2 = c->p2 * (double)c->b2;
+    L.c.bc1 = (float)(1.0 - p1);
+    L.c.bc2 = (float)(1.0 - p2);
+    L.c.inv_scale = (float)(1.0 / (double)c->scale);
+    const bool in1 = c->cur != 0;
+    const bool out1 = c->fused ? !in1 : in1;
+    L.w_in = in1 ? a.st[1][0] : a.st[0][0];
+    L.m_in = in1 ? a.st[1][1] : a.st[0][1];
+    L.v_in = in1 ? a.st[1][2] : a.st[0][2];
+    L.w_out = out1 ? a.st[1][0] : a.st[0][0];
+    L.m_out = out1 ? a.st[1][1] : a.st[0][1];
+    L.v_out = out1 ? a.st[1][2] : a.st[0][2];
+    return L;
+}
+
 template <int K>
-__device__ __forceinline__ void step_scalar(const StepArgs& a, const uint16_t* const* gp,
+__device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, const uint16_t* const* gp,
                                             uint16_t* const* op, const SegDesc& d, long long e,
                                             bool& bad)
 {
@@ -201,19 +247,19 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const uint16_t* c
     float w = 0.0f, m = 0.0f, v = 0.0f, g = 0.0f;
     if (K == K_INIT) {
         w = __ldcs(a.master_init + gi);
-        __stcs(a.w_out + si, w);
-        __stcs(a.m_out + si, 0.0f);
-        __stcs(a.v_out + si, 0.0f);
+        __stcs(L.w_out + si, w);
+        __stcs(L.m_out + si, 0.0f);
+        __stcs(L.v_out + si, 0.0f);
     } else if (K == K_CAST) {
-        w = __ldcs(a.w_in + si);
+        w = __ldcs(L.w_in + si);
     } else {
         if (K == K_STEP_FUSED || K == K_UPDATE) {
-            w = __ldcs(a.w_in + si);
-            m = __ldcs(a.m_in + si);
-            v = __ldcs(a.v_in + si);
+            w = __ldcs(L.w_in + si);
+            m = __ldcs(L.m_in + si);
+            v = __ldcs(L.v_in + si);
         }
         if (K == K_STEP_FUSED || K == K_REDUCE) {
-            g = __fmul_rn(reduce1(gp, a.nd, gi), a.c.inv_scale);
+            g = __fmul_rn(reduce1(gp, a.nd, gi), L.c.inv_scale);
             bad |= nonfinite(g);
         }
         if (K == K_REDUCE) {
@@ -221,10 +267,10 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const uint16_t* c
             return;
         }
         if (K == K_UPDATE) g = __ldcs(a.red + si);
-        adam1(g, w, m, v, a.c);
-        __stcs(a.w_out + si, w);
-        __stcs(a.m_out + si, m);
-        __stcs(a.v_out + si, v);
+        adam1(g, w, m, v, L.c);
+        __stcs(L.w_out + si, w);
+        __stcs(L.m_out + si, m);
+        __stcs(L.v_out + si, v);
     }
     const unsigned short h = f2h(w);
     for (int k = 0; k < a.n_out; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);

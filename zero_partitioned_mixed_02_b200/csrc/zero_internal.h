@@ -39,9 +39,27 @@ struct alignas(16) SegDesc {
 };
 static_assert(sizeof(SegDesc) == 48, "SegDesc layout");
 
-// Per-step binary32 constants, computed on the host.
+// Per-step binary32 constants, computed on the host (or, for the
+// asynchronous step, partly on the device from the control block).
 struct Coef {
     float inv_scale, lr, b1, b2, omb1, omb2, bc1, bc2, eps, wd;
+};
+
+// Device-resident control block of the asynchronous step: everything the host
+// would otherwise decide between steps.
+struct alignas(16) Ctrl {
+    double p1, p2;       // beta1^t, beta2^t as t-fold double products
+    long long t;         // committed steps
+    long long skipped;   // steps skipped since the asynchronous run began
+    float scale;         // current loss scale
+    float growth;        // dynamic loss scaling: growth factor,
+    float backoff;       //   back-off factor,
+    float b1, b2;        // betas the products use
+    int interval;        //   good steps before growth,
+    int good;            //   current run of good steps
+    int cur;             // live state buffer
+    int fused;           // 1: a step writes the other buffer, switched on commit
+    int pad[3];
 };
 
 struct StepArgs {
@@ -63,6 +81,11 @@ struct StepArgs {
     unsigned* flag;                // overflow word: holds the id of the last call that overflowed
     unsigned call_id;
     Coef c;
+    // asynchronous step: when ctrl is set the kernel takes inv_scale, bc1,
+    // bc2 and the in/out state buffers (from st) from the control block
+    const Ctrl* ctrl;
+    float* st[2][3];
+    unsigned* err;                 // kernel error word (roll-back condition)
 };
 
 struct GatherArgs {
@@ -147,7 +170,8 @@ enum Kernel : int {
     K_CAST = 3,        // fp16 write-back of the current master (overflow roll-back)
     K_INIT = 4,        // master = master_init, m = v = 0, fp16 write-back
     K_GATHER = 5,      // stage-3 layer gather
-    K_COUNT = 6
+    K_CAST_IF = 6,     // K_CAST only if the step overflowed (asynchronous step)
+    K_COUNT = 7
 };
 
 // Blocks per SM the kernel reaches with `smem` bytes of dynamic shared memory.
@@ -155,6 +179,8 @@ cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm);
 cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cudaStream_t s);
+// Asynchronous step: commit or roll back on the device (one thread).
+cudaError_t launch_commit(Ctrl* ctrl, unsigned* flag, const unsigned* err, cudaStream_t s);
 // TMA-staged fused step: one-time attribute set-up and blocks per SM for the
 // shape and nd ranks, launch.
 cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);

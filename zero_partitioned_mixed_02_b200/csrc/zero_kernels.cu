@@ -37,7 +37,7 @@ namespace {
 // ---- per-item bodies of the step kernels ----
 
 template <int K>
-__device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* const* gp,
+__device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const uint16_t* const* gp,
                                          uint16_t* const* op, const SegDesc& d, const Pair& p,
                                          bool& bad)
 {
@@ -50,22 +50,22 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* cons
         ld_pair(a.master_init, ga, gb, hb, w);
 #pragma unroll
         for (int j = 0; j < 8; ++j) m[j] = 0.0f;
-        st_pair(a.w_out, sa, sb, hb, w);
-        st_pair(a.m_out, sa, sb, hb, m);
-        st_pair(a.v_out, sa, sb, hb, m);
+        st_pair(L.w_out, sa, sb, hb, w);
+        st_pair(L.m_out, sa, sb, hb, m);
+        st_pair(L.v_out, sa, sb, hb, m);
     } else if (K == K_CAST) {
-        ld_pair(a.w_in, sa, sb, hb, w);
+        ld_pair(L.w_in, sa, sb, hb, w);
     } else {
         if (K == K_STEP_FUSED || K == K_UPDATE) {
-            ld_pair(a.w_in, sa, sb, hb, w);
-            ld_pair(a.m_in, sa, sb, hb, m);
-            ld_pair(a.v_in, sa, sb, hb, v);
+            ld_pair(L.w_in, sa, sb, hb, w);
+            ld_pair(L.m_in, sa, sb, hb, m);
+            ld_pair(L.v_in, sa, sb, hb, v);
         }
         if (K == K_STEP_FUSED || K == K_REDUCE) {
             reduce_pair(gp, a.nd, ga, gb, hb, g);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                g[j] = __fmul_rn(g[j], a.c.inv_scale);
+                g[j] = __fmul_rn(g[j], L.c.inv_scale);
                 bad |= nonfinite(g[j]);  // an absent second quad holds zeros
             }
         }
@@ -75,10 +75,10 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const uint16_t* cons
         }
         if (K == K_UPDATE) ld_pair(a.red, sa, sb, hb, g);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], a.c);
-        st_pair(a.w_out, sa, sb, hb, w);
-        st_pair(a.m_out, sa, sb, hb, m);
-        st_pair(a.v_out, sa, sb, hb, v);
+        for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], L.c);
+        st_pair(L.w_out, sa, sb, hb, w);
+        st_pair(L.m_out, sa, sb, hb, m);
+        st_pair(L.v_out, sa, sb, hb, v);
     }
     const uint2 h0 = pack(w), h1 = pack(w + 4);
     for (int k = 0; k < a.n_out; ++k) {
@@ -131,14 +131,22 @@ __device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long 
     }
 }
 
+// K_CAST_IF is K_CAST run only when the step overflowed or a kernel gave up.
 template <int K>
-__global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const StepArgs a)
+__global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const StepArgs a0)
 {
     extern __shared__ uintptr_t s_ptr[];
     if (K == K_UPDATE) {
         // pass 2 of the two-pass variant: the whole step is skipped on overflow
-        if (*reinterpret_cast<volatile unsigned*>(a.flag) == a.call_id) return;
+        if (*reinterpret_cast<volatile const unsigned*>(a0.flag) == a0.call_id) return;
     }
+    if (K == K_CAST_IF) {
+        if (*reinterpret_cast<volatile const unsigned*>(a0.flag) != a0.call_id &&
+            *reinterpret_cast<volatile const unsigned*>(a0.err) == 0)
+            return;
+    }
+    const StepArgs& a = a0;
+    const Live L = live_of(a);
     constexpr bool kGrads = (K == K_STEP_FUSED || K == K_REDUCE);
     const int n_g = kGrads ? a.nd : 0;
     const int n_o = (K == K_REDUCE) ? 0 : a.n_out;
@@ -149,11 +157,12 @@ __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const Ste
     const uint16_t* const* gp = reinterpret_cast<const uint16_t* const*>(s_ptr);
     uint16_t* const* op = reinterpret_cast<uint16_t* const*>(s_ptr + n_g);
 
+    constexpr int KB = (K == K_CAST_IF) ? K_CAST : K;  // the item body
     bool bad = false;
     walk(
         a.segs, a.n_segs, a.n_chunks,
-        [&](const SegDesc& d, const Pair& p) { step_vec<K>(a, gp, op, d, p, bad); },
-        [&](const SegDesc& d, long long e) { step_scalar<K>(a, gp, op, d, e, bad); });
+        [&](const SegDesc& d, const Pair& p) { step_vec<KB>(a, L, gp, op, d, p, bad); },
+        [&](const SegDesc& d, long long e) { step_scalar<KB>(a, L, gp, op, d, e, bad); });
 
     if (kGrads) {
         // one atomic per warp that saw a non-finite unscaled gradient
@@ -184,6 +193,33 @@ __global__ void __launch_bounds__(kThreads) copy_kernel(uint4* dst, const uint4*
         __stcs(dst + i, __ldcs(src + i));
 }
 
+// The asynchronous step's commit: skip (back off the loss scale) or commit
+// (advance t and the bias-correction products, switch buffers, grow the loss
+// scale after a run of good steps), then clear the overflow word.
+__global__ void commit_kernel(Ctrl* c, unsigned* flag, const unsigned* err)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const bool skip = (*reinterpret_cast<volatile unsigned*>(flag) != 0) ||
+                      (*reinterpret_cast<volatile const unsigned*>(err) != 0);
+    if (skip) {
+        c->scale = __fmul_rn(c->scale, c->backoff);
+        c->good = 0;
+        c->skipped += 1;
+    } else {
+        c->p1 = c->p1 * (double)c->b1;
+        c->p2 = c->p2 * (double)c->b2;
+        c->t += 1;
+        if (c->fused) c->cur = 1 - c->cur;
+        c->good += 1;
+        if (c->good >= c->interval) {
+            const float grown = __fmul_rn(c->scale, c->growth);
+            if (!nonfinite(grown)) c->scale = grown;
+            c->good = 0;
+        }
+    }
+    *flag = 0;
+}
+
 const void* kernel_ptr(Kernel k)
 {
     switch (k) {
@@ -193,6 +229,7 @@ const void* kernel_ptr(Kernel k)
         case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST>);
         case K_INIT: return reinterpret_cast<const void*>(&step_kernel<K_INIT>);
         case K_GATHER: return reinterpret_cast<const void*>(&gather_kernel);
+        case K_CAST_IF: return reinterpret_cast<const void*>(&step_kernel<K_CAST_IF>);
         default: return nullptr;
     }
 }
@@ -217,8 +254,15 @@ cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s)
         case K_UPDATE: step_kernel<K_UPDATE><<<grid, kThreads, smem, s>>>(a); break;
         case K_CAST: step_kernel<K_CAST><<<grid, kThreads, smem, s>>>(a); break;
         case K_INIT: step_kernel<K_INIT><<<grid, kThreads, smem, s>>>(a); break;
+        case K_CAST_IF: step_kernel<K_CAST_IF><<<grid, kThreads, smem, s>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_commit(Ctrl* ctrl, unsigned* flag, const unsigned* err, cudaStream_t s)
+{
+    commit_kernel<<<1, 32, 0, s>>>(ctrl, flag, err);
     return cudaGetLastError();
 }
 

@@ -107,6 +107,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
     constexpr int kTmaTile = WARPS * 32 * kQuad;
     extern __shared__ __align__(128) char smem[];
     const StepArgs& b = a.b;
+    const Live L = live_of(b);
     const int nd = b.nd;
     const unsigned full0 = smem_u32(smem);
     const unsigned empty0 = full0 + 8 * kTmaStages;
@@ -159,9 +160,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
             for (int k = 0; k < nd; ++k)
                 bulk_g2s(smem_u32(sp + k * kTmaTile * 2), b.grads[k] + d.gi, 2u * n, full);
             char* sw = sp + nd * kTmaTile * 2;
-            bulk_g2s(smem_u32(sw), b.w_in + d.si, 4u * n, full);
-            bulk_g2s(smem_u32(sw + kTmaTile * 4), b.m_in + d.si, 4u * n, full);
-            bulk_g2s(smem_u32(sw + 2 * kTmaTile * 4), b.v_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw), L.w_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw + kTmaTile * 4), L.m_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw + 2 * kTmaTile * 4), L.v_in + d.si, 4u * n, full);
         }
         // drain: every stage's last armed phase must have landed before exit
         for (int k = 0; k < kTmaStages && k < it; ++k) {
@@ -210,15 +211,15 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         if (active) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                g[j] = __fmul_rn(g[j], b.c.inv_scale);
+                g[j] = __fmul_rn(g[j], L.c.inv_scale);
                 bad |= nonfinite(g[j]);
-                adam1(g[j], w[j], m[j], v[j], b.c);
+                adam1(g[j], w[j], m[j], v[j], L.c);
             }
             // state indices are 4-element and output indices 8-element aligned
             // with the gradient index (the host's eligibility rule)
-            __stcs(reinterpret_cast<float4*>(b.w_out + d.si + q4), make_float4(w[0], w[1], w[2], w[3]));
-            __stcs(reinterpret_cast<float4*>(b.m_out + d.si + q4), make_float4(m[0], m[1], m[2], m[3]));
-            __stcs(reinterpret_cast<float4*>(b.v_out + d.si + q4), make_float4(v[0], v[1], v[2], v[3]));
+            __stcs(reinterpret_cast<float4*>(L.w_out + d.si + q4), make_float4(w[0], w[1], w[2], w[3]));
+            __stcs(reinterpret_cast<float4*>(L.m_out + d.si + q4), make_float4(m[0], m[1], m[2], m[3]));
+            __stcs(reinterpret_cast<float4*>(L.v_out + d.si + q4), make_float4(v[0], v[1], v[2], v[3]));
             const uint2 h = pack(w);
             for (int k = 0; k < b.n_out; ++k) __stcs(reinterpret_cast<uint2*>(b.outs[k] + d.oi + q4), h);
         }
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         sd.head = run.head;
         sd.tail = run.tail;
         const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
-        step_scalar<K_STEP_FUSED>(b, b.grads, b.outs, sd, e, bad);
+        step_scalar<K_STEP_FUSED>(b, L, b.grads, b.outs, sd, e, bad);
     }
 
     // one atomic per consumer warp that saw a non-finite unscaled gradient
