@@ -193,8 +193,9 @@ __device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, con
 }
 
 // What a launch's items use: the state buffers and the step constants. For
-// the synchronous step they come from the kernel arguments; for the
-// asynchronous step from the control block: the bias corrections for t + 1
+// the synchronous step (ASYNC = false: the kernel argument values, which the
+// compiler reads straight from the parameter bank) they come from the kernel
+// arguments; for the asynchronous step from the control block: the bias corrections for t + 1
 // (one more factor on the t-fold products) and 1 / loss scale, with the host
 // path's roundings, and the buffers picked by the live index (by selects, so
 // nothing is indexed at run time).
@@ -208,11 +209,12 @@ struct Live {
     Coef c;
 };
 
+template <bool ASYNC>
 __device__ __forceinline__ Live live_of(const StepArgs& a)
 {
     Live L;
     L.c = a.c;
-    if (!a.ctrl) {
+    if (!ASYNC) {
         L.w_in = a.w_in;
         L.m_in = a.m_in;
         L.v_in = a.v_in;

@@ -132,7 +132,8 @@ __device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long 
 }
 
 // K_CAST_IF is K_CAST run only when the step overflowed or a kernel gave up.
-template <int K>
+// ASYNC: the step constants and state buffers come from the control block.
+template <int K, bool ASYNC>
 __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const StepArgs a0)
 {
     extern __shared__ uintptr_t s_ptr[];
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const Ste
             return;
     }
     const StepArgs& a = a0;
-    const Live L = live_of(a);
+    const Live L = live_of<ASYNC>(a);
     constexpr bool kGrads = (K == K_STEP_FUSED || K == K_REDUCE);
     const int n_g = kGrads ? a.nd : 0;
     const int n_o = (K == K_REDUCE) ? 0 : a.n_out;
@@ -223,13 +224,13 @@ __global__ void commit_kernel(Ctrl* c, unsigned* flag, const unsigned* err)
 const void* kernel_ptr(Kernel k)
 {
     switch (k) {
-        case K_STEP_FUSED: return reinterpret_cast<const void*>(&step_kernel<K_STEP_FUSED>);
-        case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE>);
-        case K_UPDATE: return reinterpret_cast<const void*>(&step_kernel<K_UPDATE>);
-        case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST>);
-        case K_INIT: return reinterpret_cast<const void*>(&step_kernel<K_INIT>);
+        case K_STEP_FUSED: return reinterpret_cast<const void*>(&step_kernel<K_STEP_FUSED, false>);
+        case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE, false>);
+        case K_UPDATE: return reinterpret_cast<const void*>(&step_kernel<K_UPDATE, false>);
+        case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST, false>);
+        case K_INIT: return reinterpret_cast<const void*>(&step_kernel<K_INIT, false>);
         case K_GATHER: return reinterpret_cast<const void*>(&gather_kernel);
-        case K_CAST_IF: return reinterpret_cast<const void*>(&step_kernel<K_CAST_IF>);
+        case K_CAST_IF: return reinterpret_cast<const void*>(&step_kernel<K_CAST_IF, true>);
         default: return nullptr;
     }
 }
@@ -248,13 +249,26 @@ cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm)
 cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s)
 {
     const int smem = step_smem_bytes(a.nd, a.n_out);
+    const bool as = a.ctrl != nullptr;
     switch (k) {
-        case K_STEP_FUSED: step_kernel<K_STEP_FUSED><<<grid, kThreads, smem, s>>>(a); break;
-        case K_REDUCE: step_kernel<K_REDUCE><<<grid, kThreads, smem, s>>>(a); break;
-        case K_UPDATE: step_kernel<K_UPDATE><<<grid, kThreads, smem, s>>>(a); break;
-        case K_CAST: step_kernel<K_CAST><<<grid, kThreads, smem, s>>>(a); break;
-        case K_INIT: step_kernel<K_INIT><<<grid, kThreads, smem, s>>>(a); break;
-        case K_CAST_IF: step_kernel<K_CAST_IF><<<grid, kThreads, smem, s>>>(a); break;
+        case K_STEP_FUSED:
+            if (as) step_kernel<K_STEP_FUSED, true><<<grid, kThreads, smem, s>>>(a);
+            else step_kernel<K_STEP_FUSED, false><<<grid, kThreads, smem, s>>>(a);
+            break;
+        case K_REDUCE:
+            if (as) step_kernel<K_REDUCE, true><<<grid, kThreads, smem, s>>>(a);
+            else step_kernel<K_REDUCE, false><<<grid, kThreads, smem, s>>>(a);
+            break;
+        case K_UPDATE:
+            if (as) step_kernel<K_UPDATE, true><<<grid, kThreads, smem, s>>>(a);
+            else step_kernel<K_UPDATE, false><<<grid, kThreads, smem, s>>>(a);
+            break;
+        case K_CAST: step_kernel<K_CAST, false><<<grid, kThreads, smem, s>>>(a); break;
+        case K_INIT: step_kernel<K_INIT, false><<<grid, kThreads, smem, s>>>(a); break;
+        case K_CAST_IF:
+            if (!as) return cudaErrorInvalidValue;
+            step_kernel<K_CAST_IF, true><<<grid, kThreads, smem, s>>>(a);
+            break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

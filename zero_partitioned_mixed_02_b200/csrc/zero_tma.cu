@@ -98,7 +98,7 @@ __device__ __forceinline__ int find_tma_run(const TmaRun* runs, int n, long long
     return lo;
 }
 
-template <int WARPS, int STAGES>
+template <int WARPS, int STAGES, bool ASYNC>
 __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const TmaArgs a)
 {
     static_assert(STAGES <= kMaxStages, "too many stages");
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
     constexpr int kTmaTile = WARPS * 32 * kQuad;
     extern __shared__ __align__(128) char smem[];
     const StepArgs& b = a.b;
-    const Live L = live_of(b);
+    const Live L = live_of<ASYNC>(b);
     const int nd = b.nd;
     const unsigned full0 = smem_u32(smem);
     const unsigned empty0 = full0 + 8 * kTmaStages;
@@ -354,25 +354,33 @@ constexpr int kGatherSmem = 128 + kGatherStages * kGatherTile * 2;
 
 int smem_bytes(TmaShape sh, int nd) { return kHdrBytes + sh.stages * (nd * sh.tile * 2 + 3 * sh.tile * 4); }
 
+template <bool ASYNC>
 const void* kernel_for(TmaShape sh)
 {
     if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages)
-        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaWide.warps, kTmaWide.stages>);
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaWide.warps, kTmaWide.stages, ASYNC>);
     if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages)
-        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages>);
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, ASYNC>);
     return nullptr;
 }
 
 }  // namespace
 
+// Both the synchronous and the asynchronous kernel of the shape get the
+// shared-memory attribute; the reported occupancy is the smaller of the two.
 cudaError_t tma_prepare(TmaShape sh, int nd, int* blocks_per_sm)
 {
-    const void* f = kernel_for(sh);
-    if (!f) return cudaErrorInvalidValue;
+    const void* f = kernel_for<false>(sh);
+    const void* fa = kernel_for<true>(sh);
+    if (!f || !fa) return cudaErrorInvalidValue;
     const int smem = smem_bytes(sh, nd);
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, f, (sh.warps + 1) * 32, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fa, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int occ = 0, occ_a = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, f, (sh.warps + 1) * 32, smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, fa, (sh.warps + 1) * 32, smem);
+    *blocks_per_sm = occ < occ_a ? occ : occ_a;
+    return e;
 }
 
 cudaError_t tma_gather_prepare(int* blocks_per_sm)
@@ -391,12 +399,21 @@ cudaError_t launch_gather_tma(const TmaGatherArgs& a, int grid, cudaStream_t s)
 cudaError_t launch_step_tma(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s)
 {
     const int smem = smem_bytes(sh, a.b.nd);
-    if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages)
-        step_tma_kernel<kTmaWide.warps, kTmaWide.stages><<<grid, (sh.warps + 1) * 32, smem, s>>>(a);
-    else if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages)
-        step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages><<<grid, (sh.warps + 1) * 32, smem, s>>>(a);
-    else
+    const int threads = (sh.warps + 1) * 32;
+    const bool as = a.b.ctrl != nullptr;
+    if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages) {
+        if (as)
+            step_tma_kernel<kTmaWide.warps, kTmaWide.stages, true><<<grid, threads, smem, s>>>(a);
+        else
+            step_tma_kernel<kTmaWide.warps, kTmaWide.stages, false><<<grid, threads, smem, s>>>(a);
+    } else if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages) {
+        if (as)
+            step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, true><<<grid, threads, smem, s>>>(a);
+        else
+            step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, false><<<grid, threads, smem, s>>>(a);
+    } else {
         return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 
