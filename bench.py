@@ -50,6 +50,8 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass"], default="fused-tma")
+    p.add_argument("--async", dest="async_steps", action="store_true",
+                   help="time zero_step_async: steps enqueued back to back, no host sync")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -102,13 +104,15 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_FILES = ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu", "zero_tma.cu")
+
+
 def kernel_sha():
-    """Hash of every device source the step kernels are built from."""
+    """Hash of the device sources the step kernels are built from."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in KERNEL_FILES:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
@@ -360,8 +364,23 @@ def run_ours(args):
 
     kernel_events = []
     gather_events = []
+    if args.async_steps:
+        # steps enqueued back to back; the loss scale is dynamic on the device
+        sc = A.zero_scaler(wl.loss_scale, 2.0, 0.5, 2000)
+        A.zero_async_begin(h, gptrs, sc, wl.beta1, wl.beta2, s)
 
     def one_step(timed):
+        if args.async_steps:
+            if timed:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            A.zero_step_async(h, hp, s)
+            if timed:
+                b.record(stream)
+                kernel_events.append((a, b))
+            for u in order:
+                A.zero_gather_layer(h, u, gather_out.data_ptr(), s)
+            return
         if timed:
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -397,6 +416,10 @@ def run_ours(args):
     t1.record(stream)
     torch.cuda.synchronize()
     clock_info = clocks.stop() if clocks else None
+    if args.async_steps:
+        st = A.zero_async_end(h, s)
+        if st.skipped:
+            raise RuntimeError("unexpected skip in the benchmark workload")
     total_ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
     kern_ms = [a.elapsed_time(b) for a, b in kernel_events]
     if world > 1:
@@ -404,6 +427,8 @@ def run_ours(args):
 
     n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant)
     launches_per_step = (2 if args.variant == "two-pass" else 1) + len(order)
+    if args.async_steps:  # + the conditional roll-back (fused variants) and the commit kernel
+        launches_per_step += 1 if args.variant == "two-pass" else 2
     step_s = total_ms / 1e3 / args.steps
     value = whole_job_value(n, args.steps, world, total_ms)
     peak, peak_src = measured_peak()
@@ -429,6 +454,7 @@ def run_ours(args):
                      "frac": achieved / peak, "traffic": traffic, "kernel": kname,
                      "algorithmic_bytes_per_launch": dom_bytes,
                      "kernel_ms": statistics.mean(kern_ms), "peak_source": peak_src},
+        "mode": "async" if args.async_steps else "sync",
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
     }
