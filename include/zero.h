@@ -261,6 +261,15 @@ int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
  * pointer may be NULL. ZERO_ERR_ARG while an asynchronous run is open. */
 int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t);
 
+/* Checkpoint / resume: restore a saved state into the handle. master, m, v
+ * are device fp32 arrays in state order (ledger.state_elems values each, as
+ * zero_current_state exposes them; they may be the live arrays themselves),
+ * t the step count they belong to. The fp16 parameters (replicas or stage-3
+ * shards) are rewritten from master. To save, copy the three arrays
+ * zero_current_state points to, and t. Synchronises `stream`. */
+int zero_set_state(zero_handle* h, const float* master, const float* m, const float* v, int64_t t,
+                   void* stream);
+
 /* Memory bandwidth reference: copy `bytes` (a multiple of 16, both pointers
  * 16-byte aligned) from src to dst with 16-byte streaming loads and stores. */
 int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);

@@ -94,3 +94,22 @@ def test_limits_2psi_and_3psi():
     c = Z.comm_elements(psi, 1 << 20)
     assert c["dp"] / (1 << 20) / psi == pytest.approx(2.0, rel=1e-5)
     assert c["stage3"] / (1 << 20) / psi == pytest.approx(3.0, rel=1e-5)
+
+
+def test_printed_communication_volumes(golden_dir):
+    import os
+    rows = []
+    with open(os.path.join(golden_dir, "comm_pages.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                q, val, src = line.split()
+                rows.append((q, float(val), src))
+    assert len(rows) >= 8
+    psi, nd = 10**9, 1 << 20  # the printed figures are the large-Nd limits
+    c = Z.comm_elements(psi, nd)
+    per_rank = {k: c[k] / nd / psi for k in ("dp", "stage1", "stage2", "stage3")}
+    got = {"dp": per_rank["dp"], "s1": per_rank["stage1"], "s2": per_rank["stage2"],
+           "s3": per_rank["stage3"], "s3_over_dp": c["stage3"] / c["dp"]}
+    for q, val, src in rows:
+        assert got[q] == pytest.approx(val, rel=1e-5), (q, val, src)

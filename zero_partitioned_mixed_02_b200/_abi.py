@@ -107,6 +107,7 @@ def lib():
             "zero_current_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                              C.POINTER(C.c_int64)]),
             "zero_stream_copy": (C.c_int, [P, P, C.c_size_t, P]),
+            "zero_set_state": (C.c_int, [P, P, P, P, C.c_int64, P]),
             "zero_step_static": (C.c_int, [C.c_int64, C.c_int32, C.POINTER(P), P, P, P, C.POINTER(P),
                                            C.c_float, C.POINTER(zero_hyper),
                                            C.POINTER(C.c_int64), P, C.POINTER(C.c_int)]),
@@ -232,6 +233,10 @@ def zero_current_state(h: int) -> tuple[int, int, int, int]:
     _check(lib().zero_current_state(h, C.byref(w), C.byref(m), C.byref(v), C.byref(t)),
            "zero_current_state")
     return w.value, m.value, v.value, t.value
+
+
+def zero_set_state(h: int, master: int, m: int, v: int, t: int, stream: int) -> None:
+    _check(lib().zero_set_state(h, master, m, v, t, stream), "zero_set_state", h)
 
 
 def zero_stream_copy(dst: int, src: int, nbytes: int, stream: int) -> None:

@@ -908,6 +908,41 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
 }
 
+ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m, const float* v, int64_t t,
+                           void* stream)
+{
+    if (!h || h->pending || h->async || t < 0) return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    const size_t bytes = (size_t)L.state_elems * sizeof(float);
+    if (L.state_elems > 0 && (!master || !m || !v)) return ZERO_ERR_ARG;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZERO_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float* src[3] = {master, m, v};
+    cudaError_t e = cudaSuccess;
+    for (int k = 0; k < 3 && e == cudaSuccess && bytes > 0; ++k) {
+        float* dst = h->state(h->cur, k);
+        if (dst != src[k]) e = cudaMemcpyAsync(dst, src[k], bytes, cudaMemcpyDeviceToDevice, s);
+    }
+    if (e == cudaSuccess && L.step_chunks > 0) {
+        // the fp16 parameters follow the restored master
+        zk::StepArgs a{};
+        a.segs = h->d_step_segs;
+        a.n_segs = (int)L.step_segs.size();
+        a.n_chunks = L.step_chunks;
+        a.outs = h->d_out_tab;
+        a.n_out = (int)h->out_tab.size();
+        a.nd = L.nd;
+        a.w_in = h->state(h->cur, 0);
+        a.flag = h->d_flag;
+        e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    h->t = t;
+    h->bc_t = -1;  // recompute the bias-correction products for the new t
+    return ZERO_OK;
+}
+
 ZERO_API int zero_current_state(const zero_handle* h, float** master, float** m, float** v, int64_t* t)
 {
     if (!h || h->async) return ZERO_ERR_ARG;

@@ -5,6 +5,8 @@ supplies the stream; libzero does all the work.
     skipped = opt.step(grads, loss_scale, lr=..., betas=..., eps=..., weight_decay=...)
     opt.gather_layer(unit, out)          # stage 3
     w, m, v = opt.state()                # live fp32 state (views of the workspace)
+    sd = opt.state_dict(); opt.load_state_dict(sd)     # checkpoint / resume
+    opt.begin_async(grads, scaler); opt.step_async(...); opt.end_async()
 """
 from __future__ import annotations
 
@@ -18,7 +20,7 @@ from . import _abi as A
 class ZeroAdam:
     def __init__(self, psi: int, nd: int, stage: int, master_init: torch.Tensor,
                  param_bufs: Sequence[torch.Tensor] | None = None, *, rank_view: int = -1,
-                 variant: int = A.ZERO_VARIANT_FUSED,
+                 variant: int = A.ZERO_VARIANT_FUSED_TMA,
                  tensors: Sequence[tuple[int, int]] | None = None,
                  stream: torch.cuda.Stream | None = None):
         self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors)
@@ -74,6 +76,39 @@ class ZeroAdam:
             raise ValueError("only stage 3 keeps fp16 shards")
         n = self.ledger.state_elems
         return self.workspace[off: off + 2 * n].view(torch.int16)
+
+    def state_dict(self) -> dict:
+        """Copies of master, m, v (state order) and the step count."""
+        w, m, v = self.state()
+        return {"master": w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
+
+    def load_state_dict(self, sd: dict) -> None:
+        tensors = [sd["master"], sd["m"], sd["v"]]
+        for x in tensors:
+            if x.dtype != torch.float32 or not x.is_cuda or x.numel() != self.ledger.state_elems:
+                raise ValueError("state tensors must be CUDA float32 of ledger.state_elems elements")
+        w, m, v = (x.contiguous() for x in tensors)
+        A.zero_set_state(self.h, w.data_ptr(), m.data_ptr(), v.data_ptr(), int(sd["t"]),
+                         self.stream.cuda_stream)
+
+    def begin_async(self, grads: Sequence[torch.Tensor], init_scale: float = 65536.0,
+                    growth_factor: float = 2.0, backoff_factor: float = 0.5,
+                    growth_interval: int = 2000, betas=(0.9, 0.999)) -> None:
+        """Open an asynchronous run on fixed gradient buffers (refill them
+        between steps): steps then run without host synchronisation, with a
+        dynamic loss scale kept on the device."""
+        sc = A.zero_scaler(init_scale, growth_factor, backoff_factor, growth_interval)
+        A.zero_async_begin(self.h, [g.data_ptr() for g in grads], sc, betas[0], betas[1],
+                           self.stream.cuda_stream)
+
+    def step_async(self, *, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0) -> None:
+        hp = A.zero_hyper(lr, betas[0], betas[1], eps, weight_decay)
+        A.zero_step_async(self.h, hp, self.stream.cuda_stream)
+
+    def end_async(self) -> dict:
+        st = A.zero_async_end(self.h, self.stream.cuda_stream)
+        return {"t": st.t, "skipped": st.skipped, "loss_scale": st.loss_scale,
+                "good_steps": st.good_steps}
 
     def close(self) -> None:
         if self.h:
