@@ -52,6 +52,9 @@ def parse_args():
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass"], default="fused-tma")
     p.add_argument("--async", dest="async_steps", action="store_true",
                    help="time zero_step_async: steps enqueued back to back, no host sync")
+    p.add_argument("--prefetch", action="store_true",
+                   help="stage 3: also time the layer gathers against a stand-in GEMM, "
+                        "one after the other vs prefetched on a side stream")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -464,6 +467,9 @@ def run_ours(args):
                            "bytes_per_step": gathers, "achieved_gbs": gathers / (g_ms / 1e3) / 1e9,
                            "frac": gathers / (g_ms / 1e3) / 1e9 / peak}
 
+    if args.prefetch and wl.stage == 3:
+        line["prefetch"] = prefetch_demo(h, L, order, gather_out)
+
     # ---- end to end through the public API from pinned host buffers ----
     if not args.no_e2e and args.e2e_steps > 0:
         line["e2e"] = e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world)
@@ -475,6 +481,66 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def prefetch_demo(h, L, order, gather_out, reps=5):
+    """Layer gathers of a forward + backward pass, each unit consumed by a
+    stand-in GEMM (tokens x d times the unit's first d x d weights), one after
+    the other on one stream vs with the next unit prefetched on a side stream
+    into a second transient buffer. Returns times and the measured peak."""
+    import torch
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+    from zero_partitioned_mixed_02_b200.prefetch import LayerPrefetcher
+
+    s = torch.cuda.current_stream()
+    d, tokens = 2560, 8192
+    x = torch.randn(tokens, d, dtype=torch.float16, device="cuda")
+
+    def consume(w):
+        return torch.mm(x, w[: d * d].view(torch.float16).view(d, d))
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(reps):
+            fn()
+        b.record(s)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    def sequential():
+        for u in order:
+            A.zero_gather_layer(h, u, gather_out.data_ptr(), s.cuda_stream)
+            consume(gather_out)
+
+    def gathers_only():
+        for u in order:
+            A.zero_gather_layer(h, u, gather_out.data_ptr(), s.cuda_stream)
+
+    def gemms_only():
+        for _ in order:
+            consume(gather_out)
+
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    pf = LayerPrefetcher(h, L, s)
+
+    def prefetched():
+        for _, w in pf.walk(order):
+            consume(w)
+
+    out = {"units": len(order), "tokens": tokens, "d": d,
+           "gathers_only_ms": timed(gathers_only), "gemms_only_ms": timed(gemms_only),
+           "sequential_ms": timed(sequential), "prefetched_ms": timed(prefetched),
+           "transient_bytes": L.transient_bytes, "prefetch_transient_bytes": pf.peak_bytes}
+    out["measured_peak_extra_bytes"] = torch.cuda.max_memory_allocated() - base
+    hidden = out["sequential_ms"] - out["prefetched_ms"]
+    out["gather_time_hidden_frac"] = hidden / out["gathers_only_ms"]
+    return out
 
 
 def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):

@@ -91,3 +91,23 @@ def test_zero_adam_object_matches_oracle_and_round_trips():
     gw2, _, _ = opt.state()
     compare_f32(host_f32(gw2), w, "master after load")
     opt.close()
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_FUSED_TMA])
+def test_prefetched_gathers_match_oracle(variant):
+    from zero_partitioned_mixed_02_b200.prefetch import LayerPrefetcher
+    nd = 4
+    sizes = [8 * nd * 900, 8 * nd * 40, 8 * nd * 1500, 8 * nd * 300, 777]
+    units = [0, 1, 1, 2, 2]
+    c = Case(sum(sizes), nd, 3, variant, tensors=list(zip(sizes, units)))
+    c.step(c.grads(0))
+    pf = LayerPrefetcher(c.h, c.L, torch.cuda.current_stream())
+    assert pf.peak_bytes == 2 * c.L.transient_bytes
+    order = [0, 1, 2, 2, 1, 0]  # forward, then backward
+    seen = []
+    for u, w in pf.walk(order, unit_numel=lambda u: A.zero_unit_range(c.cfg, u)[1]):
+        want = Z.zero3_gather(c.numel, c.units, nd, u, c.p_sh)
+        compare_f16(host_u16(w), want, f"prefetched unit {u}")
+        seen.append(u)
+    assert seen == order
+    c.close()

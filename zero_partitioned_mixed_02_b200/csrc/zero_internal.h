@@ -144,8 +144,14 @@ struct TmaArgs {
 // tensor) is copied shard -> output through shared memory in tiles of
 // kGatherTile elements, kGatherStages tiles in flight per CTA. TmaRun fields:
 // grad_begin = source (shard) index, out_begin = destination index.
-constexpr int kGatherTile = 8192;
-constexpr int kGatherStages = 4;
+#ifndef ZK_GATHER_TILE
+#define ZK_GATHER_TILE 8192
+#endif
+#ifndef ZK_GATHER_STAGES
+#define ZK_GATHER_STAGES 3
+#endif
+constexpr int kGatherTile = ZK_GATHER_TILE;
+constexpr int kGatherStages = ZK_GATHER_STAGES;
 
 struct TmaGatherArgs {
     const TmaRun* runs;
