@@ -200,6 +200,18 @@ int zr_dp_step(int64_t n, int32_t nd, const uint16_t* const* grads,
                float* w, float* m, float* v, uint16_t* p16,
                float loss_scale, const zr_hyper* hp, int64_t* t)
 {
+    return zr_dp_step_masked(n, nd, grads, w, m, v, p16, loss_scale, hp, NULL, t);
+}
+
+/* The same with weight decay applied only where decay[i] != 0 (decoupled
+ * weight decay, Loshchilov and Hutter; excluding some tensors, such as biases
+ * and normalisation gains, is a convention of AdamW setups, not of the pages).
+ * An excluded element takes the update with weight decay 0. */
+int zr_dp_step_masked(int64_t n, int32_t nd, const uint16_t* const* grads,
+                      float* w, float* m, float* v, uint16_t* p16,
+                      float loss_scale, const zr_hyper* hp, const uint8_t* decay,
+                      int64_t* t)
+{
     const float inv = zr_inv_scale(loss_scale);
     float* g = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
     int overflow = 0;
@@ -213,8 +225,11 @@ int zr_dp_step(int64_t n, int32_t nd, const uint16_t* const* grads,
     }
     *t = *t + 1;
     const coef_t c = make_coef(hp, *t);
+    coef_t c_nodecay = c;
+    c_nodecay.wd = 0.0f;
     for (int64_t i = 0; i < n; ++i) {
-        adam_element(g[i], &w[i], &m[i], &v[i], &c);
+        const coef_t* ci = (decay == NULL || decay[i] != 0) ? &c : &c_nodecay;
+        adam_element(g[i], &w[i], &m[i], &v[i], ci);
         p16[i] = zr_f16_from_f32(w[i]);
     }
     free(g);

@@ -70,6 +70,14 @@ int zr_dp_step(int64_t n, int32_t nd, const uint16_t* const* grads,
                float* w, float* m, float* v, uint16_t* p16,
                float loss_scale, const zr_hyper* hp, int64_t* t);
 
+/* zr_dp_step with decoupled weight decay only where decay[i] != 0 (decay may
+ * be NULL: every element decays); elements with decay[i] == 0 are updated with
+ * weight decay 0. */
+int zr_dp_step_masked(int64_t n, int32_t nd, const uint16_t* const* grads,
+                      float* w, float* m, float* v, uint16_t* p16,
+                      float loss_scale, const zr_hyper* hp, const uint8_t* decay,
+                      int64_t* t);
+
 /* ZeRO stage 1/2 with nd ranks: reduce-scatter, a global overflow flag,
  * Adam on each rank's own partition of master/m/v, then an all-gather of the
  * fp16 partitions into every rank's replica.  w_sh[r], m_sh[r], v_sh[r] hold

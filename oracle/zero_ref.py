@@ -47,6 +47,8 @@ _bias = _sig("zr_bias_corrections", None, _f32, _f32, _i64, C.POINTER(_f32), C.P
 _inv_scale = _sig("zr_inv_scale", _f32, _f32)
 _dp_step = _sig("zr_dp_step", C.c_int, _i64, _i32, _pp, _p, _p, _p, _p, _f32,
                 C.POINTER(Hyper), C.POINTER(_i64))
+_dp_step_masked = _sig("zr_dp_step_masked", C.c_int, _i64, _i32, _pp, _p, _p, _p, _p, _f32,
+                       C.POINTER(Hyper), _p, C.POINTER(_i64))
 _z12_step = _sig("zr_zero12_step", C.c_int, _i64, _i32, _pp, _pp, _pp, _pp, _pp, _f32,
                  C.POINTER(Hyper), C.POINTER(_i64))
 _z3_step = _sig("zr_zero3_step", C.c_int, _i32, _p, _i32, _pp, _pp, _pp, _pp, _pp, _f32,
@@ -133,16 +135,30 @@ def inv_scale(loss_scale: float) -> np.float32:
 
 
 # ---- the step ---------------------------------------------------------------
-def dp_step(grads: Sequence[np.ndarray], w, m, v, p16, loss_scale, hp: Hyper, t: int):
-    """Plain data-parallel definition. Returns (skipped, new_t)."""
+def dp_step(grads: Sequence[np.ndarray], w, m, v, p16, loss_scale, hp: Hyper, t: int,
+            decay=None):
+    """Plain data-parallel definition. Returns (skipped, new_t). `decay`: optional
+    per-element mask (nonzero = apply weight decay); None = every element."""
     gs = [_u16(g) for g in grads]
     n = w.size
     for g in gs:
         assert g.size == n
     tt = _i64(t)
-    sk = _dp_step(n, len(gs), _ptrs(gs), _ptr(w), _ptr(m), _ptr(v), _ptr(_u16(p16)),
-                  loss_scale, C.byref(hp), C.byref(tt))
+    if decay is None:
+        sk = _dp_step(n, len(gs), _ptrs(gs), _ptr(w), _ptr(m), _ptr(v), _ptr(_u16(p16)),
+                      loss_scale, C.byref(hp), C.byref(tt))
+    else:
+        dm = np.ascontiguousarray(decay, dtype=np.uint8)
+        assert dm.size == n
+        sk = _dp_step_masked(n, len(gs), _ptrs(gs), _ptr(w), _ptr(m), _ptr(v), _ptr(_u16(p16)),
+                             loss_scale, C.byref(hp), _ptr(dm), C.byref(tt))
     return bool(sk), tt.value
+
+
+def decay_mask(numel: Sequence[int], no_decay: Sequence[bool]) -> np.ndarray:
+    """Per-element mask of a tensor list: 0 on tensors excluded from weight decay."""
+    return np.concatenate([np.full(int(n), 0 if nd else 1, np.uint8)
+                           for n, nd in zip(numel, no_decay)])
 
 
 def zero12_step(psi, grads, w_sh, m_sh, v_sh, replicas, loss_scale, hp: Hyper, t: int):

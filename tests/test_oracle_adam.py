@@ -304,3 +304,92 @@ def test_stage3_skip_is_global():
     # inf on rank 2 in tensor 0's chunk owned by rank 0
     res = _zero3_run(numel, 3, 2, rng, Z.hyper(), 4.0, inject=(0, 2, 0))
     assert res is not None
+
+
+# ---- per-tensor weight-decay exclusion -------------------------------------
+# Decoupled weight decay (Loshchilov and Hutter) applied to some tensors only:
+# an excluded tensor takes the Adam update with weight decay 0.
+
+def _mask_case(seed, n_tensors=7):
+    rng = np.random.default_rng(seed)
+    numel = rng.integers(1, 60, n_tensors)
+    no_decay = [bool(i % 2) for i in range(n_tensors)]
+    return rng, [int(x) for x in numel], no_decay
+
+
+def test_masked_decay_matches_torch_param_groups():
+    """Against torch.optim.AdamW in float64 with two parameter groups (weight
+    decay on the decayed tensors, 0 on the excluded ones)."""
+    rng, numel, no_decay = _mask_case(11)
+    n, nd, steps, scale = sum(numel), 4, 4, 1024.0
+    hp = Z.hyper(lr=1e-3, weight_decay=0.1)
+    mask = Z.decay_mask(numel, no_decay)
+    w = rng.uniform(-0.5, 0.5, n).astype(np.float32)
+    w0 = w.copy()
+    m, v, p16 = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
+    t, unscaled, gmax = 0, [], np.zeros(n)
+    for _ in range(steps):
+        gs = _grads(rng, nd, n, sigma=1e-3, scale=scale)
+        s = Z.f32_from_f16(gs[0])
+        for g in gs[1:]:
+            s = (s + Z.f32_from_f16(g)).astype(np.float32)
+        unscaled.append(s.astype(np.float64) / scale)
+        gmax = np.maximum(gmax, np.abs(unscaled[-1]))
+        sk, t = Z.dp_step(gs, w, m, v, p16, scale, hp, t, decay=mask)
+        assert not sk
+    # torch: one parameter per tensor, grouped by exclusion
+    offs = np.concatenate([[0], np.cumsum(numel)])
+    params = [torch.nn.Parameter(torch.from_numpy(w0[offs[i]:offs[i + 1]].astype(np.float64)))
+              for i in range(len(numel))]
+    groups = [{"params": [p for p, x in zip(params, no_decay) if not x],
+               "weight_decay": float(np.float32(hp.weight_decay))},
+              {"params": [p for p, x in zip(params, no_decay) if x], "weight_decay": 0.0}]
+    opt = torch.optim.AdamW(groups, lr=float(np.float32(hp.lr)),
+                            betas=(float(np.float32(0.9)), float(np.float32(0.999))),
+                            eps=float(np.float32(1e-8)), foreach=False)
+    for g in unscaled:
+        for i, p in enumerate(params):
+            p.grad = torch.from_numpy(g[offs[i]:offs[i + 1]].copy())
+        opt.step()
+    tw = np.concatenate([p.detach().numpy() for p in params])
+    assert _rel_close(w, tw, 1e-6)
+    # the excluded tensors really differ from a run that decays everything
+    w_all = w0.copy()
+    rng2, _, _ = _mask_case(11)
+    rng2.uniform(-0.5, 0.5, n)
+    m2, v2, t2 = np.zeros(n, np.float32), np.zeros(n, np.float32), 0
+    for _ in range(steps):
+        gs = _grads(rng2, nd, n, sigma=1e-3, scale=scale)
+        _, t2 = Z.dp_step(gs, w_all, m2, v2, p16.copy(), scale, hp, t2)
+    excl = mask == 0
+    assert (w_all[excl] != w[excl]).any()
+    assert (w_all[~excl].view(np.uint32) == w[~excl].view(np.uint32)).all()
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_masked_decay_is_elementwise_selection(seed):
+    """Elements are independent: a masked step equals, element by element, the
+    unmasked step with the weight decay or with weight decay 0, bit for bit;
+    an all-ones mask equals no mask."""
+    rng, numel, no_decay = _mask_case(seed, n_tensors=9)
+    n, nd = sum(numel), 3
+    mask = Z.decay_mask(numel, no_decay)
+    w0 = rng.uniform(-2, 2, n).astype(np.float32)
+    m0 = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    v0 = (rng.uniform(0, 1e-6, n)).astype(np.float32)
+    gs = _grads(rng, nd, n, sigma=1e-3, scale=256.0)
+    hp = Z.hyper(lr=1e-2, weight_decay=0.05)
+    hp0 = Z.hyper(lr=1e-2, weight_decay=0.0)
+    out = {}
+    for name, h, dm in (("masked", hp, mask), ("ones", hp, np.ones(n, np.uint8)),
+                        ("wd", hp, None), ("nowd", hp0, None)):
+        w, m, v, p = w0.copy(), m0.copy(), v0.copy(), np.zeros(n, np.uint16)
+        sk, t = Z.dp_step(gs, w, m, v, p, 256.0, h, 2, decay=dm)
+        assert not sk and t == 3
+        out[name] = (w, m, v, p)
+    sel = mask != 0
+    for k in range(4):
+        expect = np.where(sel, out["wd"][k], out["nowd"][k])
+        assert (out["masked"][k].view(np.uint8) == expect.view(np.uint8)).all()
+        assert (out["ones"][k].view(np.uint8) == out["wd"][k].view(np.uint8)).all()
+    assert (out["wd"][0] != out["nowd"][0]).any()
