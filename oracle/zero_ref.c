@@ -76,6 +76,67 @@ uint16_t zr_f16_from_f64(double x)
 
 uint16_t zr_f16_from_f32(float x) { return zr_f16_from_f64((double)x); }
 
+/* ======================================================================
+ * bfloat16 <-> binary32: 1 sign bit, 8 exponent bits (bias 127), 7 fraction
+ * bits ([P3] "Why parameter count is not training memory": not every BF16
+ * setup keeps fp32 master weights).
+ * ==================================================================== */
+
+float zr_f32_from_bf16(uint16_t h)
+{
+    const int neg = (h >> 15) & 1;
+    const int e = (h >> 7) & 0xff;
+    const int f = h & 0x7f;
+    double mag;
+    if (e == 0xff) {
+        if (f != 0) return neg ? -NAN : NAN;
+        mag = INFINITY;
+    } else if (e == 0) {
+        mag = ldexp((double)f, -133);             /* subnormal: f * 2^-133 */
+    } else {
+        mag = ldexp((double)(128 + f), e - 134);  /* (1 + f/128) * 2^(e-127) */
+    }
+    return (float)(neg ? -mag : mag);
+}
+
+/* Round x to the nearest bfloat16 value, ties to even, by counting quanta. */
+uint16_t zr_bf16_from_f64(double x)
+{
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    if (isnan(x)) return sign | 0x7fc0;
+    const double a = fabs(x);
+    /* the largest finite value is (2 - 2^-7) 2^127; from the halfway point
+     * (2 - 2^-8) 2^127 on, the nearest even neighbour is 2^128: overflow */
+    if (a >= ldexp(2.0 - ldexp(1.0, -8), 127)) return sign | 0x7f80;
+    int q_exp;
+    if (a >= 0x1p-126) {
+        int e;
+        frexp(a, &e);
+        q_exp = (e - 1) - 7;  /* 7 fraction bits below the leading bit */
+    } else {
+        q_exp = -133;         /* subnormal spacing */
+    }
+    const double n = rint(ldexp(a, -q_exp));
+    if (n == 0.0) return sign;
+    if (q_exp == -133) return sign | (uint16_t)n; /* n = 128 encodes 2^-126 */
+    int biased = q_exp + 7 + 127;
+    double sig = n;
+    if (sig == 256.0) { sig = 128.0; biased += 1; }
+    return sign | (uint16_t)(biased << 7) | (uint16_t)((int)sig - 128);
+}
+
+uint16_t zr_bf16_from_f32(float x) { return zr_bf16_from_f64((double)x); }
+
+void zr_f32_from_bf16_array(const uint16_t* h, float* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = zr_f32_from_bf16(h[i]);
+}
+
+void zr_bf16_from_f32_array(const float* x, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = zr_bf16_from_f32(x[i]);
+}
+
 void zr_f32_from_f16_array(const uint16_t* h, float* out, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = zr_f32_from_f16(h[i]);
@@ -231,6 +292,41 @@ int zr_dp_step_masked(int64_t n, int32_t nd, const uint16_t* const* grads,
         const coef_t* ci = (decay == NULL || decay[i] != 0) ? &c : &c_nodecay;
         adam_element(g[i], &w[i], &m[i], &v[i], ci);
         p16[i] = zr_f16_from_f32(w[i]);
+    }
+    free(g);
+    return 0;
+}
+
+/* The step of a BF16 setup without fp32 master weights ([P3] "Why parameter
+ * count is not training memory"): gradients and parameters are bfloat16, the
+ * Adam moments binary32. The reduction and the element update are the ones
+ * above; the parameter is read from and rounded back to bfloat16 every step,
+ * so K = 8 bytes of optimizer state per parameter instead of 12. */
+int zr_bf16_step(int64_t n, int32_t nd, const uint16_t* const* grads, uint16_t* w16,
+                 float* m, float* v, float loss_scale, const zr_hyper* hp,
+                 const uint8_t* decay, int64_t* t)
+{
+    const float inv = zr_inv_scale(loss_scale);
+    float* g = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    int overflow = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        float s = zr_f32_from_bf16(grads[0][i]);
+        for (int32_t r = 1; r < nd; ++r) s = s + zr_f32_from_bf16(grads[r][i]);
+        g[i] = s * inv;
+        if (!isfinite(g[i])) overflow = 1;
+    }
+    if (overflow) {
+        free(g);
+        return 1;
+    }
+    *t = *t + 1;
+    const coef_t c = make_coef(hp, *t);
+    coef_t c_nodecay = c;
+    c_nodecay.wd = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float w = zr_f32_from_bf16(w16[i]);
+        adam_element(g[i], &w, &m[i], &v[i], (decay == NULL || decay[i] != 0) ? &c : &c_nodecay);
+        w16[i] = zr_bf16_from_f32(w);
     }
     free(g);
     return 0;

@@ -45,6 +45,13 @@ void     zr_f16_from_f32_array(const float* x, uint16_t* out, int64_t n);
 uint16_t zr_direct_f16_update(uint16_t w16, float dw);
 void     zr_direct_f16_update_array(const uint16_t* w16, const float* dw, uint16_t* out, int64_t n);
 
+/* ---- bfloat16 conversions (round to nearest, ties to even) ---- */
+float    zr_f32_from_bf16(uint16_t h);
+uint16_t zr_bf16_from_f32(float x);
+uint16_t zr_bf16_from_f64(double x);
+void     zr_f32_from_bf16_array(const uint16_t* h, float* out, int64_t n);
+void     zr_bf16_from_f32_array(const float* x, uint16_t* out, int64_t n);
+
 /* ---- partitions ---- */
 /* Stage 1/2: rank r of nd owns flat [r*P, min((r+1)*P, psi)), P = ceil(psi/nd). */
 void zr_partition(int64_t psi, int32_t nd, int32_t r, int64_t* begin, int64_t* end);
@@ -77,6 +84,14 @@ int zr_dp_step_masked(int64_t n, int32_t nd, const uint16_t* const* grads,
                       float* w, float* m, float* v, uint16_t* p16,
                       float loss_scale, const zr_hyper* hp, const uint8_t* decay,
                       int64_t* t);
+
+/* A BF16 setup without fp32 master weights: nd bfloat16 gradients summed in
+ * binary32 in rank order and unscaled, the same skip rule, then per element
+ * w = fp32(w16); Adam on (w, m, v) as in zr_dp_step (decay mask as in
+ * zr_dp_step_masked); w16 = bf16(w). Returns 1 on overflow (nothing changes). */
+int zr_bf16_step(int64_t n, int32_t nd, const uint16_t* const* grads, uint16_t* w16,
+                 float* m, float* v, float loss_scale, const zr_hyper* hp,
+                 const uint8_t* decay, int64_t* t);
 
 /* ZeRO stage 1/2 with nd ranks: reduce-scatter, a global overflow flag,
  * Adam on each rank's own partition of master/m/v, then an all-gather of the

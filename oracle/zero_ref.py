@@ -49,6 +49,13 @@ _dp_step = _sig("zr_dp_step", C.c_int, _i64, _i32, _pp, _p, _p, _p, _p, _f32,
                 C.POINTER(Hyper), C.POINTER(_i64))
 _dp_step_masked = _sig("zr_dp_step_masked", C.c_int, _i64, _i32, _pp, _p, _p, _p, _p, _f32,
                        C.POINTER(Hyper), _p, C.POINTER(_i64))
+_f32_from_bf16 = _sig("zr_f32_from_bf16", _f32, C.c_uint16)
+_bf16_from_f32 = _sig("zr_bf16_from_f32", C.c_uint16, _f32)
+_bf16_from_f64 = _sig("zr_bf16_from_f64", C.c_uint16, C.c_double)
+_f32_from_bf16_array = _sig("zr_f32_from_bf16_array", None, _p, _p, _i64)
+_bf16_from_f32_array = _sig("zr_bf16_from_f32_array", None, _p, _p, _i64)
+_bf16_step = _sig("zr_bf16_step", C.c_int, _i64, _i32, _pp, _p, _p, _p, _f32, C.POINTER(Hyper), _p,
+                  C.POINTER(_i64))
 _z12_step = _sig("zr_zero12_step", C.c_int, _i64, _i32, _pp, _pp, _pp, _pp, _pp, _f32,
                  C.POINTER(Hyper), C.POINTER(_i64))
 _z3_step = _sig("zr_zero3_step", C.c_int, _i32, _p, _i32, _pp, _pp, _pp, _pp, _pp, _f32,
@@ -159,6 +166,37 @@ def decay_mask(numel: Sequence[int], no_decay: Sequence[bool]) -> np.ndarray:
     """Per-element mask of a tensor list: 0 on tensors excluded from weight decay."""
     return np.concatenate([np.full(int(n), 0 if nd else 1, np.uint8)
                            for n, nd in zip(numel, no_decay)])
+
+
+def f32_from_bf16(h) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _f32_from_bf16_array(_ptr(h), _ptr(out), h.size)
+    return out
+
+
+def bf16_from_f32(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _bf16_from_f32_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def bf16_from_f64_scalar(x: float) -> int:
+    return int(_bf16_from_f64(float(x)))
+
+
+def bf16_step(grads: Sequence[np.ndarray], w16, m, v, loss_scale, hp: Hyper, t: int, decay=None):
+    """BF16 step without fp32 master weights; w16 (uint16 bfloat16 bits), m, v
+    updated in place. Returns (skipped, new_t)."""
+    gs = [np.ascontiguousarray(g, dtype=np.uint16) for g in grads]
+    n = m.size
+    assert w16.dtype == np.uint16 and w16.size == n and all(g.size == n for g in gs)
+    dm = None if decay is None else np.ascontiguousarray(decay, dtype=np.uint8)
+    tt = _i64(t)
+    sk = _bf16_step(n, len(gs), _ptrs(gs), _ptr(w16), _ptr(m), _ptr(v), loss_scale, C.byref(hp),
+                    None if dm is None else _ptr(dm), C.byref(tt))
+    return bool(sk), tt.value
 
 
 def zero12_step(psi, grads, w_sh, m_sh, v_sh, replicas, loss_scale, hp: Hyper, t: int):
