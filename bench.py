@@ -50,11 +50,20 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass"], default="fused-tma")
+    p.add_argument("--precision", choices=["fp16", "bf16"], default="fp16",
+                   help="bf16: bfloat16 gradients and parameters without fp32 master weights "
+                        "(runs the two-pass kernels)")
     p.add_argument("--async", dest="async_steps", action="store_true",
                    help="time zero_step_async: steps enqueued back to back, no host sync")
     p.add_argument("--prefetch", action="store_true",
                    help="stage 3: also time the layer gathers against a stand-in GEMM, "
                         "one after the other vs prefetched on a side stream")
+    p.add_argument("--offload", action="store_true",
+                   help="time the offloaded step (fp32 state and Adam on the host) instead")
+    p.add_argument("--offload-threads", type=int, default=0,
+                   help="host threads of the offloaded update (0: every core this process may use)")
+    p.add_argument("--offload-chunk", type=int, default=0,
+                   help="elements per pipeline chunk of the offloaded step (0: the library default)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -77,15 +86,18 @@ def owned_range(wl):
     return 0, wl.psi
 
 
-def algorithmic_bytes(wl, variant):
+def algorithmic_bytes(wl, variant, bf16=False):
     """Minimum bytes one step of the method must move (the floor), and per
     launch of the dominant kernel. n = elements this GPU updates."""
     b0, e0 = owned_range(wl)
     n = e0 - b0
-    grads = 2 * wl.nd * n                    # every rank's fp16 gradient of each element
-    state = 24 * n                           # fp32 master, m, v read and written
+    grads = 2 * wl.nd * n                    # every rank's 16-bit gradient of each element
     n_out = wl.nd if (wl.stage <= 2 and wl.rank_view < 0) else 1
-    params = 2 * n * n_out                   # fp16 write-back to every replica / the shard
+    if bf16:
+        state = 16 * n + 2 * n               # fp32 m, v read and written; the bf16 weight read
+    else:
+        state = 24 * n                       # fp32 master, m, v read and written
+    params = 2 * n * n_out                   # 16-bit write-back to every replica / the shard
     floor = grads + state + params
     if variant in ("fused", "fused-tma"):
         per_launch = {"step_kernel<fused>": floor}
@@ -214,9 +226,21 @@ def oracle_sample_step(wl, n_s, step, state):
     from zero_partitioned_mixed_02_b200 import synth as S
 
     b0, _ = owned_range(wl)
+    hp = Z.hyper(**wl.hyper)
+    if state.get("bf16"):
+        # bfloat16 without master: the definition on the sample (ZeRO does not
+        # change the math), gradients rounded to bfloat16 from the generator
+        gs = [Z.bf16_from_f32(S.host_f32(n_s, b0, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad))
+              for k in range(wl.nd)]
+        if state.get("w16") is None:
+            w0 = S.host_f32(n_s, b0, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master)
+            state["w16"] = Z.bf16_from_f32(w0)
+            state["m"], state["v"], state["t"] = np.zeros(n_s, np.float32), np.zeros(n_s, np.float32), 0
+        t0 = time.perf_counter()
+        _, state["t"] = Z.bf16_step(gs, state["w16"], state["m"], state["v"], wl.loss_scale, hp, state["t"])
+        return time.perf_counter() - t0
     gs = [S.host_f16_bits(n_s, b0, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad)
           for k in range(wl.nd)]
-    hp = Z.hyper(**wl.hyper)
     if state.get("w") is None:
         w0 = S.host_f32(n_s, b0, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master)
         if wl.stage <= 2 and wl.rank_view < 0:
@@ -260,17 +284,17 @@ def oracle_sample_step(wl, n_s, step, state):
     return time.perf_counter() - t0
 
 
-def calibrate_sample(wl, seconds):
+def calibrate_sample(wl, seconds, bf16=False):
     n0 = 1 << 17
-    dt = oracle_sample_step(wl, n0, 0, {})
+    dt = oracle_sample_step(wl, n0, 0, {"bf16": bf16})
     rate = n0 / max(dt, 1e-6)
     b0, e0 = owned_range(wl)
     return int(max(4096, min(e0 - b0, rate * seconds)))
 
 
-def cpu_baseline(wl, seconds):
-    n_s = calibrate_sample(wl, seconds)
-    dt = oracle_sample_step(wl, n_s, 0, {})
+def cpu_baseline(wl, seconds, bf16=False):
+    n_s = calibrate_sample(wl, seconds, bf16)
+    dt = oracle_sample_step(wl, n_s, 0, {"bf16": bf16})
     model, ncpu = cpu_info()
     return {"value": n_s / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"first {n_s} of the workload's {owned_range(wl)[1] - owned_range(wl)[0]} "
@@ -300,7 +324,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": config_of(wl, args.variant),
+        "config": {**config_of(wl, args.variant), "precision": args.precision},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample, "host_cpu": model, "host_cpus": ncpu},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -336,10 +360,14 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     wl = workload(args.workload)
+    bf16 = args.precision == "bf16"
+    if bf16:
+        args.variant = "two-pass"  # without a master only the two-pass step exists
     variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
                "fused-tma": A.ZERO_VARIANT_FUSED_TMA}[args.variant]
     cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, variant=variant,
-                   tensors=wl.tensors)
+                   tensors=wl.tensors,
+                   precision=A.ZERO_PRECISION_BF16 if bf16 else A.ZERO_PRECISION_FP16)
     L = A.zero_state_bytes(cfg)
     b0, e0 = owned_range(wl)
     n_own = e0 - b0
@@ -354,7 +382,14 @@ def run_ours(args):
                 for _ in range(wl.nd if wl.rank_view < 0 else 1)]
     grads = [torch.empty(n_own, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
     for k in range(wl.nd):
-        S.fill_f16(grads[k].data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, 0, k), wl.grad, s)
+        if bf16:
+            # the generator's binary32 values rounded to bfloat16 (nearest even)
+            tmp = torch.empty(n_own, dtype=torch.float32, device="cuda")
+            S.fill_f32(tmp.data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, 0, k), wl.grad, s)
+            grads[k].copy_(tmp.to(torch.bfloat16).view(torch.int16))
+            del tmp
+        else:
+            S.fill_f16(grads[k].data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, 0, k), wl.grad, s)
     h = A.zero_init(cfg, ws.data_ptr(), L.workspace_bytes, m_init.data_ptr(),
                     [b.data_ptr() for b in bufs] if bufs else None, s)
     del m_init
@@ -428,7 +463,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
 
-    n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant)
+    n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant, bf16)
     launches_per_step = (2 if args.variant == "two-pass" else 1) + len(order)
     if args.async_steps:  # + the conditional roll-back (fused variants) and the commit kernel
         launches_per_step += 1 if args.variant == "two-pass" else 2
@@ -439,8 +474,10 @@ def run_ours(args):
     k_s = statistics.mean(kern_ms) / 1e3
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
-    traffic = recorded_traffic(args.workload, args.variant)
-    if args.variant == "two-pass":
+    traffic = None if bf16 else recorded_traffic(args.workload, args.variant)
+    if bf16:
+        kname = "step_kernel<reduce,bf16>+<update,bf16>"
+    elif args.variant == "two-pass":
         kname = "step_kernel<reduce>+<update>"
     elif A.zero_uses_tma(h):
         kname = "step_tma_kernel"
@@ -476,7 +513,7 @@ def run_ours(args):
     A.zero_destroy(h)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, bf16)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -608,10 +645,128 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
             "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
 
 
+def host_copy_gbs(threads, n_bytes=1 << 31, reps=5):
+    """Host memory bandwidth reference for the offloaded update: a torch copy
+    of n_bytes on `threads` threads, read + written bytes per second (best of
+    reps)."""
+    import torch
+
+    old = torch.get_num_threads()
+    torch.set_num_threads(threads)
+    a = torch.ones(n_bytes // 4, dtype=torch.float32)
+    b = torch.empty_like(a)
+    b.copy_(a)
+    best = float("inf")
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        b.copy_(a)
+        best = min(best, time.perf_counter() - t0)
+    torch.set_num_threads(old)
+    return 2 * n_bytes / best / 1e9
+
+
+def run_offload(args):
+    """The offloaded step on the workload: fp32 master/m/v in host memory, Adam
+    on the host cores, reduce and fp16 write-back on the GPU, chunks pipelined
+    over PCIe. Timed with CUDA events on the caller's stream, which bracket
+    every device and host part of each step (the device work of a step waits
+    for the host update of its chunks)."""
+    import numpy as np
+    import torch
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+    from zero_partitioned_mixed_02_b200 import synth as S
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--offload runs on one GPU")
+    torch.cuda.set_device(0)
+    wl = workload(args.workload)
+    cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, tensors=wl.tensors)
+    L = A.zero_offload_bytes(cfg, args.offload_chunk)
+    threads = args.offload_threads or len(os.sched_getaffinity(0))
+    threads = max(1, min(threads, 256))
+    b0, e0 = owned_range(wl)
+    n_own = e0 - b0
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    m_dev = torch.empty(n_own, dtype=torch.float32, device="cuda")
+    S.fill_f32(m_dev.data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master, s)
+    master_init = m_dev.cpu().numpy()
+    del m_dev
+    E = L.state_elems
+    state = np.empty(3 * E, np.float32)
+    dws = torch.empty(L.device_bytes, dtype=torch.uint8, device="cuda")
+    staging = torch.empty(L.host_staging_bytes, dtype=torch.uint8, pin_memory=True)
+    if wl.stage <= 2:
+        bufs = [torch.empty(wl.psi, dtype=torch.int16, device="cuda")
+                for _ in range(wl.nd if wl.rank_view < 0 else 1)]
+    else:
+        bufs = [torch.empty(E, dtype=torch.int16, device="cuda")]
+    grads = [torch.empty(n_own, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    for k in range(wl.nd):
+        S.fill_f16(grads[k].data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, 0, k), wl.grad, s)
+    t_init = time.perf_counter()
+    h = A.zero_offload_init(cfg, args.offload_chunk, dws.data_ptr(), L.device_bytes, staging.data_ptr(),
+                            L.host_staging_bytes, state.ctypes.data, master_init.ctypes.data,
+                            [b.data_ptr() for b in bufs], threads, s)
+    t_init = time.perf_counter() - t_init
+    del master_init
+    gptrs = [g.data_ptr() for g in grads]
+    hp = A.zero_hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay)
+    for _ in range(args.warmup):
+        if A.zero_offload_step(h, gptrs, wl.loss_scale, hp, s) != A.ZERO_OK:
+            raise RuntimeError("unexpected skip in the benchmark workload")
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    ev = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if A.zero_offload_step(h, gptrs, wl.loss_scale, hp, s) != A.ZERO_OK:
+            raise RuntimeError("unexpected skip in the benchmark workload")
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(ms)
+    A.zero_offload_destroy(h)
+    host_copy = host_copy_gbs(threads)
+    step_s = total_ms / 1e3 / args.steps
+    Ld = A.zero_state_bytes(cfg)
+    pcie = L.d2h_bytes_per_step + L.h2d_bytes_per_step
+    line = {
+        "metric": METRIC, "value": E * args.steps / (total_ms / 1e3) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "ms_per_step_min": min(ms), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic", "mode": "offload",
+        "config": {**config_of(wl, "offload"), "variant": "offload"},
+        "offload": {
+            "host_threads": threads, "chunk_elems": L.chunk_elems, "n_chunks": L.n_chunks,
+            "slots": A.ZERO_OFFLOAD_SLOTS, "init_s": t_init,
+            "d2h_bytes_per_step": L.d2h_bytes_per_step, "h2d_bytes_per_step": L.h2d_bytes_per_step,
+            "pcie_gbs": pcie / step_s / 1e9,
+            # host memory traffic of the update: read g, w, m, v; write w, m, v, p16
+            "host_update_gbs": 30 * E / step_s / 1e9,
+            "host_copy_gbs": host_copy,
+            "host_update_frac_of_copy": 30 * E / step_s / 1e9 / host_copy,
+            "host_state_bytes": L.host_state_bytes,
+            "device_state_bytes_per_rank": L.device_state_bytes,
+            "device_state_bytes_per_rank_without_offload": int(Ld.exact_bytes[wl.stage]),
+        },
+        "gpu_launches": (1 + 2 * L.n_chunks) * args.steps,
+        "clocks": clock_info,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.offload:
+        run_offload(args)
     else:
         run_ours(args)
 

@@ -22,7 +22,8 @@
  *   skip the whole step if any g over all partitions is inf or NaN
  *   m   = b1*m + (1-b1)*g ;  v = b2*v + (1-b2)*(g*g)
  *   u   = (m / bc1) / (sqrt(v / bc2) + eps),  bc_k = (float)(1 - beta_k^t)
- *   w   = w - lr*(u + wd*w)                              (fp32 master)
+ *   w   = w - lr*(u + wd*w)                              (fp32 master;
+ *         wd = 0 on tensors flagged ZERO_TENSOR_NO_DECAY)
  *   p16 = fp16(w), round to nearest even, written to every rank's replica
  *         (stage 1/2) or to rank r's fp16 shard (stage 3).
  * Each binary32 operation is one IEEE-rounded operation in that order (no FMA
@@ -88,13 +89,38 @@ extern "C" {
 
 #define ZERO_MAX_ND 1024
 
+/* ---- precision of the parameters and gradients ---- */
+/* fp16 gradients and parameters, fp32 master weights and Adam moments:
+ * K = 12 bytes of optimizer state per parameter ([P1] "Where 16 bytes per
+ * parameter comes from"). */
+#define ZERO_PRECISION_FP16 0
+/* bfloat16 gradients and parameters and NO fp32 master ([P3] "Why parameter
+ * count is not training memory": not every BF16 setup keeps master weights):
+ * fp32 m and v only, K = 8. Each step reads the weight from the bfloat16
+ * parameter, runs the same binary32 Adam element and rounds the result back
+ * to bfloat16 (nearest even) into every replica / the shard. Updates smaller
+ * than half a bfloat16 spacing are lost ([P1] "Why you can't just delete the
+ * fp32 copies" describes the same loss for fp16). Requires
+ * ZERO_VARIANT_TWO_PASS (without a master a speculative write cannot be rolled
+ * back). master_init of zero_init is rounded to bfloat16; the ledger's master
+ * offsets are -1 and zero_current_state returns master = NULL; for
+ * zero_set_state master may be NULL (the parameters stay as they are) or
+ * fp32 values in state order to round into the parameters. */
+#define ZERO_PRECISION_BF16 1
+
+/* Tensor flag: exclude the tensor from weight decay (it takes the Adam update
+ * with wd = 0). Decoupled weight decay (Loshchilov and Hutter) is commonly not
+ * applied to biases and normalisation gains; the pages do not discuss it.
+ * Numerics are unchanged for tensors without the flag. */
+#define ZERO_TENSOR_NO_DECAY 1
+
 /* One tensor of the flat parameter vector, in flat order. `unit` is the layer
  * unit a stage-3 gather rebuilds (units are numbered 0, 1, ... and appear in
  * non-decreasing order along the tensor list). */
 typedef struct zero_tensor {
     int64_t numel;
     int32_t unit;
-    int32_t reserved; /* must be 0 */
+    int32_t flags; /* 0 or ZERO_TENSOR_NO_DECAY; other bits: ZERO_ERR_ARG */
 } zero_tensor;
 
 typedef struct zero_config {
@@ -105,7 +131,7 @@ typedef struct zero_config {
                           act as rank r alone, owning partition r */
     int32_t variant;   /* ZERO_VARIANT_FUSED, _TWO_PASS or _FUSED_TMA */
     int32_t n_tensors; /* 0 allowed for stage 1/2 (one flat tensor) */
-    int32_t reserved;  /* must be 0 */
+    int32_t precision; /* ZERO_PRECISION_FP16 (0) or ZERO_PRECISION_BF16 */
     const zero_tensor* tensors; /* host array of n_tensors; sum of numel == psi;
                                    required for stage 3 */
 } zero_config;

@@ -116,7 +116,8 @@ class GuardedWorkspace:
 def state_offsets(h: int, ws: GuardedWorkspace) -> tuple[int, int, int, int]:
     w, m, v, t = A.zero_current_state(h)
     base = ws.ptr()
-    return w - base, m - base, v - base, t
+    # no master (bfloat16 without master weights): None
+    return (None if w is None else w - base), m - base, v - base, t
 
 
 def hyper(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0) -> A.zero_hyper:

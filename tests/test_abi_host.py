@@ -142,6 +142,8 @@ def test_workspace_layout():
     dict(psi=10, nd=2, stage=3, tensors=[(4, 1), (6, 1)]),  # units must start at 0
     dict(psi=10, nd=2, stage=3, tensors=[(4, 0), (6, 2)]),  # units must be contiguous
     dict(psi=10, nd=A.ZERO_MAX_ND + 1, stage=1),
+    dict(psi=10, nd=2, stage=2, tensors=[(4, 0, 2), (6, 0)]),  # unknown tensor flag
+    dict(psi=10, nd=2, stage=3, tensors=[(4, 0, -1), (6, 1)]),
 ])
 def test_invalid_configs_rejected(kw):
     cfg = A.Config(**kw)
@@ -174,3 +176,48 @@ def test_init_validation_before_device_work():
 def test_error_strings():
     for code in (0, 1, -1, -2, -3, -4, -5, -6):
         assert A.error_string(code) and A.error_string(code) != "unknown error code"
+
+
+def test_no_decay_flag_accepted_and_layout_unchanged_in_size_order():
+    """The weight-decay flag does not change the ledger; it only adds run
+    table entries (a few bytes of workspace)."""
+    ND = A.ZERO_TENSOR_NO_DECAY
+    for stage in (1, 2, 3):
+        plain = [(1000, 0), (17, 0), (3000, 1), (5, 1)]
+        flagged = [(1000, 0), (17, 0, ND), (3000, 1), (5, 1, ND)]
+        a = A.zero_state_bytes(A.Config(4022, 3, stage, tensors=plain))
+        b = A.zero_state_bytes(A.Config(4022, 3, stage, tensors=flagged))
+        assert list(a.exact_bytes) == list(b.exact_bytes)
+        assert a.state_elems == b.state_elems and a.transient_bytes == b.transient_bytes
+        assert b.workspace_bytes >= a.workspace_bytes
+        assert b.workspace_bytes - a.workspace_bytes <= 4096
+
+
+def test_bf16_precision_ledger_and_validation():
+    """Without fp32 master weights K = 8 ([P3] "Why parameter count is not
+    training memory"; [P2] "The Mathematics": (2 + 2 + K) Psi)."""
+    BF = A.ZERO_PRECISION_BF16
+    tensors = [(1000, 0), (17, 1), (3001, 1)]
+    psi, nd = 4018, 3
+    numel = [n for n, _ in tensors]
+    P = max(e - b for b, e in (Z.partition(psi, nd, r) for r in range(nd)))
+    S = max(sum(e - b for b, e in (Z.chunk(n, nd, r) for n in numel)) for r in range(nd))
+    for stage in (1, 2, 3):
+        L = A.zero_state_bytes(A.Config(psi, nd, stage, variant=A.ZERO_VARIANT_TWO_PASS,
+                                        tensors=tensors, precision=BF))
+        assert list(L.exact_bytes) == [12 * psi, 4 * psi + 8 * P, 2 * psi + 10 * P, 12 * S]
+        f = list(L.formula_bytes)
+        assert f == pytest.approx([12 * psi, 4 * psi + 8 * psi / nd, 2 * psi + 10 * psi / nd,
+                                   12 * psi / nd], rel=1e-12)
+        assert list(L.off_master) == [-1, -1] and L.off_m[0] >= 0 and L.off_v[0] >= 0
+        L16 = A.zero_state_bytes(A.Config(psi, nd, stage, variant=A.ZERO_VARIANT_TWO_PASS,
+                                          tensors=tensors))
+        # the master array is gone from the workspace
+        assert L16.workspace_bytes - L.workspace_bytes >= 4 * psi
+    for kw in (dict(precision=2), dict(precision=BF, variant=A.ZERO_VARIANT_FUSED),
+               dict(precision=BF, variant=A.ZERO_VARIANT_FUSED_TMA)):
+        with pytest.raises(A.ZeroError) as ei:
+            A.zero_state_bytes(A.Config(psi, nd, 2, **kw))
+        assert ei.value.code == A.ZERO_ERR_ARG
+    with pytest.raises(A.ZeroError):
+        A.zero_offload_bytes(A.Config(psi, nd, 2, variant=A.ZERO_VARIANT_TWO_PASS, precision=BF))

@@ -46,8 +46,8 @@ class Case:
                  hp=None, grad_dist=None, master_dist=None, seed=0):
         self.psi, self.nd, self.stage, self.variant, self.view = psi, nd, stage, variant, view
         self.tensors = tensors
-        self.numel = [n for n, _ in tensors] if tensors else [psi]
-        self.units = [u for _, u in tensors] if tensors else [0]
+        self.numel = [t[0] for t in tensors] if tensors else [psi]
+        self.units = [t[1] for t in tensors] if tensors else [0]
         self.loss_scale = loss_scale
         self.hp = hp or {}
         self.grad_dist = grad_dist or S.normal(1e-3, loss_scale)
@@ -456,4 +456,133 @@ def test_async_rejects_mismatched_betas_and_sync_calls():
         A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], 1.0, hyper(), c.stream)
     st = A.zero_async_end(c.h, c.stream)
     assert st.t == 0
+    c.close()
+
+
+# ---- tensors excluded from weight decay ------------------------------------
+# The oracle here is the plain data-parallel step with a per-element decay
+# mask on the whole vector (ZeRO leaves the math untouched); the GPU state is
+# compared in its own order through the state-to-flat permutation.
+
+def _state_perm(numel, nd, stage, psi, view):
+    if stage <= 2:
+        if view < 0:
+            return np.arange(psi)
+        b, e = Z.partition(psi, nd, view)
+        return np.arange(e - b)
+    offs = np.concatenate([[0], np.cumsum(numel)])
+    return np.concatenate([np.arange(offs[t] + b, offs[t] + e)
+                           for r in range(nd) for t, n in enumerate(numel)
+                           for b, e in [Z.chunk(n, nd, r)]])
+
+
+class MaskedCase(Case):
+    def __init__(self, *args, **kw):
+        super().__init__(*args, **kw)
+        no_decay = [bool(t[2] & A.ZERO_TENSOR_NO_DECAY) if len(t) > 2 else False
+                    for t in (self.tensors or [(self.psi, 0)])]
+        self.mask = Z.decay_mask(self.numel, no_decay)[self.b0:self.e0].copy()
+        self.perm = _state_perm(self.numel, self.nd, self.stage, self.psi, self.view)
+        self.w = self.master0.copy()
+        self.m = np.zeros_like(self.w)
+        self.v = np.zeros_like(self.w)
+        self.p16 = Z.f16_from_f32(self.w)
+
+    def oracle_step(self, gs, loss_scale):
+        sk, self.t = Z.dp_step(gs, self.w, self.m, self.v, self.p16, loss_scale,
+                               Z.hyper(**self.hp), self.t, decay=self.mask)
+        return sk
+
+    def check(self, tag=""):
+        wo, mo, vo, t = state_offsets(self.h, self.ws)
+        assert t == self.t
+        n = self.L.state_elems
+        compare_f32(self.ws.f32(wo, n), self.w[self.perm], f"master {tag}")
+        compare_f32(self.ws.f32(mo, n), self.m[self.perm], f"m {tag}")
+        compare_f32(self.ws.f32(vo, n), self.v[self.perm], f"v {tag}")
+        if self.stage <= 2 and self.view < 0:
+            for k, b in enumerate(self.bufs):
+                compare_f16(b.bits(), self.p16, f"replica {k} {tag}")
+        elif self.view >= 0:
+            compare_f16(self.bufs[0].bits()[self.b0:self.e0], self.p16, f"partition {tag}")
+        else:
+            compare_f16(self.ws.u16(self.L.off_shard16, n), self.p16[self.perm], f"shards {tag}")
+            for u in range(self.L.n_units):
+                fb, cnt = A.zero_unit_range(self.cfg, u)
+                out = GuardedF16(cnt)
+                A.zero_gather_layer(self.h, u, out.ptr(), self.stream)
+                compare_f16(out.bits(), self.p16[fb:fb + cnt], f"gather unit {u} {tag}")
+        for b in self.bufs:
+            assert b.guards_intact()
+        assert self.ws.guards_intact()
+
+
+def _flagged(tensors, rng):
+    return [(n, u, A.ZERO_TENSOR_NO_DECAY if rng.random() < 0.5 else 0) for n, u in tensors]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("stage", [1, 2, 3])
+@pytest.mark.parametrize("nd", [1, 2, 3, 5, 8])
+def test_no_decay_tensors_grid(nd, stage, variant):
+    rng = np.random.default_rng(100 * nd + 10 * stage + variant)
+    for psi in (1, 9, 257, 4099, 70001):
+        tensors = _flagged(_tensor_list(rng, psi, n_max=9), rng)
+        _run(MaskedCase(psi, nd, stage, variant, tensors=tensors,
+                        hp=dict(lr=1e-2, weight_decay=0.1)), 2)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("view", [0, 3])
+def test_no_decay_tensors_rank_view(view, variant):
+    rng = np.random.default_rng(view)
+    tensors = _flagged(_tensor_list(rng, 70001, n_max=12), rng)
+    _run(MaskedCase(70001, 4, 1, variant, tensors=tensors, view=view,
+                    hp=dict(lr=1e-2, weight_decay=0.1)), 2)
+
+
+def _gpt2_like(vocab, d, layers, ctx):
+    """GPT-2's tensor list at a small width, biases and layer-norm gains and
+    biases excluded from weight decay (embeddings and matrices decay)."""
+    ND = A.ZERO_TENSOR_NO_DECAY
+    t = [(vocab * d, 0, 0), (ctx * d, 0, 0)]
+    for l in range(layers):
+        u = l + 1
+        t += [(d, u, ND), (d, u, ND), (d * 3 * d, u, 0), (3 * d, u, ND), (d * d, u, 0), (d, u, ND),
+              (d, u, ND), (d, u, ND), (d * 4 * d, u, 0), (4 * d, u, ND), (4 * d * d, u, 0), (d, u, ND)]
+    t += [(d, layers + 1, ND), (d, layers + 1, ND)]
+    return t
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("stage", [2, 3])
+def test_no_decay_gpt2_structure(stage, variant):
+    tensors = _gpt2_like(1000, 96, 3, 128)
+    psi = sum(n for n, _, _ in tensors)
+    c = MaskedCase(psi, 8, stage, variant, tensors=tensors, loss_scale=4096.0,
+                   hp=dict(lr=1e-3, weight_decay=0.01))
+    if variant == A.ZERO_VARIANT_FUSED_TMA and stage == 2:
+        assert c.uses_tma()  # stage-3 shards of odd-sized tensors are out of 16-byte phase
+    _run(c, 3, inject=[(1, 5, psi - 1, 0x7C00)])
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_no_decay_async_steps(variant):
+    tensors = _gpt2_like(500, 64, 2, 64)
+    psi = sum(n for n, _, _ in tensors)
+    c = MaskedCase(psi, 4, 2, variant, tensors=tensors, hp=dict(lr=1e-3, weight_decay=0.05))
+    A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], A.zero_scaler(1024.0, 2.0, 0.5, 2),
+                       0.9, 0.999, c.stream)
+    scale, good = 1024.0, 0
+    for s in range(4):
+        gs = c.grads(s)
+        if s == 1:
+            gs[2][3] = 0x7C00
+        c.upload(gs)
+        A.zero_step_async(c.h, hyper(**c.hp), c.stream)
+        sk = c.oracle_step(gs, scale)
+        scale, good = Z.scaler_update(scale, good, sk, 2.0, 0.5, 2)
+    st = A.zero_async_end(c.h, c.stream)
+    assert (st.t, st.skipped) == (c.t, 1)
+    c.check("after the asynchronous run")
     c.close()

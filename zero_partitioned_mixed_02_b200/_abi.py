@@ -23,6 +23,10 @@ ZERO_ERR_WORKSPACE = -4
 ZERO_ERR_CUDA = -5
 ZERO_ERR_INTERNAL = -6
 
+ZERO_TENSOR_NO_DECAY = 1
+ZERO_PRECISION_FP16 = 0
+ZERO_PRECISION_BF16 = 1
+
 ZERO_VARIANT_FUSED = 0
 ZERO_VARIANT_TWO_PASS = 1
 ZERO_VARIANT_FUSED_TMA = 2
@@ -39,13 +43,13 @@ class ZeroError(RuntimeError):
 
 
 class zero_tensor(C.Structure):
-    _fields_ = [("numel", C.c_int64), ("unit", C.c_int32), ("reserved", C.c_int32)]
+    _fields_ = [("numel", C.c_int64), ("unit", C.c_int32), ("flags", C.c_int32)]
 
 
 class zero_config(C.Structure):
     _fields_ = [("psi", C.c_int64), ("nd", C.c_int32), ("stage", C.c_int32),
                 ("rank_view", C.c_int32), ("variant", C.c_int32), ("n_tensors", C.c_int32),
-                ("reserved", C.c_int32), ("tensors", C.POINTER(zero_tensor))]
+                ("precision", C.c_int32), ("tensors", C.POINTER(zero_tensor))]
 
 
 class zero_hyper(C.Structure):
@@ -73,6 +77,17 @@ class zero_ledger(C.Structure):
                 ("off_shard16", C.c_int64), ("off_reduced", C.c_int64),
                 ("n_units", C.c_int32), ("n_out", C.c_int32)]
 
+
+class zero_offload_ledger(C.Structure):
+    _fields_ = [("state_elems", C.c_int64), ("host_state_bytes", C.c_int64),
+                ("host_staging_bytes", C.c_int64), ("device_bytes", C.c_int64),
+                ("chunk_elems", C.c_int64), ("n_chunks", C.c_int64),
+                ("d2h_bytes_per_step", C.c_int64), ("h2d_bytes_per_step", C.c_int64),
+                ("device_state_bytes", C.c_int64), ("n_out", C.c_int32), ("reserved", C.c_int32)]
+
+
+ZERO_OFFLOAD_SLOTS = 3
+ZERO_OFFLOAD_DEFAULT_CHUNK = 1 << 24
 
 _lib = None
 
@@ -116,6 +131,17 @@ def lib():
             "zero_test_hold_tile": (C.c_int, [P, C.c_int64, C.c_uint32]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
+            "zero_offload_bytes": (C.c_int, [C.POINTER(zero_config), C.c_int64,
+                                             C.POINTER(zero_offload_ledger)]),
+            "zero_offload_init": (C.c_int, [C.POINTER(zero_config), C.c_int64, P, C.c_size_t, P,
+                                            C.c_size_t, P, P, C.POINTER(P), C.c_int, P,
+                                            C.POINTER(P)]),
+            "zero_offload_step": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P]),
+            "zero_offload_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
+                                             C.POINTER(C.c_int64)]),
+            "zero_offload_host_update": (C.c_int, [P, P, P, P, P, C.c_int64, C.POINTER(zero_hyper),
+                                                   C.c_int64, C.c_int, C.c_int]),
+            "zero_offload_destroy": (None, [P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -134,15 +160,20 @@ class Config:
 
     def __init__(self, psi: int, nd: int, stage: int, rank_view: int = -1,
                  variant: int = ZERO_VARIANT_FUSED,
-                 tensors: Sequence[tuple[int, int]] | None = None):
+                 tensors: Sequence[tuple[int, ...]] | None = None,
+                 precision: int = ZERO_PRECISION_FP16):
+        """tensors: (numel, unit) or (numel, unit, flags) per tensor, flat order;
+        flags = ZERO_TENSOR_NO_DECAY excludes the tensor from weight decay."""
         self._tensors = None
         n = 0
         ptr = None
         if tensors:
             n = len(tensors)
-            self._tensors = (zero_tensor * n)(*[zero_tensor(int(a), int(u), 0) for a, u in tensors])
+            self._tensors = (zero_tensor * n)(*[
+                zero_tensor(int(t[0]), int(t[1]), int(t[2]) if len(t) > 2 else 0) for t in tensors])
             ptr = C.cast(self._tensors, C.POINTER(zero_tensor))
-        self.c = zero_config(int(psi), int(nd), int(stage), int(rank_view), int(variant), n, 0, ptr)
+        self.c = zero_config(int(psi), int(nd), int(stage), int(rank_view), int(variant), n,
+                             int(precision), ptr)
 
     def byref(self):
         return C.byref(self.c)
@@ -270,3 +301,45 @@ def zero_uses_tma(h: int) -> bool:
 
 def zero_destroy(h: int) -> None:
     lib().zero_destroy(h)
+
+
+# ---- offloaded step (include/zero_offload.h) ----
+
+def zero_offload_bytes(cfg: Config, chunk_elems: int = 0) -> zero_offload_ledger:
+    out = zero_offload_ledger()
+    _check(lib().zero_offload_bytes(cfg.byref(), int(chunk_elems), C.byref(out)), "zero_offload_bytes")
+    return out
+
+
+def zero_offload_init(cfg: Config, chunk_elems: int, device_ws: int, device_bytes: int,
+                      host_staging: int, staging_bytes: int, host_state: int, master_init: int,
+                      param_bufs: Sequence[int], n_threads: int, stream: int) -> int:
+    h = C.c_void_p()
+    _check(lib().zero_offload_init(cfg.byref(), int(chunk_elems), device_ws, device_bytes, host_staging,
+                                   staging_bytes, host_state, master_init, _ptr_array(param_bufs),
+                                   int(n_threads), stream, C.byref(h)), "zero_offload_init")
+    return h.value
+
+
+def zero_offload_step(h: int, grads: Sequence[int], loss_scale: float, hp: zero_hyper,
+                      stream: int) -> int:
+    return _check(lib().zero_offload_step(h, _ptr_array(grads), float(loss_scale), C.byref(hp), stream),
+                  "zero_offload_step")
+
+
+def zero_offload_state(h: int) -> tuple[int, int, int, int]:
+    w, m, v = C.c_void_p(), C.c_void_p(), C.c_void_p()
+    t = C.c_int64()
+    _check(lib().zero_offload_state(h, C.byref(w), C.byref(m), C.byref(v), C.byref(t)),
+           "zero_offload_state")
+    return w.value, m.value, v.value, t.value
+
+
+def zero_offload_host_update(g: int, w: int, m: int, v: int, p16: int, n: int, hp: zero_hyper, t: int,
+                             decay: bool, path: int = 0) -> None:
+    _check(lib().zero_offload_host_update(g, w, m, v, p16, int(n), C.byref(hp), int(t), int(bool(decay)),
+                                          int(path)), "zero_offload_host_update")
+
+
+def zero_offload_destroy(h: int) -> None:
+    lib().zero_offload_destroy(h)

@@ -1,6 +1,8 @@
 """Build the package's native libraries in-tree for sm_100a.
 
-  libzero.so          the ZeRO step library (csrc/*.cu, C ABI in include/zero.h)
+  libzero.so          the ZeRO step library (csrc/*.cu and the host update
+                      csrc/zero_host_adam.cpp; C ABI in include/zero.h and
+                      include/zero_offload.h)
   synth/libzsynth.so  the seeded synthetic-input generator (host + device)
 
 Flags: arithmetic is IEEE binary32 as written -- no FMA contraction
@@ -29,9 +31,18 @@ COMMON = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-fmad=false", "-f
           "-prec-div=true", "-prec-sqrt=true", "-Xcompiler", "-fPIC,-ffp-contract=off"]
 
 ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu"),
-                os.path.join(CSRC, "zero_static.cu"), os.path.join(CSRC, "zero_tma.cu")]
-ZERO_DEPS = ZERO_SOURCES + [os.path.join(CSRC, "zero_internal.h"), os.path.join(CSRC, "zero_device.cuh"),
-                            os.path.join(INCLUDE, "zero.h")]
+                os.path.join(CSRC, "zero_static.cu"), os.path.join(CSRC, "zero_tma.cu"),
+                os.path.join(CSRC, "zero_offload.cu")]
+HOST_ADAM = os.path.join(CSRC, "zero_host_adam.cpp")
+ZERO_DEPS = ZERO_SOURCES + [HOST_ADAM, os.path.join(CSRC, "zero_host_adam.h"),
+                            os.path.join(CSRC, "zero_internal.h"), os.path.join(CSRC, "zero_device.cuh"),
+                            os.path.join(CSRC, "zero_layout.h"), os.path.join(INCLUDE, "zero.h"),
+                            os.path.join(INCLUDE, "zero_offload.h")]
+# the host update is built twice: AVX2 + F16C, and the baseline instruction set
+# (picked at run time); binary32 as written, no contraction into FMA
+CXX = os.environ.get("CXX", "g++")
+HOST_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-ffp-contract=off", "-fno-fast-math"]
+HOST_VARIANTS = {"avx2": ["-DZH_AVX2", "-mavx2", "-mf16c"], "base": []}
 SYNTH_SOURCES = [os.path.join(SYNTH, "zsynth.cu")]
 SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(SYNTH, "zsynth.h")]
 
@@ -56,11 +67,27 @@ def _nvcc(out: str, sources: list[str], extra: list[str], log: str | None = None
     os.replace(tmp, out)
 
 
+def _host_objects() -> list[str]:
+    objs = []
+    for name, flags in HOST_VARIANTS.items():
+        obj = os.path.join(PKG, f"zero_host_adam_{name}.o")
+        cmd = [CXX, *HOST_FLAGS, *flags, "-I", CSRC, "-c", HOST_ADAM, "-o", obj]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError(f"{CXX} failed building {os.path.basename(obj)}")
+        objs.append(obj)
+    return objs
+
+
 def build(force: bool = False) -> None:
     if force or _stale(LIBZERO, ZERO_DEPS):
-        _nvcc(LIBZERO, ZERO_SOURCES,
+        objs = _host_objects()
+        _nvcc(LIBZERO, ZERO_SOURCES + objs,
               ["-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v"],
               log=PTXAS_LOG)
+        for o in objs:
+            os.remove(o)
     if force or _stale(LIBSYNTH, SYNTH_DEPS):
         _nvcc(LIBSYNTH, SYNTH_SOURCES, ["-I", SYNTH])
 

@@ -7,12 +7,18 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "zero.h"
 #include "zero_internal.h"
+#include "zero_layout.h"
 
 #define ZERO_API extern "C" __attribute__((visibility("default")))
+
+using zl::Layout;
+using zl::split;
+using zl::Unit;
 
 namespace {
 
@@ -23,60 +29,13 @@ int64_t align_up(int64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Ceil split ([P1] "The replication nobody questioned": the state is divided
-// across the Nd ranks; trailing ranks may be short or empty).
-void split(int64_t n, int nd, int r, int64_t* b, int64_t* e)
-{
-    const int64_t p = (n + nd - 1) / nd;
-    *b = std::min<int64_t>((int64_t)r * p, n);
-    *e = std::min<int64_t>(*b + p, n);
-}
-
-struct Unit {
-    int64_t seg0 = 0;     // first gather run of the unit
-    int64_t n_segs = 0;
-    int64_t n_chunks = 0;
-    int64_t flat_begin = 0;
-    int64_t numel = 0;
-    bool tma_ok = false;  // bulk-copy gather table built (TMA variant, runs in 16-byte phase)
-    int64_t tma_run0 = 0;
-    int64_t tma_n_runs = 0;
-    int64_t tma_tiles = 0;
-    int64_t tma_scal = 0;
-};
-
-// Everything that follows from a configuration: partitions, run tables,
-// ledger and workspace layout.
-struct Layout {
-    int64_t psi = 0;
-    int nd = 0, stage = 0, view = -1, variant = 0;
-    std::vector<int64_t> numel;  // tensor sizes (one flat tensor if none given)
-    std::vector<int32_t> unit_of;
-    int64_t P = 0, state_elems = 0, grad_len = 0;
-    int n_out = 0, n_units = 0;
-    std::vector<int64_t> shard_begin, shard_len;  // per rank, in state elements
-    std::vector<zk::SegDesc> step_segs;
-    int64_t step_chunks = 0;
-    std::vector<zk::SegDesc> gather_segs;
-    std::vector<zk::TmaRun> tma_gather;  // TMA variant: bulk-copy gather runs of all units
-    std::vector<Unit> units;
-    std::vector<zk::TmaRun> tma_runs;  // TMA variant, when every run is eligible
-    bool tma_ok = false;
-    zk::TmaShape tma_shape = zk::kTmaDeep;
-    int64_t tma_tiles = 0, tma_scal = 0;
-    int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
-            off_gather_segs = 0, off_tma_runs = -1, off_tma_gather = -1, off_reduced = -1, off_shard16 = -1,
-            total = 0;
-    int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
-    int64_t transient_elems = 0;
-};
-
 // Cut a run at the first line-aligned gradient index and give it its chunks.
 void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, int64_t state_begin,
-             int64_t out_begin, int64_t len)
+             int64_t out_begin, int64_t len, int decay = 1)
 {
     if (len <= 0) return;
     zk::SegDesc d{};
+    d.decay = decay;
     d.grad_begin = grad_begin;
     d.state_begin = state_begin;
     d.out_begin = out_begin;
@@ -92,7 +51,9 @@ void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, i
     v.push_back(d);
 }
 
-int build_layout(const zero_config* cfg, Layout* L)
+}  // namespace
+
+int zl::build_layout(const zero_config* cfg, Layout* L)
 {
     if (!cfg) return ZERO_ERR_ARG;
     if (cfg->psi < 1 || cfg->psi > kMaxPsi) return ZERO_ERR_ARG;
@@ -101,7 +62,10 @@ int build_layout(const zero_config* cfg, Layout* L)
     if (cfg->variant != ZERO_VARIANT_FUSED && cfg->variant != ZERO_VARIANT_TWO_PASS &&
         cfg->variant != ZERO_VARIANT_FUSED_TMA)
         return ZERO_ERR_ARG;
-    if (cfg->reserved != 0 || cfg->n_tensors < 0) return ZERO_ERR_ARG;
+    if (cfg->n_tensors < 0) return ZERO_ERR_ARG;
+    if (cfg->precision != ZERO_PRECISION_FP16 && cfg->precision != ZERO_PRECISION_BF16) return ZERO_ERR_ARG;
+    // without a master nothing can be rolled back: the two-pass step only
+    if (cfg->precision == ZERO_PRECISION_BF16 && cfg->variant != ZERO_VARIANT_TWO_PASS) return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
     if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
     if (cfg->stage == 3 && cfg->n_tensors == 0) return ZERO_ERR_ARG;
@@ -112,25 +76,28 @@ int build_layout(const zero_config* cfg, Layout* L)
     L->stage = cfg->stage;
     L->view = cfg->rank_view;
     L->variant = cfg->variant;
+    L->bf16 = cfg->precision == ZERO_PRECISION_BF16;
     const int nd = cfg->nd;
     if (cfg->n_tensors > 0) {
         int64_t sum = 0;
         int32_t prev_unit = 0;
         for (int i = 0; i < cfg->n_tensors; ++i) {
             const zero_tensor& t = cfg->tensors[i];
-            if (t.numel < 1 || t.reserved != 0 || t.unit < 0) return ZERO_ERR_ARG;
+            if (t.numel < 1 || (t.flags & ~ZERO_TENSOR_NO_DECAY) != 0 || t.unit < 0) return ZERO_ERR_ARG;
             if (i == 0 ? t.unit != 0 : (t.unit != prev_unit && t.unit != prev_unit + 1)) return ZERO_ERR_ARG;
             prev_unit = t.unit;
             sum += t.numel;
             if (sum > kMaxPsi) return ZERO_ERR_ARG;
             L->numel.push_back(t.numel);
             L->unit_of.push_back(t.unit);
+            L->decay_of.push_back((t.flags & ZERO_TENSOR_NO_DECAY) ? 0 : 1);
         }
         if (sum != cfg->psi) return ZERO_ERR_ARG;
         L->n_units = prev_unit + 1;
     } else {
         L->numel.push_back(cfg->psi);
         L->unit_of.push_back(0);
+        L->decay_of.push_back(1);
         L->n_units = 1;
     }
     L->P = (cfg->psi + nd - 1) / nd;
@@ -139,13 +106,36 @@ int build_layout(const zero_config* cfg, Layout* L)
     L->shard_begin.assign(nd, 0);
     L->shard_len.assign(nd, 0);
     if (cfg->stage <= 2) {
+        // flat spans of equal decay (consecutive tensors with the same flag
+        // merge); a partition is cut where it crosses from one span to the next
+        std::vector<std::pair<int64_t, int>> span_end;  // (end, decay)
+        int64_t flat = 0;
+        for (size_t t = 0; t < L->numel.size(); ++t) {
+            flat += L->numel[t];
+            if (!span_end.empty() && span_end.back().second == L->decay_of[t])
+                span_end.back().first = flat;
+            else
+                span_end.push_back({flat, L->decay_of[t]});
+        }
+        // runs of the flat range [b, e): grad and state indices are flat - base
+        auto add_partition = [&](int64_t b, int64_t e, int64_t base) {
+            int64_t x = b, span_begin = 0;
+            for (const auto& sp : span_end) {
+                const int64_t lo = std::max(x, span_begin), hi = std::min(e, sp.first);
+                if (hi > lo) {
+                    add_run(L->step_segs, &L->step_chunks, lo - base, lo - base, lo, hi - lo, sp.second);
+                    x = hi;
+                }
+                span_begin = sp.first;
+            }
+        };
         if (cfg->rank_view < 0) {
             for (int r = 0; r < nd; ++r) {
                 int64_t b, e;
                 split(cfg->psi, nd, r, &b, &e);
                 L->shard_begin[r] = b;
                 L->shard_len[r] = e - b;
-                add_run(L->step_segs, &L->step_chunks, b, b, b, e - b);
+                add_partition(b, e, 0);
             }
             L->state_elems = cfg->psi;
             L->grad_len = cfg->psi;
@@ -154,7 +144,7 @@ int build_layout(const zero_config* cfg, Layout* L)
             int64_t b, e;
             split(cfg->psi, nd, cfg->rank_view, &b, &e);
             L->shard_len[cfg->rank_view] = e - b;
-            add_run(L->step_segs, &L->step_chunks, 0, 0, b, e - b);
+            add_partition(b, e, b);
             L->state_elems = e - b;
             L->grad_len = e - b;
             L->n_out = 1;
@@ -169,7 +159,7 @@ int build_layout(const zero_config* cfg, Layout* L)
             for (size_t t = 0; t < L->numel.size(); ++t) {
                 int64_t b, e;
                 split(L->numel[t], nd, r, &b, &e);
-                add_run(L->step_segs, &L->step_chunks, off + b, pos + q, pos + q, e - b);
+                add_run(L->step_segs, &L->step_chunks, off + b, pos + q, pos + q, e - b, L->decay_of[t]);
                 q += e - b;
                 off += L->numel[t];
             }
@@ -255,6 +245,7 @@ int build_layout(const zero_config* cfg, Layout* L)
         if (ok) {
             for (const zk::SegDesc& d : L->step_segs) {
                 zk::TmaRun t{};
+                t.decay = d.decay;
                 t.grad_begin = d.grad_begin;
                 t.state_begin = d.state_begin;
                 t.out_begin = d.out_begin;
@@ -297,6 +288,7 @@ int build_layout(const zero_config* cfg, Layout* L)
     const int n_buf = cfg->variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
     for (int b = 0; b < n_buf; ++b)
         for (int k = 0; k < 3; ++k) {
+            if (k == 0 && L->bf16) continue;  // no master: the parameters are the weights
             L->off_state[b][k] = off;
             off += align_up(L->state_elems * 4);
         }
@@ -312,12 +304,16 @@ int build_layout(const zero_config* cfg, Layout* L)
     return ZERO_OK;
 }
 
+namespace {
+
 void fill_ledger(const Layout& L, zero_ledger* out)
 {
     std::memset(out, 0, sizeof(*out));
-    const double psi = (double)L.psi, nd = (double)L.nd, K = 12.0;
     // [P1] "Where 16 bytes per parameter comes from": 2 + 2 + K, K = 12;
-    // [P2] "The Mathematics": M_states(p, Nd)
+    // [P2] "The Mathematics": M_states(p, Nd). Without fp32 master weights
+    // ([P3] "Why parameter count is not training memory") K = 8: m and v.
+    const int64_t Ki = L.bf16 ? 8 : 12;
+    const double psi = (double)L.psi, nd = (double)L.nd, K = (double)Ki;
     out->formula_bytes[0] = (2.0 + 2.0 + K) * psi;
     out->formula_bytes[1] = 4.0 * psi + K * psi / nd;
     out->formula_bytes[2] = 2.0 * psi + (2.0 + K) * psi / nd;
@@ -335,10 +331,10 @@ void fill_ledger(const Layout& L, zero_ledger* out)
         }
         max_shard = std::max(max_shard, s);
     }
-    out->exact_bytes[0] = 16 * L.psi;
-    out->exact_bytes[1] = 4 * L.psi + 12 * max_part;
-    out->exact_bytes[2] = 2 * L.psi + 14 * max_part;
-    out->exact_bytes[3] = 16 * max_shard;
+    out->exact_bytes[0] = (4 + Ki) * L.psi;
+    out->exact_bytes[1] = 4 * L.psi + Ki * max_part;
+    out->exact_bytes[2] = 2 * L.psi + (2 + Ki) * max_part;
+    out->exact_bytes[3] = (4 + Ki) * max_shard;
     // ring collectives: each rank sends everything but the chunk it keeps
     const int64_t rs = (int64_t)L.nd * L.psi - L.psi;
     out->comm_elements[0] = rs;
@@ -406,7 +402,10 @@ struct zero_handle {
     int64_t bc_t = -1;
     double bc_p1 = 1.0, bc_p2 = 1.0;
 
-    float* state(int buf, int k) const { return reinterpret_cast<float*>(ws + L.off_state[buf][k]); }
+    float* state(int buf, int k) const
+    {
+        return L.off_state[buf][k] < 0 ? nullptr : reinterpret_cast<float*>(ws + L.off_state[buf][k]);
+    }
 };
 
 namespace {
@@ -521,7 +520,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
     const int smem = zk::step_smem_bytes(L.nd, L.n_out);
     for (int k = 0; k < zk::K_COUNT && e == cudaSuccess; ++k)
-        e = zk::occupancy((zk::Kernel)k, k == zk::K_GATHER ? 0 : smem, &h->occ[k]);
+        e = zk::occupancy((zk::Kernel)k, k == zk::K_GATHER ? 0 : smem, &h->occ[k], L.bf16);
     if (e != cudaSuccess) {
         rc = cuda_fail(h, e);
         delete h;
@@ -586,7 +585,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
         a.v_out = h->state(0, 2);
         a.master_init = master_init;
         a.flag = h->d_flag;
-        e = zk::launch_step(zk::K_INIT, a, grid_for(h, zk::K_INIT, L.step_chunks), s);
+        e = zk::launch_step(zk::K_INIT, a, grid_for(h, zk::K_INIT, L.step_chunks), s, L.bf16);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) {
@@ -672,9 +671,9 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
             e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
         } else {
             a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
-            e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s);
+            e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s, L.bf16);
             if (e == cudaSuccess)
-                e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s);
+                e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s, L.bf16);
         }
         if (e != cudaSuccess) return cuda_fail(h, e);
     }
@@ -827,8 +826,9 @@ ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
         e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
     } else {
         a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
-        e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s);
-        if (e == cudaSuccess) e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s);
+        e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s, L.bf16);
+        if (e == cudaSuccess)
+            e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s, L.bf16);
     }
     // the fused passes wrote fp16 parameters: rewrite them from the unchanged
     // master if the step overflowed (the kernel returns at once otherwise)
@@ -914,17 +914,19 @@ ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m,
     if (!h || h->pending || h->async || t < 0) return ZERO_ERR_ARG;
     const Layout& L = h->L;
     const size_t bytes = (size_t)L.state_elems * sizeof(float);
-    if (L.state_elems > 0 && (!master || !m || !v)) return ZERO_ERR_ARG;
+    // without a master (bfloat16) the parameters live in the outputs; a
+    // non-NULL master is then written to them, rounded to bfloat16
+    if (L.state_elems > 0 && ((!master && !L.bf16) || !m || !v)) return ZERO_ERR_ARG;
     if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZERO_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float* src[3] = {master, m, v};
     cudaError_t e = cudaSuccess;
     for (int k = 0; k < 3 && e == cudaSuccess && bytes > 0; ++k) {
         float* dst = h->state(h->cur, k);
-        if (dst != src[k]) e = cudaMemcpyAsync(dst, src[k], bytes, cudaMemcpyDeviceToDevice, s);
+        if (dst && dst != src[k]) e = cudaMemcpyAsync(dst, src[k], bytes, cudaMemcpyDeviceToDevice, s);
     }
-    if (e == cudaSuccess && L.step_chunks > 0) {
-        // the fp16 parameters follow the restored master
+    if (e == cudaSuccess && L.step_chunks > 0 && master) {
+        // the 16-bit parameters follow the restored master
         zk::StepArgs a{};
         a.segs = h->d_step_segs;
         a.n_segs = (int)L.step_segs.size();
@@ -932,9 +934,9 @@ ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m,
         a.outs = h->d_out_tab;
         a.n_out = (int)h->out_tab.size();
         a.nd = L.nd;
-        a.w_in = h->state(h->cur, 0);
+        a.w_in = L.bf16 ? master : h->state(h->cur, 0);
         a.flag = h->d_flag;
-        e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
+        e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s, L.bf16);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(h, e);

@@ -3,6 +3,7 @@
 // and the scalar (head/tail) item body. Internal to libzero.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -40,6 +41,53 @@ __device__ __forceinline__ uint2 pack(const float* x) { return make_uint2(pack2(
 
 // 4 fp16 values from p (8-byte aligned: quads start on multiples of 4).
 __device__ __forceinline__ uint2 ld_hq(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+
+// 4 16-bit values from p with the widest loads p's alignment allows (the
+// parameter buffers read back by the step without a master may be out of
+// phase with the gradient index).
+__device__ __forceinline__ uint2 ld_hq_any(const uint16_t* p)
+{
+    const unsigned a = (unsigned)reinterpret_cast<uintptr_t>(p);
+    if ((a & 7u) == 0) return __ldcs(reinterpret_cast<const uint2*>(p));
+    if ((a & 3u) == 0) {
+        const unsigned* u = reinterpret_cast<const unsigned*>(p);
+        return make_uint2(__ldcs(u), __ldcs(u + 1));
+    }
+    const unsigned short* h = reinterpret_cast<const unsigned short*>(p);
+    return make_uint2((unsigned)__ldcs(h) | ((unsigned)__ldcs(h + 1) << 16),
+                      (unsigned)__ldcs(h + 2) | ((unsigned)__ldcs(h + 3) << 16));
+}
+
+// ---- element formats of the 16-bit streams ----
+// F16: IEEE binary16 gradients and parameters, fp32 master weights.
+// BF16: bfloat16 gradients and parameters and no fp32 master: the parameter
+// itself is the weight state, read back and rounded to bfloat16 every step.
+struct F16 {
+    static constexpr bool kMaster = true;
+    __device__ static float dec(unsigned short b) { return h2f(b); }
+    __device__ static unsigned short enc(float x) { return f2h(x); }
+};
+struct BF16 {
+    static constexpr bool kMaster = false;
+    __device__ static float dec(unsigned short b) { return __uint_as_float((unsigned)b << 16); }
+    __device__ static unsigned short enc(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+};
+
+template <class C>
+__device__ __forceinline__ void unpack_as(const uint2 q, float* x)
+{
+    x[0] = C::dec((unsigned short)(q.x & 0xffffu));
+    x[1] = C::dec((unsigned short)(q.x >> 16));
+    x[2] = C::dec((unsigned short)(q.y & 0xffffu));
+    x[3] = C::dec((unsigned short)(q.y >> 16));
+}
+
+template <class C>
+__device__ __forceinline__ uint2 pack_as(const float* x)
+{
+    return make_uint2((unsigned)C::enc(x[0]) | ((unsigned)C::enc(x[1]) << 16),
+                      (unsigned)C::enc(x[2]) | ((unsigned)C::enc(x[3]) << 16));
+}
 
 // Store 4 fp16 values with the widest accesses p's alignment allows (the
 // branch is uniform over a run).
@@ -124,8 +172,9 @@ __device__ __forceinline__ void st_pair(float* base, long long ia, long long ib,
 
 // ---- the step's arithmetic ----
 
-// Rank-ordered binary32 sum of the Nd fp16 gradients of a lane's two quads.
+// Rank-ordered binary32 sum of the Nd 16-bit gradients of a lane's two quads.
 // Loads are issued 8 ranks at a time ahead of the additions.
+template <class C = F16>
 __device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, long long ga,
                                             long long gb, bool hb, float (&s)[8])
 {
@@ -137,14 +186,14 @@ __device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, l
             qb[j] = hb ? ld_hq(gp[j] + gb) : make_uint2(0u, 0u);
         }
     }
-    unpack(qa[0], s);
-    unpack(qb[0], s + 4);
+    unpack_as<C>(qa[0], s);
+    unpack_as<C>(qb[0], s + 4);
 #pragma unroll
     for (int j = 1; j < 8; ++j) {
         if (j < nd) {
             float x[8];
-            unpack(qa[j], x);
-            unpack(qb[j], x + 4);
+            unpack_as<C>(qa[j], x);
+            unpack_as<C>(qb[j], x + 4);
 #pragma unroll
             for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
         }
@@ -161,8 +210,8 @@ __device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, l
         for (int j = 0; j < 8; ++j) {
             if (r0 + j < nd) {
                 float x[8];
-                unpack(qa[j], x);
-                unpack(qb[j], x + 4);
+                unpack_as<C>(qa[j], x);
+                unpack_as<C>(qb[j], x + 4);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) s[i] = __fadd_rn(s[i], x[i]);
             }
@@ -170,24 +219,26 @@ __device__ __forceinline__ void reduce_pair(const uint16_t* const* gp, int nd, l
     }
 }
 
+template <class C = F16>
 __device__ __forceinline__ float reduce1(const uint16_t* const* gp, int nd, long long gi)
 {
-    float s = h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[0] + gi)));
+    float s = C::dec(__ldcs(reinterpret_cast<const unsigned short*>(gp[0] + gi)));
     for (int r = 1; r < nd; ++r)
-        s = __fadd_rn(s, h2f(__ldcs(reinterpret_cast<const unsigned short*>(gp[r] + gi))));
+        s = __fadd_rn(s, C::dec(__ldcs(reinterpret_cast<const unsigned short*>(gp[r] + gi))));
     return s;
 }
 
 // One element of mixed-precision Adam (bias-corrected, decoupled weight decay
-// scaled by lr), binary32, in the order of the step's definition.
-__device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, const Coef& c)
+// wd scaled by lr), binary32, in the order of the step's definition. wd is
+// c.wd, or 0 for a tensor excluded from weight decay.
+__device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, const Coef& c, float wd)
 {
     const float m1 = __fadd_rn(__fmul_rn(c.b1, m), __fmul_rn(c.omb1, g));
     const float v1 = __fadd_rn(__fmul_rn(c.b2, v), __fmul_rn(c.omb2, __fmul_rn(g, g)));
     const float mh = __fdiv_rn(m1, c.bc1);
     const float vh = __fdiv_rn(v1, c.bc2);
     const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), c.eps));
-    w = __fsub_rn(w, __fmul_rn(c.lr, __fadd_rn(u, __fmul_rn(c.wd, w))));
+    w = __fsub_rn(w, __fmul_rn(c.lr, __fadd_rn(u, __fmul_rn(wd, w))));
     m = m1;
     v = v1;
 }
@@ -240,7 +291,10 @@ __device__ __forceinline__ Live live_of(const StepArgs& a)
     return L;
 }
 
-template <int K>
+// C::kMaster false (no fp32 master): K_INIT writes no master, K_UPDATE reads
+// the weight from the first output (the parameter itself) and writes no
+// master; the state buffers hold m and v only.
+template <int K, class C = F16>
 __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, const uint16_t* const* gp,
                                             uint16_t* const* op, const SegDesc& d, long long e,
                                             bool& bad)
@@ -249,19 +303,22 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, co
     float w = 0.0f, m = 0.0f, v = 0.0f, g = 0.0f;
     if (K == K_INIT) {
         w = __ldcs(a.master_init + gi);
-        __stcs(L.w_out + si, w);
+        if (C::kMaster) __stcs(L.w_out + si, w);
         __stcs(L.m_out + si, 0.0f);
         __stcs(L.v_out + si, 0.0f);
     } else if (K == K_CAST) {
         w = __ldcs(L.w_in + si);
     } else {
         if (K == K_STEP_FUSED || K == K_UPDATE) {
-            w = __ldcs(L.w_in + si);
+            if (C::kMaster)
+                w = __ldcs(L.w_in + si);
+            else
+                w = C::dec(__ldcs(reinterpret_cast<const unsigned short*>(op[0] + oi)));
             m = __ldcs(L.m_in + si);
             v = __ldcs(L.v_in + si);
         }
         if (K == K_STEP_FUSED || K == K_REDUCE) {
-            g = __fmul_rn(reduce1(gp, a.nd, gi), L.c.inv_scale);
+            g = __fmul_rn(reduce1<C>(gp, a.nd, gi), L.c.inv_scale);
             bad |= nonfinite(g);
         }
         if (K == K_REDUCE) {
@@ -269,12 +326,12 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, co
             return;
         }
         if (K == K_UPDATE) g = __ldcs(a.red + si);
-        adam1(g, w, m, v, L.c);
-        __stcs(L.w_out + si, w);
+        adam1(g, w, m, v, L.c, d.decay ? L.c.wd : 0.0f);
+        if (C::kMaster) __stcs(L.w_out + si, w);
         __stcs(L.m_out + si, m);
         __stcs(L.v_out + si, v);
     }
-    const unsigned short h = f2h(w);
+    const unsigned short h = C::enc(w);
     for (int k = 0; k < a.n_out; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);
 }
 

@@ -36,8 +36,10 @@ struct alignas(16) SegDesc {
     long long chunk_begin;  // first chunk of this run in the launch's chunk numbering
     int head;               // scalar elements before the body
     int tail;               // scalar elements after the body
+    int decay;              // 1: weight decay applies to the run; 0: excluded tensor
+    int pad;
 };
-static_assert(sizeof(SegDesc) == 48, "SegDesc layout");
+static_assert(sizeof(SegDesc) == 64, "SegDesc layout");
 
 // Per-step binary32 constants, computed on the host (or, for the
 // asynchronous step, partly on the device from the control block).
@@ -110,7 +112,8 @@ struct alignas(16) TmaRun {
     long long scal_begin;  // first scalar item in the launch's scalar numbering
     int head;
     int tail;
-    int pad[2];
+    int decay;             // as SegDesc::decay
+    int pad;
 };
 static_assert(sizeof(TmaRun) == 64, "TmaRun layout");
 
@@ -180,9 +183,12 @@ enum Kernel : int {
     K_COUNT = 7
 };
 
-// Blocks per SM the kernel reaches with `smem` bytes of dynamic shared memory.
-cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm);
-cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s);
+// Blocks per SM the kernel reaches with `smem` bytes of dynamic shared memory
+// (0 for a kind not built for the format). bf16: the bfloat16 step without an
+// fp32 master (kinds K_REDUCE, K_UPDATE, K_CAST, K_INIT; state = m and v only,
+// the weight read back from the first output).
+cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm, bool bf16 = false);
+cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s, bool bf16 = false);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cudaStream_t s);
 // Asynchronous step: commit or roll back on the device (one thread).

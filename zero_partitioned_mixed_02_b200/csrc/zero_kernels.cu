@@ -36,7 +36,9 @@ namespace {
 
 // ---- per-item bodies of the step kernels ----
 
-template <int K>
+// C: the 16-bit element format (F16 with an fp32 master; BF16 without one,
+// where the weight is read back from the first output and no master is kept).
+template <int K, class C>
 __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const uint16_t* const* gp,
                                          uint16_t* const* op, const SegDesc& d, const Pair& p,
                                          bool& bad)
@@ -50,19 +52,24 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const
         ld_pair(a.master_init, ga, gb, hb, w);
 #pragma unroll
         for (int j = 0; j < 8; ++j) m[j] = 0.0f;
-        st_pair(L.w_out, sa, sb, hb, w);
+        if (C::kMaster) st_pair(L.w_out, sa, sb, hb, w);
         st_pair(L.m_out, sa, sb, hb, m);
         st_pair(L.v_out, sa, sb, hb, m);
     } else if (K == K_CAST) {
         ld_pair(L.w_in, sa, sb, hb, w);
     } else {
         if (K == K_STEP_FUSED || K == K_UPDATE) {
-            ld_pair(L.w_in, sa, sb, hb, w);
+            if (C::kMaster) {
+                ld_pair(L.w_in, sa, sb, hb, w);
+            } else {
+                unpack_as<C>(ld_hq_any(op[0] + oa), w);
+                unpack_as<C>(hb ? ld_hq_any(op[0] + ob) : make_uint2(0u, 0u), w + 4);
+            }
             ld_pair(L.m_in, sa, sb, hb, m);
             ld_pair(L.v_in, sa, sb, hb, v);
         }
         if (K == K_STEP_FUSED || K == K_REDUCE) {
-            reduce_pair(gp, a.nd, ga, gb, hb, g);
+            reduce_pair<C>(gp, a.nd, ga, gb, hb, g);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 g[j] = __fmul_rn(g[j], L.c.inv_scale);
@@ -74,13 +81,14 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const
             return;
         }
         if (K == K_UPDATE) ld_pair(a.red, sa, sb, hb, g);
+        const float wd = d.decay ? L.c.wd : 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], L.c);
-        st_pair(L.w_out, sa, sb, hb, w);
+        for (int j = 0; j < 8; ++j) adam1(g[j], w[j], m[j], v[j], L.c, wd);
+        if (C::kMaster) st_pair(L.w_out, sa, sb, hb, w);
         st_pair(L.m_out, sa, sb, hb, m);
         st_pair(L.v_out, sa, sb, hb, v);
     }
-    const uint2 h0 = pack(w), h1 = pack(w + 4);
+    const uint2 h0 = pack_as<C>(w), h1 = pack_as<C>(w + 4);
     for (int k = 0; k < a.n_out; ++k) {
         st_hq(op[k] + oa, h0);
         if (hb) st_hq(op[k] + ob, h1);
@@ -133,7 +141,7 @@ __device__ __forceinline__ void walk(const SegDesc* segs, int n_segs, long long 
 
 // K_CAST_IF is K_CAST run only when the step overflowed or a kernel gave up.
 // ASYNC: the step constants and state buffers come from the control block.
-template <int K, bool ASYNC>
+template <int K, bool ASYNC, class C = F16>
 __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const StepArgs a0)
 {
     extern __shared__ uintptr_t s_ptr[];
@@ -162,8 +170,8 @@ __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const Ste
     bool bad = false;
     walk(
         a.segs, a.n_segs, a.n_chunks,
-        [&](const SegDesc& d, const Pair& p) { step_vec<KB>(a, L, gp, op, d, p, bad); },
-        [&](const SegDesc& d, long long e) { step_scalar<KB>(a, L, gp, op, d, e, bad); });
+        [&](const SegDesc& d, const Pair& p) { step_vec<KB, C>(a, L, gp, op, d, p, bad); },
+        [&](const SegDesc& d, long long e) { step_scalar<KB, C>(a, L, gp, op, d, e, bad); });
 
     if (kGrads) {
         // one atomic per warp that saw a non-finite unscaled gradient
@@ -221,8 +229,18 @@ __global__ void commit_kernel(Ctrl* c, unsigned* flag, const unsigned* err)
     *flag = 0;
 }
 
-const void* kernel_ptr(Kernel k)
+const void* kernel_ptr(Kernel k, bool bf16)
 {
+    if (bf16) {
+        switch (k) {
+            case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE, false, BF16>);
+            case K_UPDATE: return reinterpret_cast<const void*>(&step_kernel<K_UPDATE, false, BF16>);
+            case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST, false, BF16>);
+            case K_INIT: return reinterpret_cast<const void*>(&step_kernel<K_INIT, false, BF16>);
+            case K_GATHER: return reinterpret_cast<const void*>(&gather_kernel);
+            default: return nullptr;
+        }
+    }
     switch (k) {
         case K_STEP_FUSED: return reinterpret_cast<const void*>(&step_kernel<K_STEP_FUSED, false>);
         case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE, false>);
@@ -239,17 +257,37 @@ const void* kernel_ptr(Kernel k)
 
 int step_smem_bytes(int nd, int n_out) { return (nd + n_out) * (int)sizeof(uintptr_t); }
 
-cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm)
+cudaError_t occupancy(Kernel k, int smem, int* blocks_per_sm, bool bf16)
 {
-    const void* f = kernel_ptr(k);
-    if (!f) return cudaErrorInvalidValue;
+    const void* f = kernel_ptr(k, bf16);
+    if (!f) {
+        *blocks_per_sm = 0;
+        return cudaSuccess;  // not instantiated for this format
+    }
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, f, kThreads, smem);
 }
 
-cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s)
+cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s, bool bf16)
 {
     const int smem = step_smem_bytes(a.nd, a.n_out);
     const bool as = a.ctrl != nullptr;
+    if (bf16) {
+        // the step without a master runs the two passes only (nothing to roll back)
+        switch (k) {
+            case K_REDUCE:
+                if (as) step_kernel<K_REDUCE, true, BF16><<<grid, kThreads, smem, s>>>(a);
+                else step_kernel<K_REDUCE, false, BF16><<<grid, kThreads, smem, s>>>(a);
+                break;
+            case K_UPDATE:
+                if (as) step_kernel<K_UPDATE, true, BF16><<<grid, kThreads, smem, s>>>(a);
+                else step_kernel<K_UPDATE, false, BF16><<<grid, kThreads, smem, s>>>(a);
+                break;
+            case K_CAST: step_kernel<K_CAST, false, BF16><<<grid, kThreads, smem, s>>>(a); break;
+            case K_INIT: step_kernel<K_INIT, false, BF16><<<grid, kThreads, smem, s>>>(a); break;
+            default: return cudaErrorInvalidValue;
+        }
+        return cudaGetLastError();
+    }
     switch (k) {
         case K_STEP_FUSED:
             if (as) step_kernel<K_STEP_FUSED, true><<<grid, kThreads, smem, s>>>(a);

@@ -67,6 +67,7 @@ void add_run(zk::SegDesc* runs, int* n, int64_t* chunks, int64_t begin, int64_t 
     zk::SegDesc d{};
     d.grad_begin = d.state_begin = d.out_begin = begin;
     d.len = len;
+    d.decay = 1;
     int64_t head = (zk::kLineElems - begin % zk::kLineElems) % zk::kLineElems;
     if (head > len) head = len;
     const int64_t quads = (len - head) / zk::kQuad;

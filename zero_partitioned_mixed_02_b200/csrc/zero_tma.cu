@@ -32,7 +32,7 @@ constexpr int kHdrBytes = 1024;             // barriers and tile descriptors
 struct TileDesc {
     long long gi, si, oi;
     int n;
-    int pad;
+    int decay;
 };
 constexpr int kMaxStages = 8;
 static_assert(16 * kMaxStages + sizeof(TileDesc) * kMaxStages <= kHdrBytes, "header overflow");
@@ -154,6 +154,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
             d.si = run.state_begin + e0;
             d.oi = run.out_begin + e0;
             d.n = n;
+            d.decay = run.decay;
             char* sp = stage0 + st * stage_bytes;
             const unsigned full = full0 + 8 * st;
             mbar_expect_tx(full, (unsigned)n * (unsigned)(2 * nd + 12));
@@ -209,11 +210,12 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * st);  // the warp is done reading the stage
         if (active) {
+            const float wd = d.decay ? L.c.wd : 0.0f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 g[j] = __fmul_rn(g[j], L.c.inv_scale);
                 bad |= nonfinite(g[j]);
-                adam1(g[j], w[j], m[j], v[j], L.c);
+                adam1(g[j], w[j], m[j], v[j], L.c, wd);
             }
             // state indices are 4-element and output indices 8-element aligned
             // with the gradient index (the host's eligibility rule)
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
         sd.chunk_begin = 0;
         sd.head = run.head;
         sd.tail = run.tail;
+        sd.decay = run.decay;
         const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
         step_scalar<K_STEP_FUSED>(b, L, b.grads, b.outs, sd, e, bad);
     }
