@@ -119,13 +119,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_FILES = ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu", "zero_tma.cu")
+# device sources each variant's step kernel is built from
+KERNEL_FILES = {
+    "fused-tma": ("zero_device.cuh", "zero_internal.h", "zero_tma.cu"),
+    "fused": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
+    "two-pass": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
+    "two-pass-bf16": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
+}
 
 
-def kernel_sha():
-    """Hash of the device sources the step kernels are built from."""
+def kernel_sha(variant):
+    """Hash of the device sources the variant's step kernel is built from."""
     h = hashlib.sha256()
-    for name in KERNEL_FILES:
+    for name in KERNEL_FILES[variant]:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
@@ -141,7 +147,7 @@ def recorded_traffic(wl_name, variant):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", txt)
-    if not m or not h or h.group(1) != kernel_sha():
+    if not m or not h or h.group(1) != kernel_sha(variant):
         return None
     return float(m.group(1))
 
@@ -474,7 +480,7 @@ def run_ours(args):
     k_s = statistics.mean(kern_ms) / 1e3
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
-    traffic = None if bf16 else recorded_traffic(args.workload, args.variant)
+    traffic = recorded_traffic(args.workload, args.variant + ("-bf16" if bf16 else ""))
     if bf16:
         kname = "step_kernel<reduce,bf16>+<update,bf16>"
     elif args.variant == "two-pass":

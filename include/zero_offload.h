@@ -59,7 +59,7 @@ extern "C" {
 #endif
 
 #define ZERO_OFFLOAD_SLOTS 3                      /* chunks in flight per direction */
-#define ZERO_OFFLOAD_DEFAULT_CHUNK (1LL << 24)    /* largest default chunk (elements) */
+#define ZERO_OFFLOAD_DEFAULT_CHUNK (1LL << 22)    /* largest default chunk (elements) */
 
 typedef struct zero_offload_ledger {
     int64_t state_elems;        /* elements of each host state array */

@@ -121,8 +121,8 @@ def test_offload_ledger(stage):
     assert L.host_staging_bytes >= A.ZERO_OFFLOAD_SLOTS * 6 * 1024
     # the default chunk, shrunk to the state for a small problem
     assert A.zero_offload_bytes(cfg, 0).chunk_elems == (psi + 255) // 256 * 256
-    big = A.Config(1 << 26, 8, 2)
-    assert A.zero_offload_bytes(big, 0).chunk_elems == 1 << 23  # 8 chunks
+    mid = A.Config(1 << 24, 8, 2)
+    assert A.zero_offload_bytes(mid, 0).chunk_elems == 1 << 21  # 8 chunks
     huge = A.Config(1 << 30, 8, 2)
     assert A.zero_offload_bytes(huge, 0).chunk_elems == A.ZERO_OFFLOAD_DEFAULT_CHUNK
     # rank view: one partition

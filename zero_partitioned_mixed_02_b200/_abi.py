@@ -87,7 +87,7 @@ class zero_offload_ledger(C.Structure):
 
 
 ZERO_OFFLOAD_SLOTS = 3
-ZERO_OFFLOAD_DEFAULT_CHUNK = 1 << 24
+ZERO_OFFLOAD_DEFAULT_CHUNK = 1 << 22
 
 _lib = None
 
