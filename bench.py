@@ -49,10 +49,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
-    p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass"], default="fused-tma")
+    p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass", "two-pass-tma"], default="fused-tma")
     p.add_argument("--precision", choices=["fp16", "bf16"], default="fp16",
                    help="bf16: bfloat16 gradients and parameters without fp32 master weights "
-                        "(runs the two-pass kernels)")
+                        "(two-pass variants only; a fused --variant becomes two-pass-tma)")
     p.add_argument("--async", dest="async_steps", action="store_true",
                    help="time zero_step_async: steps enqueued back to back, no host sync")
     p.add_argument("--prefetch", action="store_true",
@@ -121,10 +121,12 @@ def measured_peak():
 
 # device sources each variant's step kernel is built from
 KERNEL_FILES = {
-    "fused-tma": ("zero_device.cuh", "zero_internal.h", "zero_tma.cu"),
+    "fused-tma": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma.cu"),
     "fused": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
     "two-pass": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
     "two-pass-bf16": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
+    "two-pass-tma": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma_pass.cu"),
+    "two-pass-tma-bf16": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma_pass.cu"),
 }
 
 
@@ -367,10 +369,11 @@ def run_ours(args):
 
     wl = workload(args.workload)
     bf16 = args.precision == "bf16"
-    if bf16:
-        args.variant = "two-pass"  # without a master only the two-pass step exists
+    if bf16 and args.variant in ("fused", "fused-tma"):
+        args.variant = "two-pass-tma"  # without a master only the two-pass step exists
     variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
-               "fused-tma": A.ZERO_VARIANT_FUSED_TMA}[args.variant]
+               "fused-tma": A.ZERO_VARIANT_FUSED_TMA, "two-pass-tma": A.ZERO_VARIANT_TWO_PASS_TMA}[args.variant]
+    two_pass = args.variant.startswith("two-pass")
     cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, variant=variant,
                    tensors=wl.tensors,
                    precision=A.ZERO_PRECISION_BF16 if bf16 else A.ZERO_PRECISION_FP16)
@@ -470,9 +473,9 @@ def run_ours(args):
         dist.barrier()
 
     n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant, bf16)
-    launches_per_step = (2 if args.variant == "two-pass" else 1) + len(order)
+    launches_per_step = (2 if two_pass else 1) + len(order)
     if args.async_steps:  # + the conditional roll-back (fused variants) and the commit kernel
-        launches_per_step += 1 if args.variant == "two-pass" else 2
+        launches_per_step += 1 if two_pass else 2
     step_s = total_ms / 1e3 / args.steps
     value = whole_job_value(n, args.steps, world, total_ms)
     peak, peak_src = measured_peak()
@@ -481,10 +484,11 @@ def run_ours(args):
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
     traffic = recorded_traffic(args.workload, args.variant + ("-bf16" if bf16 else ""))
-    if bf16:
-        kname = "step_kernel<reduce,bf16>+<update,bf16>"
-    elif args.variant == "two-pass":
-        kname = "step_kernel<reduce>+<update>"
+    codec = ",bf16" if bf16 else ""
+    if two_pass and A.zero_uses_tma(h):
+        kname = f"pass_tma_kernel<reduce{codec}>+<update{codec}>"
+    elif two_pass:
+        kname = f"step_kernel<reduce{codec}>+<update{codec}>"
     elif A.zero_uses_tma(h):
         kname = "step_tma_kernel"
     else:

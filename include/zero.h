@@ -86,6 +86,15 @@ extern "C" {
  * in 16-byte phase with their place in the output); a gather whose bounded
  * wait gave up is reported by the next zero_step as ZERO_ERR_INTERNAL. */
 #define ZERO_VARIANT_FUSED_TMA 2
+/* The two passes of ZERO_VARIANT_TWO_PASS with their loads done by the Tensor
+ * Memory Accelerator (bulk copies of gradient, reduced-gradient, moment and
+ * weight tiles into shared memory, as in ZERO_VARIANT_FUSED_TMA); same
+ * arithmetic, bytes and workspace as ZERO_VARIANT_TWO_PASS, under the same
+ * eligibility rule as ZERO_VARIANT_FUSED_TMA (otherwise the plain two-pass
+ * kernels run). Valid with both precisions. The update pass writes in place:
+ * should one of its bounded waits give up (ZERO_ERR_INTERNAL), part of the
+ * state may already be updated. */
+#define ZERO_VARIANT_TWO_PASS_TMA 3
 
 #define ZERO_MAX_ND 1024
 
@@ -101,8 +110,8 @@ extern "C" {
  * to bfloat16 (nearest even) into every replica / the shard. Updates smaller
  * than half a bfloat16 spacing are lost ([P1] "Why you can't just delete the
  * fp32 copies" describes the same loss for fp16). Requires
- * ZERO_VARIANT_TWO_PASS (without a master a speculative write cannot be rolled
- * back). master_init of zero_init is rounded to bfloat16; the ledger's master
+ * ZERO_VARIANT_TWO_PASS or ZERO_VARIANT_TWO_PASS_TMA (without a master a
+ * speculative write cannot be rolled back). master_init of zero_init is rounded to bfloat16; the ledger's master
  * offsets are -1 and zero_current_state returns master = NULL; for
  * zero_set_state master may be NULL (the parameters stay as they are) or
  * fp32 values in state order to round into the parameters. */
@@ -129,7 +138,7 @@ typedef struct zero_config {
     int32_t stage;     /* ZeRO stage 1, 2 or 3 */
     int32_t rank_view; /* -1: emulate all Nd ranks; r >= 0 (stage 1/2 only):
                           act as rank r alone, owning partition r */
-    int32_t variant;   /* ZERO_VARIANT_FUSED, _TWO_PASS or _FUSED_TMA */
+    int32_t variant;   /* ZERO_VARIANT_FUSED, _TWO_PASS, _FUSED_TMA or _TWO_PASS_TMA */
     int32_t n_tensors; /* 0 allowed for stage 1/2 (one flat tensor) */
     int32_t precision; /* ZERO_PRECISION_FP16 (0) or ZERO_PRECISION_BF16 */
     const zero_tensor* tensors; /* host array of n_tensors; sum of numel == psi;

@@ -113,6 +113,15 @@ int zero_offload_init(const zero_config* cfg, int64_t chunk_elems, void* device_
 int zero_offload_step(zero_offload_handle* h, const uint16_t* const* grads, float loss_scale,
                       const zero_hyper* hp, void* stream);
 
+/* Checkpoint / resume: replace the host state with master, m, v (HOST
+ * arrays of state_elems floats in state order, e.g. saved from
+ * zero_offload_state) and the step count t, and rewrite the fp16 parameters
+ * from the restored master on `stream` (complete when the call returns).
+ * ZERO_OK, ZERO_ERR_ARG (NULL array with state_elems > 0, t < 0, or a handle
+ * refusing steps), ZERO_ERR_CUDA. */
+int zero_offload_set_state(zero_offload_handle* h, const float* master, const float* m, const float* v,
+                           int64_t t, void* stream);
+
 /* Host pointers to the live state (state order) and the step count. */
 int zero_offload_state(zero_offload_handle* h, const float** master, const float** m, const float** v,
                        int64_t* t);

@@ -214,6 +214,14 @@ def test_bf16_precision_ledger_and_validation():
                                           tensors=tensors))
         # the master array is gone from the workspace
         assert L16.workspace_bytes - L.workspace_bytes >= 4 * psi
+    # both two-pass variants take bfloat16; the TMA one has the same workspace
+    # plus its second run table
+    Lt = A.zero_state_bytes(A.Config(psi, nd, 2, variant=A.ZERO_VARIANT_TWO_PASS_TMA, tensors=tensors,
+                                     precision=BF))
+    L2 = A.zero_state_bytes(A.Config(psi, nd, 2, variant=A.ZERO_VARIANT_TWO_PASS, tensors=tensors,
+                                     precision=BF))
+    assert list(Lt.exact_bytes) == list(L2.exact_bytes) and Lt.off_reduced > 0
+    assert 0 <= Lt.workspace_bytes - L2.workspace_bytes <= 4096
     for kw in (dict(precision=2), dict(precision=BF, variant=A.ZERO_VARIANT_FUSED),
                dict(precision=BF, variant=A.ZERO_VARIANT_FUSED_TMA)):
         with pytest.raises(A.ZeroError) as ei:

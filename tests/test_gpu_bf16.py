@@ -31,6 +31,8 @@ if not torch.cuda.is_available():
 
 BF = A.ZERO_PRECISION_BF16
 TWO = A.ZERO_VARIANT_TWO_PASS
+TWO_TMA = A.ZERO_VARIANT_TWO_PASS_TMA
+BF_VARIANTS = [TWO, TWO_TMA]
 NO_DECAY = A.ZERO_TENSOR_NO_DECAY
 
 
@@ -48,7 +50,7 @@ def _perm(numel, nd, stage, psi, view):
 
 class Bf16Case:
     def __init__(self, psi, nd, stage, *, tensors=None, view=-1, loss_scale=1.0, hp=None,
-                 master_dist=None, grad_sigma=1e-3, seed=0):
+                 master_dist=None, grad_sigma=1e-3, seed=0, variant=TWO):
         self.psi, self.nd, self.stage, self.view = psi, nd, stage, view
         self.tensors = tensors or [(psi, 0)]
         self.numel = [t[0] for t in self.tensors]
@@ -57,7 +59,7 @@ class Bf16Case:
         self.hp = hp or dict(lr=1e-2, weight_decay=0.1)
         self.grad_sigma = grad_sigma
         self.seed = seed
-        self.cfg = A.Config(psi, nd, stage, rank_view=view, variant=TWO, tensors=tensors, precision=BF)
+        self.cfg = A.Config(psi, nd, stage, rank_view=view, variant=variant, tensors=tensors, precision=BF)
         self.L = A.zero_state_bytes(self.cfg)
         self.b0, self.e0 = Z.partition(psi, nd, view) if view >= 0 else (0, psi)
         n_own = self.e0 - self.b0
@@ -171,26 +173,41 @@ def _tensors(rng, psi, n_max=7):
     return out
 
 
+@pytest.mark.parametrize("variant", BF_VARIANTS)
 @pytest.mark.parametrize("stage", [1, 2, 3])
 @pytest.mark.parametrize("nd", [1, 2, 3, 5, 8, 9])
-def test_bf16_grid(nd, stage):
+def test_bf16_grid(nd, stage, variant):
     rng = np.random.default_rng(7 * nd + stage)
     for psi in (1, 7, 64, 257, 4099, 70001):
-        _run(Bf16Case(psi, nd, stage, tensors=_tensors(rng, psi), loss_scale=float(2 ** (psi % 9))), 2)
+        _run(Bf16Case(psi, nd, stage, tensors=_tensors(rng, psi), loss_scale=float(2 ** (psi % 9)),
+                      variant=variant), 2)
 
 
+@pytest.mark.parametrize("variant", BF_VARIANTS)
 @pytest.mark.parametrize("view", [0, 1, 3])
-def test_bf16_rank_view_out_of_phase(view):
+def test_bf16_rank_view_out_of_phase(view, variant):
     # 70001 / 4: partitions start at odd offsets, so the parameter reads are
     # out of phase with the gradient index
     rng = np.random.default_rng(view)
-    _run(Bf16Case(70001, 4, 1, tensors=_tensors(rng, 70001), view=view), 2)
+    _run(Bf16Case(70001, 4, 1, tensors=_tensors(rng, 70001), view=view, variant=variant), 2)
 
 
-def test_bf16_skips_are_global():
+@pytest.mark.parametrize("nd", [1, 2, 4, 8])
+def test_bf16_tma_passes_engage(nd):
+    """Partitions in 16-byte phase: the TMA-staged passes run (whole tiles,
+    partial tiles, heads and tails), with an excluded tensor."""
+    for psi in (1024, 8 * 1024 * 5 + 200, 1_000_003):
+        cut = psi // 3 // 64 * 64
+        c = Bf16Case(psi, nd, 2, tensors=[(cut, 0), (psi - cut, 0, NO_DECAY)], variant=TWO_TMA)
+        assert A.zero_uses_tma(c.h)
+        _run(c, 2)
+
+
+@pytest.mark.parametrize("variant", BF_VARIANTS)
+def test_bf16_skips_are_global(variant):
     psi = 20_000
-    assert _run(Bf16Case(psi, 8, 2), 3, inject=[(1, 7, 5, 0x7F80)]) == [False, True, False]
-    c = Bf16Case(psi, 4, 3, tensors=[(12_000, 0), (8_000, 1, NO_DECAY)])
+    assert _run(Bf16Case(psi, 8, 2, variant=variant), 3, inject=[(1, 7, 5, 0x7F80)]) == [False, True, False]
+    c = Bf16Case(psi, 4, 3, tensors=[(12_000, 0), (8_000, 1, NO_DECAY)], variant=variant)
     assert _run(c, 2, inject=[(0, 0, psi - 1, 0xFFC0)]) == [True, False]
 
 
@@ -202,8 +219,9 @@ def test_bf16_subnormal_and_tiny_values():
     _run(c, 2)
 
 
-def test_bf16_asynchronous_steps():
-    c = Bf16Case(50_001, 4, 2, tensors=[(30_000, 0), (20_001, 1, NO_DECAY)], loss_scale=1.0)
+@pytest.mark.parametrize("variant", BF_VARIANTS)
+def test_bf16_asynchronous_steps(variant):
+    c = Bf16Case(50_000, 4, 2, tensors=[(30_000, 0), (20_000, 1, NO_DECAY)], loss_scale=1.0, variant=variant)
     c.check("after init")
     A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], A.zero_scaler(256.0, 2.0, 0.5, 2), 0.9, 0.999,
                        c.stream)

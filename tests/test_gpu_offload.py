@@ -201,3 +201,34 @@ def test_offload_init_validation():
         assert ei.value.code == code
     h = A.zero_offload_init(**args)
     A.zero_offload_destroy(h)
+
+
+def test_offload_checkpoint_resume():
+    """Two steps, save the host state; a fresh handle restored from it and
+    continued equals the original run continued, bit for bit (parameters
+    rewritten from the restored master)."""
+    psi, nd = 60_000, 4
+    tensors = [(35_000, 0), (25_000, 1, ND_FLAG)]
+    a = OffloadCase(psi, nd, 2, tensors=tensors, chunk=4096)
+    for s in range(2):
+        a.step(a.grads(s))
+    E = a.L.state_elems
+    saved = a.state[:3 * E].copy()
+    for s in range(2, 4):
+        a.step(a.grads(s))
+    a.check("original run")
+    b = OffloadCase(psi, nd, 2, tensors=tensors, chunk=4096)
+    A.zero_offload_set_state(b.h, saved[:E].ctypes.data, saved[E:2 * E].ctypes.data,
+                             saved[2 * E:].ctypes.data, 2, b.stream)
+    torch.cuda.synchronize()
+    for k, buf in enumerate(b.bufs):
+        compare_f16(buf.bits(), Z.f16_from_f32(saved[:E]), f"replica {k} after restore")
+    # continue b from the restored state; its oracle mirror is a's
+    b.w, b.m, b.v, b.t = saved[:E].copy(), saved[E:2 * E].copy(), saved[2 * E:].copy(), 2
+    b.p16 = Z.f16_from_f32(b.w)
+    for s in range(2, 4):
+        b.step(b.grads(s))
+    b.check("resumed run")
+    assert (b.state[:3 * E].view(np.uint32) == a.state[:3 * E].view(np.uint32)).all()
+    a.close()
+    b.close()

@@ -24,7 +24,9 @@ from gpu_common import (GuardedF16, GuardedWorkspace, SENTINEL16, compare_f16, c
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA]
+VARIANTS = [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA,
+            A.ZERO_VARIANT_TWO_PASS_TMA]
+TMA_VARIANTS = [A.ZERO_VARIANT_FUSED_TMA, A.ZERO_VARIANT_TWO_PASS_TMA]
 
 if not torch.cuda.is_available():  # collected on CPU machines, never run there
     pytest.skip("needs a GPU", allow_module_level=True)
@@ -303,43 +305,48 @@ def test_workload_precision_stress(variant):
     c.close()
 
 
+@pytest.mark.parametrize("variant", TMA_VARIANTS)
 @pytest.mark.parametrize("nd", [1, 2, 3, 4, 8])
-def test_tma_path_runs_and_matches(nd):
+def test_tma_path_runs_and_matches(nd, variant):
     # sizes with whole tiles, partial tiles, and heads/tails around them; every
-    # partition in 16-byte phase, so the TMA kernel is the one that runs
+    # partition in 16-byte phase, so the TMA kernels are the ones that run
     for psi in [64, 1024, 1024 * 3 + 8, 8 * 1024 * 5 + 200, 250_000, 1_000_003]:
-        c = Case(psi, nd, 2, A.ZERO_VARIANT_FUSED_TMA, hp=dict(weight_decay=0.01))
+        c = Case(psi, nd, 2, variant, hp=dict(weight_decay=0.01))
         assert c.uses_tma()
         assert _run(c, 2) == [False, False]
-    c = Case(4099, 9, 2, A.ZERO_VARIANT_FUSED_TMA)  # Nd > 8: the plain fused kernel
+    c = Case(4099, 9, 2, variant)  # Nd > 8: the plain kernels
     assert not c.uses_tma()
     _run(c, 1)
 
 
+@pytest.mark.parametrize("variant", TMA_VARIANTS)
 @pytest.mark.parametrize("nd", [2, 4, 8])
-def test_tma_stage3_eligible_tensors(nd):
+def test_tma_stage3_eligible_tensors(nd, variant):
     # tensor sizes that keep every chunk in 16-byte phase: multiples of 8 * nd
     rng = np.random.default_rng(nd)
     for trial in range(4):
         sizes = [int(x) * 8 * nd for x in rng.integers(1, 400, size=6)]
         units = [0, 0, 1, 1, 1, 2]
-        c = Case(sum(sizes), nd, 3, A.ZERO_VARIANT_FUSED_TMA, tensors=list(zip(sizes, units)))
+        c = Case(sum(sizes), nd, 3, variant, tensors=list(zip(sizes, units)))
         assert c.uses_tma()
         assert _run(c, 2, inject=[(1, nd - 1, 5, 0x7C00)]) == [False, True]
 
 
-def test_tma_skip_restores_params():
-    c = Case(200_000, 8, 1, A.ZERO_VARIANT_FUSED_TMA)
+@pytest.mark.parametrize("variant", TMA_VARIANTS)
+def test_tma_skip_restores_params(variant):
+    c = Case(200_000, 8, 1, variant)
     assert c.uses_tma()
     assert _run(c, 3, inject=[(1, 7, 123_456, 0x7E00)]) == [False, True, False]
 
 
-def test_tma_wait_that_gives_up_is_reported_and_rolled_back():
+@pytest.mark.parametrize("variant", TMA_VARIANTS)
+def test_tma_wait_that_gives_up_is_reported_and_rolled_back(variant):
     # A tile left unarmed makes the kernel's bounded waits run out (no fault):
     # the step returns ZERO_ERR_INTERNAL, nothing changes, and the next step
-    # is exactly the oracle's next step.
+    # is exactly the oracle's next step. For the two-pass TMA variant the
+    # unarmed tile is in the reduce pass; the update pass then does nothing.
     for psi, nd, stage in [(200_000, 8, 1), (50_000, 2, 2)]:
-        c = Case(psi, nd, stage, A.ZERO_VARIANT_FUSED_TMA)
+        c = Case(psi, nd, stage, variant)
         assert c.uses_tma()
         c.check("after init")
         c.step(c.grads(0))
@@ -358,10 +365,11 @@ def test_tma_wait_that_gives_up_is_reported_and_rolled_back():
         c.close()
 
 
-def test_tma_gather_wait_that_gives_up_is_reported():
+@pytest.mark.parametrize("variant", TMA_VARIANTS)
+def test_tma_gather_wait_that_gives_up_is_reported(variant):
     nd = 4
     sizes = [8 * nd * 700, 8 * nd * 300, 8 * nd * 1200]
-    c = Case(sum(sizes), nd, 3, A.ZERO_VARIANT_FUSED_TMA, tensors=list(zip(sizes, [0, 1, 1])))
+    c = Case(sum(sizes), nd, 3, variant, tensors=list(zip(sizes, [0, 1, 1])))
     assert c.uses_tma()
     c.step(c.grads(0))
     c.check("after step 0")
@@ -561,7 +569,7 @@ def test_no_decay_gpt2_structure(stage, variant):
     psi = sum(n for n, _, _ in tensors)
     c = MaskedCase(psi, 8, stage, variant, tensors=tensors, loss_scale=4096.0,
                    hp=dict(lr=1e-3, weight_decay=0.01))
-    if variant == A.ZERO_VARIANT_FUSED_TMA and stage == 2:
+    if variant in TMA_VARIANTS and stage == 2:
         assert c.uses_tma()  # stage-3 shards of odd-sized tensors are out of 16-byte phase
     _run(c, 3, inject=[(1, 5, psi - 1, 0x7C00)])
 

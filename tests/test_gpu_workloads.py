@@ -160,16 +160,131 @@ def _run(wl: W.Workload, variant: int):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA,
+                                     A.ZERO_VARIANT_TWO_PASS_TMA])
 def test_gpt2_1p5b_stage2(variant):
     _run(W.gpt2_1p5b(), variant)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA,
+                                     A.ZERO_VARIANT_TWO_PASS_TMA])
 def test_running_example_7p5b_rank_view(variant):
     _run(W.running_example_7p5b(), variant)
 
 
-@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA])
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA,
+                                     A.ZERO_VARIANT_TWO_PASS_TMA])
 def test_llama_2p7b_stage3(variant):
     _run(W.llama_2p7b(), variant)
+
+
+def _bf16_grad(k, step, wl, b0, n_own, out, s):
+    """The generator's binary32 gradient rounded to bfloat16 on the device,
+    the way the benchmark makes it."""
+    tmp = torch.empty(n_own, dtype=torch.float32, device="cuda")
+    S.fill_f32(tmp.data_ptr(), n_own, b0, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad, s)
+    out.copy_(tmp.to(torch.bfloat16).view(torch.int16))
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_TWO_PASS_TMA])
+def test_gpt2_1p5b_bf16_without_master(variant):
+    """The bfloat16 step without master weights at full size (bench
+    --precision bf16): sampled m, v and parameters against the oracle's
+    zr_bf16_step, every replica identical."""
+    wl = W.gpt2_1p5b()
+    rng = np.random.default_rng(321)
+    cfg = A.Config(wl.psi, wl.nd, wl.stage, variant=variant, tensors=wl.tensors,
+                   precision=A.ZERO_PRECISION_BF16)
+    L = A.zero_state_bytes(cfg)
+    n = wl.psi
+    s = torch.cuda.current_stream().cuda_stream
+    ws = torch.empty(L.workspace_bytes, dtype=torch.uint8, device="cuda")
+    kmaster = S.key(wl.seed, S.STREAM_MASTER, 0, 0)
+    m_init = torch.empty(n, dtype=torch.float32, device="cuda")
+    S.fill_f32(m_init.data_ptr(), n, 0, kmaster, wl.master, s)
+    bufs = [torch.full((n,), SENT, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    grads = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    h = A.zero_init(cfg, ws.data_ptr(), L.workspace_bytes, m_init.data_ptr(), [b.data_ptr() for b in bufs], s)
+    del m_init
+    idx = _samples(wl, 0, n, rng)
+    w16 = Z.bf16_from_f32(S.host_f32_at(idx, kmaster, wl.master))
+    m_o, v_o, t_o = np.zeros(idx.size, np.float32), np.zeros(idx.size, np.float32), 0
+    steps = 3
+    for step in range(steps):
+        for k in range(wl.nd):
+            _bf16_grad(k, step, wl, 0, n, grads[k], s)
+        rc = A.zero_step(h, [g.data_ptr() for g in grads], wl.loss_scale, hyper(**wl.hyper), s)
+        gs = [Z.bf16_from_f32(S.host_f32_at(idx, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad))
+              for k in range(wl.nd)]
+        sk, t_o = Z.bf16_step(gs, w16, m_o, v_o, wl.loss_scale, Z.hyper(**wl.hyper), t_o)
+        assert rc == A.ZERO_OK and not sk
+    wp, mp, vp, t = A.zero_current_state(h)
+    assert wp is None and t == t_o == steps
+    base = ws.data_ptr()
+    sel = torch.from_numpy(idx).cuda()
+    compare_f32(host_f32(ws[mp - base: mp - base + 4 * n].view(torch.float32)[sel]), m_o, "m (sampled)")
+    compare_f32(host_f32(ws[vp - base: vp - base + 4 * n].view(torch.float32)[sel]), v_o, "v (sampled)")
+    for k, b in enumerate(bufs):
+        compare_f16(host_u16(b[sel]), w16, f"bf16 replica {k} (sampled)")
+    for b in bufs[1:]:
+        assert torch.equal(b, bufs[0]), "replicas differ"
+    A.zero_destroy(h)
+    del ws, bufs, grads
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_gpt2_1p5b_offload():
+    """The offloaded step at full size with the default chunk and all host
+    threads (bench --offload): the host master, m, v sampled against the
+    oracle, every replica identical and equal to fp16 of the host master."""
+    import os
+
+    wl = W.gpt2_1p5b()
+    rng = np.random.default_rng(654)
+    cfg = A.Config(wl.psi, wl.nd, wl.stage, tensors=wl.tensors)
+    L = A.zero_offload_bytes(cfg, 0)
+    n = wl.psi
+    s = torch.cuda.current_stream().cuda_stream
+    kmaster = S.key(wl.seed, S.STREAM_MASTER, 0, 0)
+    m_dev = torch.empty(n, dtype=torch.float32, device="cuda")
+    S.fill_f32(m_dev.data_ptr(), n, 0, kmaster, wl.master, s)
+    master_init = m_dev.cpu().numpy()
+    del m_dev
+    state = np.empty(3 * n, np.float32)
+    dws = torch.empty(L.device_bytes, dtype=torch.uint8, device="cuda")
+    staging = torch.empty(L.host_staging_bytes, dtype=torch.uint8, pin_memory=True)
+    bufs = [torch.full((n,), SENT, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    grads = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(wl.nd)]
+    threads = len(os.sched_getaffinity(0))
+    h = A.zero_offload_init(cfg, 0, dws.data_ptr(), L.device_bytes, staging.data_ptr(), L.host_staging_bytes,
+                            state.ctypes.data, master_init.ctypes.data, [b.data_ptr() for b in bufs],
+                            threads, s)
+    del master_init
+    idx = _samples(wl, 0, n, rng)
+    w_o = S.host_f32_at(idx, kmaster, wl.master)
+    m_o, v_o, p_o, t_o = np.zeros_like(w_o), np.zeros_like(w_o), Z.f16_from_f32(w_o), 0
+    steps = 2
+    for step in range(steps):
+        for k in range(wl.nd):
+            S.fill_f16(grads[k].data_ptr(), n, 0, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad, s)
+        rc = A.zero_offload_step(h, [g.data_ptr() for g in grads], wl.loss_scale, hyper(**wl.hyper), s)
+        gs = [S.host_f16_bits_at(idx, S.key(wl.seed, S.STREAM_GRAD, step, k), wl.grad) for k in range(wl.nd)]
+        sk, t_o = Z.dp_step(gs, w_o, m_o, v_o, p_o, wl.loss_scale, Z.hyper(**wl.hyper), t_o)
+        assert rc == A.ZERO_OK and not sk
+    torch.cuda.synchronize()
+    assert A.zero_offload_state(h)[3] == t_o == steps
+    compare_f32(state[idx], w_o, "host master (sampled)")
+    compare_f32(state[n + idx], m_o, "host m (sampled)")
+    compare_f32(state[2 * n + idx], v_o, "host v (sampled)")
+    sel = torch.from_numpy(idx).cuda()
+    for k, b in enumerate(bufs):
+        compare_f16(host_u16(b[sel]), p_o, f"replica {k} (sampled)")
+    for b in bufs[1:]:
+        assert torch.equal(b, bufs[0]), "replicas differ"
+    half_master = torch.from_numpy(state[:n]).cuda().half().view(torch.int16)
+    assert torch.equal(bufs[0], half_master), "fp16 params != fp16(host master) somewhere"
+    A.zero_offload_destroy(h)
+    del dws, bufs, grads, half_master, state
+    gc.collect()
+    torch.cuda.empty_cache()

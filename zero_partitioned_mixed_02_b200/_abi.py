@@ -30,6 +30,7 @@ ZERO_PRECISION_BF16 = 1
 ZERO_VARIANT_FUSED = 0
 ZERO_VARIANT_TWO_PASS = 1
 ZERO_VARIANT_FUSED_TMA = 2
+ZERO_VARIANT_TWO_PASS_TMA = 3
 ZERO_MAX_ND = 1024
 
 
@@ -139,6 +140,7 @@ def lib():
             "zero_offload_step": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P]),
             "zero_offload_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                              C.POINTER(C.c_int64)]),
+            "zero_offload_set_state": (C.c_int, [P, P, P, P, C.c_int64, P]),
             "zero_offload_host_update": (C.c_int, [P, P, P, P, P, C.c_int64, C.POINTER(zero_hyper),
                                                    C.c_int64, C.c_int, C.c_int]),
             "zero_offload_destroy": (None, [P]),
@@ -333,6 +335,10 @@ def zero_offload_state(h: int) -> tuple[int, int, int, int]:
     _check(lib().zero_offload_state(h, C.byref(w), C.byref(m), C.byref(v), C.byref(t)),
            "zero_offload_state")
     return w.value, m.value, v.value, t.value
+
+
+def zero_offload_set_state(h: int, master: int, m: int, v: int, t: int, stream: int) -> None:
+    _check(lib().zero_offload_set_state(h, master, m, v, int(t), stream), "zero_offload_set_state")
 
 
 def zero_offload_host_update(g: int, w: int, m: int, v: int, p16: int, n: int, hp: zero_hyper, t: int,

@@ -29,6 +29,11 @@ int64_t align_up(int64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// fused variants: one pass into a second state buffer, roll-back by re-cast;
+// two-pass variants: reduce into a scratch, then update in place
+bool is_fused(int variant) { return variant == ZERO_VARIANT_FUSED || variant == ZERO_VARIANT_FUSED_TMA; }
+bool is_tma(int variant) { return variant == ZERO_VARIANT_FUSED_TMA || variant == ZERO_VARIANT_TWO_PASS_TMA; }
+
 // Cut a run at the first line-aligned gradient index and give it its chunks.
 void add_run(std::vector<zk::SegDesc>& v, int64_t* chunks, int64_t grad_begin, int64_t state_begin,
              int64_t out_begin, int64_t len, int decay = 1)
@@ -60,12 +65,12 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
     if (cfg->nd < 1 || cfg->nd > ZERO_MAX_ND) return ZERO_ERR_ARG;
     if (cfg->stage < 1 || cfg->stage > 3) return ZERO_ERR_ARG;
     if (cfg->variant != ZERO_VARIANT_FUSED && cfg->variant != ZERO_VARIANT_TWO_PASS &&
-        cfg->variant != ZERO_VARIANT_FUSED_TMA)
+        cfg->variant != ZERO_VARIANT_FUSED_TMA && cfg->variant != ZERO_VARIANT_TWO_PASS_TMA)
         return ZERO_ERR_ARG;
     if (cfg->n_tensors < 0) return ZERO_ERR_ARG;
     if (cfg->precision != ZERO_PRECISION_FP16 && cfg->precision != ZERO_PRECISION_BF16) return ZERO_ERR_ARG;
     // without a master nothing can be rolled back: the two-pass step only
-    if (cfg->precision == ZERO_PRECISION_BF16 && cfg->variant != ZERO_VARIANT_TWO_PASS) return ZERO_ERR_ARG;
+    if (cfg->precision == ZERO_PRECISION_BF16 && is_fused(cfg->variant)) return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
     if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
     if (cfg->stage == 3 && cfg->n_tensors == 0) return ZERO_ERR_ARG;
@@ -204,7 +209,7 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             U.n_segs = (int64_t)L->gather_segs.size() - U.seg0;
             U.n_chunks = chunks;
             L->transient_elems = std::max(L->transient_elems, U.numel);
-            if (cfg->variant == ZERO_VARIANT_FUSED_TMA) {
+            if (is_tma(cfg->variant)) {
                 bool ok = U.n_segs > 0;
                 for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
                     const zk::SegDesc& g = L->gather_segs[i];
@@ -236,13 +241,15 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
         }
     }
 
-    // ---- TMA run table: the same runs, bodies cut at 8-element multiples ----
-    if (cfg->variant == ZERO_VARIANT_FUSED_TMA && nd <= zk::kTmaMaxNd) {
-        L->tma_shape = zk::tma_shape(L->n_out);
+    // ---- TMA run tables: the same runs, bodies cut at 8-element multiples ----
+    // Tiles are numbered per table for one tile size: the fused kernel's
+    // shape, or for the two-pass TMA variant the update pass's (tma_runs) and
+    // the reduce pass's (tma_runs_r).
+    if (is_tma(cfg->variant) && nd <= zk::kTmaMaxNd) {
         bool ok = true;
         for (const zk::SegDesc& d : L->step_segs)
             if ((d.state_begin - d.grad_begin) % 4 != 0 || (d.out_begin - d.grad_begin) % 8 != 0) ok = false;
-        if (ok) {
+        auto table = [&](int tile, std::vector<zk::TmaRun>& out, int64_t* tiles, int64_t* scal) {
             for (const zk::SegDesc& d : L->step_segs) {
                 zk::TmaRun t{};
                 t.decay = d.decay;
@@ -255,12 +262,22 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
                 const int64_t body = (d.len - head) / 8 * 8;
                 t.head = (int)head;
                 t.tail = (int)(d.len - head - body);
-                t.tile_begin = L->tma_tiles;
-                t.scal_begin = L->tma_scal;
-                L->tma_tiles += (body + L->tma_shape.tile - 1) / L->tma_shape.tile;
-                L->tma_scal += t.head + t.tail;
-                L->tma_runs.push_back(t);
+                t.tile_begin = *tiles;
+                t.scal_begin = *scal;
+                *tiles += (body + tile - 1) / tile;
+                *scal += t.head + t.tail;
+                out.push_back(t);
             }
+        };
+        if (ok) {
+            if (is_fused(cfg->variant)) {
+                L->tma_shape = zk::tma_shape(L->n_out);
+            } else {
+                L->tma_shape = zk::tma_pass_shape(zk::kPassUpdate, L->n_out);
+                L->tma_shape_r = zk::tma_pass_shape(zk::kPassReduce, L->n_out);
+                table(L->tma_shape_r.tile, L->tma_runs_r, &L->tma_tiles_r, &L->tma_scal_r);
+            }
+            table(L->tma_shape.tile, L->tma_runs, &L->tma_tiles, &L->tma_scal);
             L->tma_ok = !L->tma_runs.empty();
         }
     }
@@ -280,19 +297,23 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
     if (L->tma_ok) {
         L->off_tma_runs = off;
         off += align_up((int64_t)L->tma_runs.size() * sizeof(zk::TmaRun));
+        if (!L->tma_runs_r.empty()) {
+            L->off_tma_runs_r = off;
+            off += align_up((int64_t)L->tma_runs_r.size() * sizeof(zk::TmaRun));
+        }
     }
     if (!L->tma_gather.empty()) {
         L->off_tma_gather = off;
         off += align_up((int64_t)L->tma_gather.size() * sizeof(zk::TmaRun));
     }
-    const int n_buf = cfg->variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
+    const int n_buf = is_fused(cfg->variant) ? 2 : 1;
     for (int b = 0; b < n_buf; ++b)
         for (int k = 0; k < 3; ++k) {
             if (k == 0 && L->bf16) continue;  // no master: the parameters are the weights
             L->off_state[b][k] = off;
             off += align_up(L->state_elems * 4);
         }
-    if (cfg->variant == ZERO_VARIANT_TWO_PASS) {
+    if (!is_fused(cfg->variant)) {
         L->off_reduced = off;
         off += align_up(L->state_elems * 4);
     }
@@ -373,7 +394,9 @@ struct zero_handle {
     zk::SegDesc* d_gather_segs = nullptr;
     zk::TmaRun* d_tma_runs = nullptr;
     bool use_tma = false;  // TMA variant and its kernel fits on this device
-    int occ_tma = 0;
+    int occ_tma = 0;       // fused kernel, or the update pass of the two-pass TMA variant
+    zk::TmaRun* d_tma_runs_r = nullptr;  // two-pass TMA variant: the reduce pass's table
+    int occ_tma_r = 0;
     zk::TmaRun* d_tma_gather = nullptr;
     int occ_gather_tma = 0;
     int64_t hold_tile = -1;  // test hook for the bounded waits (zero_test_hold_tile)
@@ -410,6 +433,14 @@ struct zero_handle {
 
 namespace {
 
+int cuda_fail(zero_handle* h, cudaError_t e);
+
+// The TMA-staged step with arguments a: the fused kernel, or the reduce and
+// update passes (a.red set by the caller). hold_tile / wait_rounds: the test
+// hook, applied to the first launch only.
+cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_tile, unsigned wait_rounds,
+                            cudaStream_t s);
+
 int cuda_fail(zero_handle* h, cudaError_t e)
 {
     if (h) h->last_cuda = (int)e;
@@ -442,6 +473,47 @@ void bias_corrections(zero_handle* h, float b1, float b2, int64_t t, float* bc1,
     }
     *bc1 = (float)(1.0 - h->bc_p1);
     *bc2 = (float)(1.0 - h->bc_p2);
+}
+
+}  // namespace
+
+namespace {
+
+cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_tile, unsigned wait_rounds,
+                            cudaStream_t s)
+{
+    const Layout& L = h->L;
+    zk::TmaArgs ta{};
+    ta.b = a;
+    ta.err = h->d_flag + 1;
+    ta.wait_rounds = wait_rounds;
+    ta.hold_tile = hold_tile;
+    if (is_fused(L.variant)) {
+        ta.runs = h->d_tma_runs;
+        ta.n_runs = (int)L.tma_runs.size();
+        ta.n_tiles = L.tma_tiles;
+        ta.n_scal = L.tma_scal;
+        const int64_t cap = (int64_t)h->sms * h->occ_tma;
+        const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
+        return zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
+    }
+    ta.runs = h->d_tma_runs_r;
+    ta.n_runs = (int)L.tma_runs_r.size();
+    ta.n_tiles = L.tma_tiles_r;
+    ta.n_scal = L.tma_scal_r;
+    int64_t cap = (int64_t)h->sms * h->occ_tma_r;
+    int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles_r, (L.tma_scal_r + 255) / 256));
+    cudaError_t e = zk::launch_pass_tma(zk::kPassReduce, ta, (int)std::min(want, cap), s, L.bf16);
+    if (e != cudaSuccess) return e;
+    ta.runs = h->d_tma_runs;
+    ta.n_runs = (int)L.tma_runs.size();
+    ta.n_tiles = L.tma_tiles;
+    ta.n_scal = L.tma_scal;
+    ta.hold_tile = -1;
+    ta.wait_rounds = zk::kTmaWaitRounds;
+    cap = (int64_t)h->sms * h->occ_tma;
+    want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
+    return zk::launch_pass_tma(zk::kPassUpdate, ta, (int)std::min(want, cap), s, L.bf16);
 }
 
 }  // namespace
@@ -534,13 +606,19 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     h->d_gather_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_gather_segs);
     if (L.tma_ok) {
         h->d_tma_runs = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs);
-        e = zk::tma_prepare(L.tma_shape, L.nd, &h->occ_tma);
+        if (is_fused(L.variant)) {
+            e = zk::tma_prepare(L.tma_shape, L.nd, &h->occ_tma);
+            h->occ_tma_r = h->occ_tma;
+        } else {
+            h->d_tma_runs_r = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs_r);
+            e = zk::tma_pass_prepare(L.nd, L.n_out, L.bf16, &h->occ_tma_r, &h->occ_tma);
+        }
         if (e != cudaSuccess) {
             rc = cuda_fail(h, e);
             delete h;
             return rc;
         }
-        h->use_tma = h->occ_tma >= 1;
+        h->use_tma = h->occ_tma >= 1 && h->occ_tma_r >= 1;
     }
     if (!L.tma_gather.empty()) {
         h->d_tma_gather = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_gather);
@@ -565,6 +643,9 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && L.tma_ok)
         e = cudaMemcpyAsync(h->d_tma_runs, L.tma_runs.data(), L.tma_runs.size() * sizeof(zk::TmaRun),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !L.tma_runs_r.empty())
+        e = cudaMemcpyAsync(h->d_tma_runs_r, L.tma_runs_r.data(), L.tma_runs_r.size() * sizeof(zk::TmaRun),
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && !L.tma_gather.empty())
         e = cudaMemcpyAsync(h->d_tma_gather, L.tma_gather.data(), L.tma_gather.size() * sizeof(zk::TmaRun),
@@ -644,7 +725,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.c.wd = hp->weight_decay;
     bias_corrections(h, hp->beta1, hp->beta2, t_new, &a.c.bc1, &a.c.bc2);
 
-    const bool fused = L.variant != ZERO_VARIANT_TWO_PASS;
+    const bool fused = is_fused(L.variant);
     const int nxt = fused ? 1 - h->cur : h->cur;
     a.w_in = h->state(h->cur, 0);
     a.m_in = h->state(h->cur, 1);
@@ -654,19 +735,9 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.v_out = h->state(nxt, 2);
     if (L.step_chunks > 0) {
         if (h->use_tma) {
-            zk::TmaArgs ta{};
-            ta.b = a;
-            ta.runs = h->d_tma_runs;
-            ta.n_runs = (int)L.tma_runs.size();
-            ta.n_tiles = L.tma_tiles;
-            ta.n_scal = L.tma_scal;
-            ta.err = h->d_flag + 1;
-            ta.wait_rounds = h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds;
-            ta.hold_tile = h->hold_tile;
+            if (!fused) a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
+            e = launch_tma_step(h, a, h->hold_tile, h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds, s);
             h->hold_tile = -1;
-            const int64_t cap = (int64_t)h->sms * h->occ_tma;
-            const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
-            e = zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
         } else if (fused) {
             e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
         } else {
@@ -701,7 +772,7 @@ ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
         // switch (fused) or were never written (two-pass). The fused pass
         // already wrote fp16 parameters, so rewrite them from the unchanged
         // master.
-        if (L.variant != ZERO_VARIANT_TWO_PASS && L.step_chunks > 0) {
+        if (is_fused(L.variant) && L.step_chunks > 0) {
             zk::StepArgs a = h->args;
             a.w_in = h->state(h->cur, 0);
             e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
@@ -765,7 +836,7 @@ ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, cons
     c.b2 = beta2;
     c.interval = sc->growth_interval;
     c.cur = h->cur;
-    c.fused = L.variant != ZERO_VARIANT_TWO_PASS;
+    c.fused = is_fused(L.variant);
     e = cudaMemcpyAsync(h->d_ctrl, &c, sizeof(zk::Ctrl), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->d_flag, 0, sizeof(unsigned), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -804,24 +875,14 @@ ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
     a.c.eps = hp->eps;
     a.c.wd = hp->weight_decay;
     a.ctrl = h->d_ctrl;
-    const int nb = L.variant == ZERO_VARIANT_TWO_PASS ? 1 : 2;
+    const int nb = is_fused(L.variant) ? 2 : 1;
     for (int b = 0; b < 2; ++b)
         for (int k = 0; k < 3; ++k) a.st[b][k] = h->state(b < nb ? b : 0, k);
-    const bool fused = L.variant != ZERO_VARIANT_TWO_PASS;
+    const bool fused = is_fused(L.variant);
     cudaError_t e;
     if (h->use_tma) {
-        zk::TmaArgs ta{};
-        ta.b = a;
-        ta.runs = h->d_tma_runs;
-        ta.n_runs = (int)L.tma_runs.size();
-        ta.n_tiles = L.tma_tiles;
-        ta.n_scal = L.tma_scal;
-        ta.err = h->d_flag + 1;
-        ta.wait_rounds = zk::kTmaWaitRounds;
-        ta.hold_tile = -1;
-        const int64_t cap = (int64_t)h->sms * h->occ_tma;
-        const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
-        e = zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
+        if (!fused) a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
+        e = launch_tma_step(h, a, -1, zk::kTmaWaitRounds, s);
     } else if (fused) {
         e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
     } else {

@@ -143,6 +143,13 @@ struct TmaArgs {
     long long hold_tile;    // test hook: this tile is never armed (-1: none)
 };
 
+// ---- the two-pass step with TMA staging (ZERO_VARIANT_TWO_PASS_TMA) ----
+constexpr int kPassReduce = 0;  // Nd gradient slices in, the reduced gradient out
+constexpr int kPassUpdate = 1;  // reduced gradient, m, v, weight in; m, v, (master,) parameters out
+// the reduce pass has Nd input streams and one output: the deeper shape; the
+// update pass is store-heavy with many outputs: the shape of the fused step
+inline TmaShape tma_pass_shape(int mode, int n_out) { return mode == kPassReduce ? kTmaDeep : tma_shape(n_out); }
+
 // The stage-3 layer gather with bulk copies: each run (one rank's chunk of one
 // tensor) is copied shard -> output through shared memory in tiles of
 // kGatherTile elements, kGatherStages tiles in flight per CTA. TmaRun fields:
@@ -198,6 +205,12 @@ cudaError_t launch_commit(Ctrl* ctrl, unsigned* flag, const unsigned* err, cudaS
 cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);
 cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s);
 cudaError_t tma_gather_prepare(int* blocks_per_sm);
+// Two-pass step with TMA staging: attribute set-up and blocks per SM of the
+// two passes (bf16: the bfloat16 codec without master), launch of one pass.
+// Both use TmaArgs; the update pass returns at once if the overflow word holds
+// the call's id or the error word is set.
+cudaError_t tma_pass_prepare(int nd, int n_out, bool bf16, int* occ_reduce, int* occ_update);
+cudaError_t launch_pass_tma(int mode, const TmaArgs& a, int grid, cudaStream_t s, bool bf16);
 cudaError_t launch_gather_tma(const TmaGatherArgs& a, int grid, cudaStream_t s);
 int step_smem_bytes(int nd, int n_out);
 

@@ -51,12 +51,17 @@ struct Layout {
     std::vector<zk::SegDesc> gather_segs;
     std::vector<zk::TmaRun> tma_gather;  // TMA variant: bulk-copy gather runs of all units
     std::vector<Unit> units;
-    std::vector<zk::TmaRun> tma_runs;  // TMA variant, when every run is eligible
+    std::vector<zk::TmaRun> tma_runs;  // TMA variants, when every run is eligible
     bool tma_ok = false;
     zk::TmaShape tma_shape = zk::kTmaDeep;
     int64_t tma_tiles = 0, tma_scal = 0;
+    // two-pass TMA variant: the reduce pass's table (its own tile size)
+    std::vector<zk::TmaRun> tma_runs_r;
+    zk::TmaShape tma_shape_r = zk::kTmaDeep;
+    int64_t tma_tiles_r = 0, tma_scal_r = 0;
     int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
-            off_gather_segs = 0, off_tma_runs = -1, off_tma_gather = -1, off_reduced = -1, off_shard16 = -1,
+            off_gather_segs = 0, off_tma_runs = -1, off_tma_runs_r = -1, off_tma_gather = -1, off_reduced = -1,
+            off_shard16 = -1,
             total = 0;
     int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
     int64_t transient_elems = 0;

@@ -506,6 +506,32 @@ cudaError_t download_chunk(zero_offload_handle* h, int64_t k, int s, float inv)
     return e;
 }
 
+// Write the host state chunk by chunk with fill(piece, chunk begin, from, to)
+// on the pool, upload the fp16 of each chunk's master and broadcast it; the
+// caller's stream waits for the last broadcast, and so does the host.
+template <class F>
+cudaError_t fill_state(zero_offload_handle* h, cudaStream_t cs, F fill)
+{
+    cudaError_t e = cudaEventRecord(h->ev_start, cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->s_bc, h->ev_start, 0);
+    for (int64_t k = 0; k < h->O.n_chunks && e == cudaSuccess; ++k) {
+        const int s = (int)(k % S);
+        e = cudaEventSynchronize(h->ev_h2d[s]);  // host slot s free
+        if (e != cudaSuccess) break;
+        const int64_t c0 = h->chunk_begin(k);
+        uint16_t* p16 = h->h_p16(s);
+        for_chunk(h, k, [&](const OffRun& r, int64_t a, int64_t b) {
+            fill(r, c0, a, b);
+            h->cast(h->w + c0 + a, p16 + a, b - a);
+        });
+        e = upload_chunk(h, k, s);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_end, h->s_bc);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, h->ev_end, 0);
+    if (e == cudaSuccess) e = cudaEventSynchronize(h->ev_end);
+    return e;
+}
+
 }  // namespace
 
 ZERO_API int zero_offload_bytes(const zero_config* cfg, int64_t chunk_elems, zero_offload_ledger* out)
@@ -608,24 +634,12 @@ ZERO_API int zero_offload_init(const zero_config* cfg, int64_t chunk_elems, void
 
     // host state in state order (each thread first-touches the pages it will
     // update), fp16 parameters uploaded chunk by chunk
-    for (int64_t k = 0; k < O.n_chunks && e == cudaSuccess; ++k) {
-        const int s = (int)(k % S);
-        e = cudaEventSynchronize(h->ev_h2d[s]);  // host slot s free
-        if (e != cudaSuccess) break;
-        const int64_t c0 = h->chunk_begin(k);
-        uint16_t* p16 = h->h_p16(s);
-        for_chunk(h, k, [&](const OffRun& r, int64_t a, int64_t b) {
-            const float* src = master_init + r.grad_begin + (a - r.local_begin);
-            std::memcpy(h->w + c0 + a, src, (size_t)(b - a) * 4);
+    if (e == cudaSuccess)
+        e = fill_state(h, cs, [&](const OffRun& r, int64_t c0, int64_t a, int64_t b) {
+            std::memcpy(h->w + c0 + a, master_init + r.grad_begin + (a - r.local_begin), (size_t)(b - a) * 4);
             std::memset(h->m + c0 + a, 0, (size_t)(b - a) * 4);
             std::memset(h->v + c0 + a, 0, (size_t)(b - a) * 4);
-            h->cast(h->w + c0 + a, p16 + a, b - a);
         });
-        e = upload_chunk(h, k, s);
-    }
-    if (e == cudaSuccess) e = cudaEventRecord(h->ev_end, h->s_bc);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, h->ev_end, 0);
-    if (e == cudaSuccess) e = cudaEventSynchronize(h->ev_end);
     if (e != cudaSuccess) {
         rc = fail(h, e);
         release(h);
@@ -705,6 +719,23 @@ ZERO_API int zero_offload_step(zero_offload_handle* h, const uint16_t* const* gr
     e = cudaEventRecord(h->ev_end, h->s_bc);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, h->ev_end, 0);
     if (e != cudaSuccess) return fail(h, e);
+    return ZERO_OK;
+}
+
+ZERO_API int zero_offload_set_state(zero_offload_handle* h, const float* master, const float* m, const float* v,
+                                    int64_t t, void* stream)
+{
+    if (!h || h->broken || t < 0) return ZERO_ERR_ARG;
+    if (h->O.E > 0 && (!master || !m || !v)) return ZERO_ERR_ARG;
+    const cudaError_t e =
+        fill_state(h, static_cast<cudaStream_t>(stream), [&](const OffRun&, int64_t c0, int64_t a, int64_t b) {
+            const size_t bytes = (size_t)(b - a) * 4;
+            if (h->w + c0 + a != master + c0 + a) std::memcpy(h->w + c0 + a, master + c0 + a, bytes);
+            if (h->m + c0 + a != m + c0 + a) std::memcpy(h->m + c0 + a, m + c0 + a, bytes);
+            if (h->v + c0 + a != v + c0 + a) std::memcpy(h->v + c0 + a, v + c0 + a, bytes);
+        });
+    if (e != cudaSuccess) return fail(h, e);
+    h->t = t;
     return ZERO_OK;
 }
 
