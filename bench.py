@@ -317,8 +317,9 @@ def run_reference(args):
     wl = workload(args.workload)
     budget = 150.0  # seconds of CPU for warm-up + timed steps
     per_step = budget / max(1, args.steps + args.warmup)
-    n_s = calibrate_sample(wl, per_step)
-    state = {}
+    bf16 = args.precision == "bf16"
+    n_s = calibrate_sample(wl, per_step, bf16)
+    state = {"bf16": bf16}
     for i in range(args.warmup):
         oracle_sample_step(wl, n_s, i, state)
     times = [oracle_sample_step(wl, n_s, args.warmup + i, state) for i in range(args.steps)]
@@ -326,7 +327,7 @@ def run_reference(args):
     value = n_s * args.steps / total / 1e9
     model, ncpu = cpu_info()
     sample = (f"first {n_s} elements of the workload per step, Nd={wl.nd}, stage {wl.stage}, "
-              f"single thread")
+              f"{'bfloat16 without master, ' if bf16 else ''}single thread")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

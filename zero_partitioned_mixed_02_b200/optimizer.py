@@ -7,6 +7,9 @@ supplies the stream; libzero does all the work.
     w, m, v = opt.state()                # live fp32 state (views of the workspace)
     sd = opt.state_dict(); opt.load_state_dict(sd)     # checkpoint / resume
     opt.begin_async(grads, scaler); opt.step_async(...); opt.end_async()
+
+    off = ZeroOffloadAdam(psi, nd, stage, master_init_host, param_bufs)   # host fp32 state
+    skipped = off.step(grads, loss_scale, lr=...)
 """
 from __future__ import annotations
 
@@ -21,9 +24,13 @@ class ZeroAdam:
     def __init__(self, psi: int, nd: int, stage: int, master_init: torch.Tensor,
                  param_bufs: Sequence[torch.Tensor] | None = None, *, rank_view: int = -1,
                  variant: int = A.ZERO_VARIANT_FUSED_TMA,
-                 tensors: Sequence[tuple[int, int]] | None = None,
-                 stream: torch.cuda.Stream | None = None):
-        self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors)
+                 tensors: Sequence[tuple[int, ...]] | None = None,
+                 stream: torch.cuda.Stream | None = None,
+                 precision: int = A.ZERO_PRECISION_FP16):
+        """precision = ZERO_PRECISION_BF16: bfloat16 gradients and parameters
+        without fp32 master weights (variant must be a two-pass one)."""
+        self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors,
+                            precision=precision)
         self.ledger = A.zero_state_bytes(self.cfg)
         dev = master_init.device
         if dev.type != "cuda":
@@ -60,7 +67,9 @@ class ZeroAdam:
     def t(self) -> int:
         return A.zero_current_state(self.h)[3]
 
-    def _view_f32(self, ptr: int) -> torch.Tensor:
+    def _view_f32(self, ptr: int | None) -> torch.Tensor | None:
+        if ptr is None:
+            return None  # no master (bfloat16 without master weights)
         off = ptr - self.workspace.data_ptr()
         n = self.ledger.state_elems
         return self.workspace[off: off + 4 * n].view(torch.float32)
@@ -78,17 +87,18 @@ class ZeroAdam:
         return self.workspace[off: off + 2 * n].view(torch.int16)
 
     def state_dict(self) -> dict:
-        """Copies of master, m, v (state order) and the step count."""
+        """Copies of master (None without one), m, v (state order) and the step count."""
         w, m, v = self.state()
-        return {"master": w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
+        return {"master": None if w is None else w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
 
     def load_state_dict(self, sd: dict) -> None:
-        tensors = [sd["master"], sd["m"], sd["v"]]
+        tensors = [x for x in (sd["master"], sd["m"], sd["v"]) if x is not None]
         for x in tensors:
             if x.dtype != torch.float32 or not x.is_cuda or x.numel() != self.ledger.state_elems:
                 raise ValueError("state tensors must be CUDA float32 of ledger.state_elems elements")
-        w, m, v = (x.contiguous() for x in tensors)
-        A.zero_set_state(self.h, w.data_ptr(), m.data_ptr(), v.data_ptr(), int(sd["t"]),
+        w = None if sd["master"] is None else sd["master"].contiguous()
+        m, v = sd["m"].contiguous(), sd["v"].contiguous()
+        A.zero_set_state(self.h, 0 if w is None else w.data_ptr(), m.data_ptr(), v.data_ptr(), int(sd["t"]),
                          self.stream.cuda_stream)
 
     def begin_async(self, grads: Sequence[torch.Tensor], init_scale: float = 65536.0,
@@ -113,6 +123,79 @@ class ZeroAdam:
     def close(self) -> None:
         if self.h:
             A.zero_destroy(self.h)
+            self.h = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class ZeroOffloadAdam:
+    """The offloaded step (include/zero_offload.h): fp32 master, m, v in host
+    memory and Adam on the host cores; the reduce and the fp16 write-back run
+    on the GPU. PyTorch allocates the device workspace, the page-locked
+    staging and the host state; libzero does the work."""
+
+    def __init__(self, psi: int, nd: int, stage: int, master_init, param_bufs: Sequence[torch.Tensor], *,
+                 rank_view: int = -1, tensors: Sequence[tuple[int, ...]] | None = None,
+                 chunk_elems: int = 0, threads: int = 0, stream: torch.cuda.Stream | None = None):
+        import os
+
+        import numpy as np
+
+        self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, tensors=tensors)
+        self.ledger = A.zero_offload_bytes(self.cfg, chunk_elems)
+        self.nd = nd
+        m0 = np.ascontiguousarray(master_init.cpu().numpy() if isinstance(master_init, torch.Tensor)
+                                  else master_init, dtype=np.float32)
+        self.stream = stream or torch.cuda.current_stream()
+        E = self.ledger.state_elems
+        self.device_ws = torch.empty(self.ledger.device_bytes, dtype=torch.uint8, device=self.stream.device)
+        self.staging = torch.empty(self.ledger.host_staging_bytes, dtype=torch.uint8, pin_memory=True)
+        self.host_state = torch.empty(3 * max(E, 1), dtype=torch.float32)
+        self.param_bufs = list(param_bufs)
+        threads = threads or len(os.sched_getaffinity(0))
+        self.h = A.zero_offload_init(self.cfg, chunk_elems, self.device_ws.data_ptr(), self.ledger.device_bytes,
+                                     self.staging.data_ptr(), self.ledger.host_staging_bytes,
+                                     self.host_state.data_ptr(), m0.ctypes.data,
+                                     [p.data_ptr() for p in self.param_bufs], min(threads, 256),
+                                     self.stream.cuda_stream)
+
+    def step(self, grads: Sequence[torch.Tensor] | Sequence[int], loss_scale: float, *, lr=1e-3,
+             betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0) -> bool:
+        ptrs = [g if isinstance(g, int) else g.data_ptr() for g in grads]
+        if len(ptrs) != self.nd:
+            raise ValueError(f"expected {self.nd} gradient buffers, got {len(ptrs)}")
+        hp = A.zero_hyper(lr, betas[0], betas[1], eps, weight_decay)
+        return A.zero_offload_step(self.h, ptrs, loss_scale, hp, self.stream.cuda_stream) == A.ZERO_SKIPPED
+
+    @property
+    def t(self) -> int:
+        return A.zero_offload_state(self.h)[3]
+
+    def state(self) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """Live host master, m, v (state order; views of the host state)."""
+        E = self.ledger.state_elems
+        return self.host_state[:E], self.host_state[E:2 * E], self.host_state[2 * E:3 * E]
+
+    def state_dict(self) -> dict:
+        w, m, v = self.state()
+        return {"master": w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
+
+    def load_state_dict(self, sd: dict) -> None:
+        E = self.ledger.state_elems
+        xs = [sd["master"].contiguous(), sd["m"].contiguous(), sd["v"].contiguous()]
+        for x in xs:
+            if x.dtype != torch.float32 or x.is_cuda or x.numel() != E:
+                raise ValueError("state tensors must be host float32 of ledger.state_elems elements")
+        A.zero_offload_set_state(self.h, xs[0].data_ptr(), xs[1].data_ptr(), xs[2].data_ptr(), int(sd["t"]),
+                                 self.stream.cuda_stream)
+
+    def close(self) -> None:
+        if self.h:
+            A.zero_offload_destroy(self.h)
             self.h = 0
 
     def __del__(self):
