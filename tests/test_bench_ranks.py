@@ -58,3 +58,24 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
         workload, steps, warmup, gpus, variant = "flat-1m", 1, 0, 2, "fused-tma"
     bench.run_reference(A)
     assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_bytes_per_element():
+    """The roofline's numerator: bytes per updated element of each workload,
+    variant and precision, from the step's definition (SURVEY's per-unit
+    figures: (24 + 4 Nd) for stage 1/2, (26 + 2 Nd) for stage 3, 154 per
+    element of the Nd = 64 rank view)."""
+    from zero_partitioned_mixed_02_b200.synth import workloads as W
+    g = W.gpt2_1p5b()
+    n, floor, per, gathers = bench.algorithmic_bytes(g, "fused-tma")
+    assert n == g.psi and floor == 56 * g.psi and gathers == 0
+    n, floor, per, _ = bench.algorithmic_bytes(g, "two-pass-tma")
+    assert floor == 56 * g.psi and sum(per.values()) == 64 * g.psi  # + 8 B of reduced gradient
+    n, floor, per, _ = bench.algorithmic_bytes(g, "two-pass-tma", bf16=True)
+    assert floor == 50 * g.psi and sum(per.values()) == 58 * g.psi
+    ll = W.llama_2p7b()
+    n, floor, _, gathers = bench.algorithmic_bytes(ll, "fused-tma")
+    assert floor == 42 * ll.psi and gathers == 8 * ll.psi
+    rv = W.running_example_7p5b()
+    n, floor, _, _ = bench.algorithmic_bytes(rv, "fused")
+    assert n == 117_187_500 and floor == 154 * n
