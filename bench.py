@@ -605,10 +605,17 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
         result = ws[L.off_shard16: L.off_shard16 + 2 * L.state_elems].view(torch.int16)
     need = (len(grads) * n_own + result.numel()) * 2
     avail = psutil.virtual_memory().available
-    if need > 0.7 * avail:
+    # every rank on this node pins its own copies at the same time
+    local_ranks = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    ok = need * local_ranks <= 0.6 * avail
+    if world > 1:  # every rank takes the same decision (the steps below hold collectives)
+        flag = torch.tensor([1 if ok else 0], device="cuda")
+        dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+        ok = bool(flag.item())
+    if not ok:
         return {"value": None, "unit": UNIT,
-                "unavailable": f"needs {need / 1e9:.1f} GB pinned host memory, "
-                               f"{avail / 1e9:.1f} GB available"}
+                "unavailable": f"needs {need / 1e9:.1f} GB pinned host memory per rank x {local_ranks} "
+                               f"ranks, {avail / 1e9:.1f} GB available"}
     s = torch.cuda.current_stream()
     side = torch.cuda.Stream()  # device->host reads of the result
     host_g = [torch.empty(n_own, dtype=torch.int16, pin_memory=True) for _ in grads]

@@ -594,3 +594,16 @@ def test_no_decay_async_steps(variant):
     assert (st.t, st.skipped) == (c.t, 1)
     c.check("after the asynchronous run")
     c.close()
+
+
+@pytest.mark.parametrize("variant", [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS])
+@pytest.mark.parametrize("stage", [1, 3])
+def test_maximum_nd(stage, variant):
+    """Nd = ZERO_MAX_ND (1024 gradient pointers and, for stage 1/2, 1024
+    replica pointers in the kernels' shared-memory tables; most partitions and
+    chunks a handful of elements long, the last ones empty)."""
+    nd = A.ZERO_MAX_ND
+    psi = 5 * nd + 37
+    tensors = [(3 * nd + 5, 0), (2 * nd + 32, 1)] if stage == 3 else None
+    c = Case(psi, nd, stage, variant, tensors=tensors, hp=dict(lr=1e-2, weight_decay=0.01))
+    assert _run(c, 2, inject=[(1, nd - 1, 0, 0x7C00)]) == [False, True]
