@@ -143,6 +143,12 @@ typedef struct zero_config {
     int32_t precision; /* ZERO_PRECISION_FP16 (0) or ZERO_PRECISION_BF16 */
     const zero_tensor* tensors; /* host array of n_tensors; sum of numel == psi;
                                    required for stage 3 */
+    int32_t view_outputs; /* single-rank view only (else 0): parameter buffers
+                             written, 0 or 1 = one buffer, nd = every rank's
+                             replica (rank r of a real Nd-rank job: param_bufs
+                             are all ranks' replicas, e.g. peer-mapped; see
+                             zero_flag_words) */
+    int32_t reserved;     /* must be 0 */
 } zero_config;
 
 typedef struct zero_hyper {
@@ -243,6 +249,24 @@ int zero_step(zero_handle* h, const uint16_t* const* grads, float loss_scale,
 int zero_step_launch(zero_handle* h, const uint16_t* const* grads, float loss_scale,
                      const zero_hyper* hp, void* stream);
 int zero_step_commit(zero_handle* h, void* stream, int* skipped);
+
+/* The handle's overflow word and kernel-error word: two consecutive uint32 in
+ * the workspace (device memory). A step of ZeRO stage 1/2 is skipped if ANY
+ * rank's reduced gradient overflows ([P1] "The part that sounds too good:
+ * communication": the ranks reduce-scatter, update their slices, all-gather;
+ * one overflow decision for the step). When each rank of a real Nd-rank job
+ * runs its own single-rank-view handle (view_outputs = nd), the ranks agree by
+ * reducing these two words with MAX across ranks on `stream` between
+ * zero_step_launch and zero_step_commit (for instance ncclAllReduce with
+ * ncclMax on ncclUint32, count 2); the words hold the handle's step call id on
+ * overflow, which advances identically on every rank. With a two-pass variant
+ * such a handle's zero_step_launch enqueues only the reduce pass and its
+ * zero_step_commit enqueues the in-place update pass after the agreement (the
+ * pass returns at once if the agreed words say overflow); the fused variants
+ * write speculatively and roll back on an agreed overflow. Such handles take
+ * no asynchronous steps (zero_async_begin: ZERO_ERR_ARG). Host only (returns
+ * the address). ZERO_OK or ZERO_ERR_ARG. */
+int zero_flag_words(zero_handle* h, uint32_t** words);
 
 /* ---- asynchronous steps ([P1]-[P3] do not cover loss scaling; the usual
  * dynamic loss scaling is the reading) ----

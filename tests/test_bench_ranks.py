@@ -79,3 +79,34 @@ def test_algorithmic_bytes_per_element():
     rv = W.running_example_7p5b()
     n, floor, _, _ = bench.algorithmic_bytes(rv, "fused")
     assert n == 117_187_500 and floor == 154 * n
+
+
+def _agree_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    from zero_partitioned_mixed_02_b200.distributed import agree_overflow
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # step 7: only rank 1 overflowed (its word holds the call id); rank 0 had
+    # an old overflow at step 3; nobody's kernel gave up
+    words = torch.tensor([3, 0] if rank == 0 else [7, 0], dtype=torch.int32)
+    agree_overflow(words)
+    q.put((rank, words.tolist()))
+    dist.destroy_process_group()
+
+
+def test_overflow_agreement_gloo():
+    """Host side of the multi-rank step: MAX of the flag words makes every
+    rank see the current step's overflow (call id 7), whoever raised it."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_agree_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    got = dict(q.get() for _ in range(2))
+    assert got == {0: [7, 0], 1: [7, 0]}

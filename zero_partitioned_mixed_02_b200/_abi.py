@@ -50,7 +50,8 @@ class zero_tensor(C.Structure):
 class zero_config(C.Structure):
     _fields_ = [("psi", C.c_int64), ("nd", C.c_int32), ("stage", C.c_int32),
                 ("rank_view", C.c_int32), ("variant", C.c_int32), ("n_tensors", C.c_int32),
-                ("precision", C.c_int32), ("tensors", C.POINTER(zero_tensor))]
+                ("precision", C.c_int32), ("tensors", C.POINTER(zero_tensor)),
+                ("view_outputs", C.c_int32), ("reserved", C.c_int32)]
 
 
 class zero_hyper(C.Structure):
@@ -129,6 +130,7 @@ def lib():
                                            C.POINTER(C.c_int64), P, C.POINTER(C.c_int)]),
             "zero_last_cuda_error": (C.c_int, [P]),
             "zero_uses_tma": (C.c_int, [P]),
+            "zero_flag_words": (C.c_int, [P, C.POINTER(P)]),
             "zero_test_hold_tile": (C.c_int, [P, C.c_int64, C.c_uint32]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
@@ -163,7 +165,7 @@ class Config:
     def __init__(self, psi: int, nd: int, stage: int, rank_view: int = -1,
                  variant: int = ZERO_VARIANT_FUSED,
                  tensors: Sequence[tuple[int, ...]] | None = None,
-                 precision: int = ZERO_PRECISION_FP16):
+                 precision: int = ZERO_PRECISION_FP16, view_outputs: int = 0):
         """tensors: (numel, unit) or (numel, unit, flags) per tensor, flat order;
         flags = ZERO_TENSOR_NO_DECAY excludes the tensor from weight decay."""
         self._tensors = None
@@ -175,7 +177,7 @@ class Config:
                 zero_tensor(int(t[0]), int(t[1]), int(t[2]) if len(t) > 2 else 0) for t in tensors])
             ptr = C.cast(self._tensors, C.POINTER(zero_tensor))
         self.c = zero_config(int(psi), int(nd), int(stage), int(rank_view), int(variant), n,
-                             int(precision), ptr)
+                             int(precision), ptr, int(view_outputs), 0)
 
     def byref(self):
         return C.byref(self.c)
@@ -295,6 +297,13 @@ def zero_step_static(psi: int, grads: Sequence[int], master: int, m: int, v: int
 
 def zero_test_hold_tile(h: int, tile: int, wait_rounds: int) -> None:
     _check(lib().zero_test_hold_tile(h, tile, wait_rounds), "zero_test_hold_tile")
+
+
+def zero_flag_words(h: int) -> int:
+    """Device address of the handle's overflow and kernel-error words (two uint32)."""
+    p = C.c_void_p()
+    _check(lib().zero_flag_words(h, C.byref(p)), "zero_flag_words")
+    return p.value
 
 
 def zero_uses_tma(h: int) -> bool:

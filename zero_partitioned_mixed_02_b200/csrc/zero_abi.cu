@@ -73,6 +73,10 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
     if (cfg->precision == ZERO_PRECISION_BF16 && is_fused(cfg->variant)) return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
     if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
+    if (cfg->reserved != 0) return ZERO_ERR_ARG;
+    if (cfg->rank_view < 0 ? cfg->view_outputs != 0
+                           : (cfg->view_outputs != 0 && cfg->view_outputs != 1 && cfg->view_outputs != cfg->nd))
+        return ZERO_ERR_ARG;
     if (cfg->stage == 3 && cfg->n_tensors == 0) return ZERO_ERR_ARG;
     if (cfg->n_tensors > 0 && !cfg->tensors) return ZERO_ERR_ARG;
 
@@ -152,7 +156,7 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             add_partition(b, e, b);
             L->state_elems = e - b;
             L->grad_len = e - b;
-            L->n_out = 1;
+            L->n_out = cfg->view_outputs == nd ? nd : 1;
         }
     } else {
         // stage 3: every tensor split per rank; rank r's shard is its chunks
@@ -438,8 +442,17 @@ int cuda_fail(zero_handle* h, cudaError_t e);
 // The TMA-staged step with arguments a: the fused kernel, or the reduce and
 // update passes (a.red set by the caller). hold_tile / wait_rounds: the test
 // hook, applied to the first launch only.
+// passes of a two-pass step to enqueue (the fused step is one pass)
+constexpr int kRunReduce = 1, kRunUpdate = 2, kRunBoth = 3;
 cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_tile, unsigned wait_rounds,
-                            cudaStream_t s);
+                            cudaStream_t s, int passes = kRunBoth);
+
+// A single-rank-view handle that writes every rank's replica is rank r of a
+// real job: the ranks agree on overflow between zero_step_launch and
+// zero_step_commit. A two-pass step updates in place, so its update pass must
+// wait for that agreement: zero_step_launch enqueues the reduce pass only and
+// zero_step_commit the update pass.
+bool defers_update(const Layout& L) { return L.view >= 0 && L.n_out > 1 && !is_fused(L.variant); }
 
 int cuda_fail(zero_handle* h, cudaError_t e)
 {
@@ -480,7 +493,7 @@ void bias_corrections(zero_handle* h, float b1, float b2, int64_t t, float* bc1,
 namespace {
 
 cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_tile, unsigned wait_rounds,
-                            cudaStream_t s)
+                            cudaStream_t s, int passes)
 {
     const Layout& L = h->L;
     zk::TmaArgs ta{};
@@ -497,22 +510,25 @@ cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_
         const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
         return zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
     }
-    ta.runs = h->d_tma_runs_r;
-    ta.n_runs = (int)L.tma_runs_r.size();
-    ta.n_tiles = L.tma_tiles_r;
-    ta.n_scal = L.tma_scal_r;
-    int64_t cap = (int64_t)h->sms * h->occ_tma_r;
-    int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles_r, (L.tma_scal_r + 255) / 256));
-    cudaError_t e = zk::launch_pass_tma(zk::kPassReduce, ta, (int)std::min(want, cap), s, L.bf16);
-    if (e != cudaSuccess) return e;
+    if (passes & kRunReduce) {
+        ta.runs = h->d_tma_runs_r;
+        ta.n_runs = (int)L.tma_runs_r.size();
+        ta.n_tiles = L.tma_tiles_r;
+        ta.n_scal = L.tma_scal_r;
+        const int64_t cap = (int64_t)h->sms * h->occ_tma_r;
+        const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles_r, (L.tma_scal_r + 255) / 256));
+        const cudaError_t e = zk::launch_pass_tma(zk::kPassReduce, ta, (int)std::min(want, cap), s, L.bf16);
+        if (e != cudaSuccess) return e;
+    }
+    if (!(passes & kRunUpdate)) return cudaSuccess;
     ta.runs = h->d_tma_runs;
     ta.n_runs = (int)L.tma_runs.size();
     ta.n_tiles = L.tma_tiles;
     ta.n_scal = L.tma_scal;
     ta.hold_tile = -1;
     ta.wait_rounds = zk::kTmaWaitRounds;
-    cap = (int64_t)h->sms * h->occ_tma;
-    want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
+    const int64_t cap = (int64_t)h->sms * h->occ_tma;
+    const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
     return zk::launch_pass_tma(zk::kPassUpdate, ta, (int)std::min(want, cap), s, L.bf16);
 }
 
@@ -734,16 +750,18 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.m_out = h->state(nxt, 1);
     a.v_out = h->state(nxt, 2);
     if (L.step_chunks > 0) {
+        const int passes = defers_update(L) ? kRunReduce : kRunBoth;
         if (h->use_tma) {
             if (!fused) a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
-            e = launch_tma_step(h, a, h->hold_tile, h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds, s);
+            e = launch_tma_step(h, a, h->hold_tile, h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds, s,
+                                passes);
             h->hold_tile = -1;
         } else if (fused) {
             e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
         } else {
             a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
             e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s, L.bf16);
-            if (e == cudaSuccess)
+            if (e == cudaSuccess && (passes & kRunUpdate))
                 e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s, L.bf16);
         }
         if (e != cudaSuccess) return cuda_fail(h, e);
@@ -761,9 +779,18 @@ ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
     h->pending = false;
     const Layout& L = h->L;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (defers_update(L) && L.step_chunks > 0) {
+        // the update pass, after the ranks' agreement on the flag words (it
+        // returns at once if the agreed words say overflow or a failed wait)
+        if (h->use_tma)
+            e = launch_tma_step(h, h->args, -1, zk::kTmaWaitRounds, s, kRunUpdate);
+        else
+            e = zk::launch_step(zk::K_UPDATE, h->args, grid_for(h, zk::K_UPDATE, L.step_chunks), s, L.bf16);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+    }
     // a copy into pageable host memory returns once the stream has reached it
-    cudaError_t e = cudaMemcpyAsync(h->host_flag, h->d_flag, 2 * sizeof(unsigned),
-                                    cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(h->host_flag, h->d_flag, 2 * sizeof(unsigned), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(h, e);
     const bool kernel_error = h->host_flag[1] != 0;
@@ -805,6 +832,8 @@ ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, cons
                               float beta1, float beta2, void* stream)
 {
     if (!h || !grads || !sc || h->pending || h->async) return ZERO_ERR_ARG;
+    // a rank of a real job agrees with the other ranks through launch/commit
+    if (h->L.view >= 0 && h->L.n_out > 1) return ZERO_ERR_ARG;
     if (!(sc->init_scale > 0.0f) || !std::isfinite(sc->init_scale) || !(sc->growth_factor >= 1.0f) ||
         !std::isfinite(sc->growth_factor) || !(sc->backoff_factor > 0.0f) || !(sc->backoff_factor <= 1.0f) ||
         sc->growth_interval < 1 || !std::isfinite(beta1) || !std::isfinite(beta2))
@@ -1034,6 +1063,13 @@ ZERO_API int zero_test_hold_tile(zero_handle* h, int64_t tile, uint32_t wait_rou
     if (!h || tile < 0 || wait_rounds == 0) return ZERO_ERR_ARG;
     h->hold_tile = tile;
     h->hold_rounds = wait_rounds;
+    return ZERO_OK;
+}
+
+ZERO_API int zero_flag_words(zero_handle* h, uint32_t** words)
+{
+    if (!h || !words) return ZERO_ERR_ARG;
+    *words = h->d_flag;
     return ZERO_OK;
 }
 
