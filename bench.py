@@ -576,18 +576,26 @@ def prefetch_demo(h, L, order, gather_out, reps=5):
     torch.cuda.reset_peak_memory_stats()
     base = torch.cuda.memory_allocated()
     pf = LayerPrefetcher(h, L, s)
+    pf_hi = LayerPrefetcher(h, L, s, priority=-1)  # side stream at high priority
 
     def prefetched():
         for _, w in pf.walk(order):
             consume(w)
 
+    def prefetched_hi():
+        for _, w in pf_hi.walk(order):
+            consume(w)
+
     out = {"units": len(order), "tokens": tokens, "d": d,
            "gathers_only_ms": timed(gathers_only), "gemms_only_ms": timed(gemms_only),
            "sequential_ms": timed(sequential), "prefetched_ms": timed(prefetched),
+           "prefetched_high_priority_ms": timed(prefetched_hi),
            "transient_bytes": L.transient_bytes, "prefetch_transient_bytes": pf.peak_bytes}
     out["measured_peak_extra_bytes"] = torch.cuda.max_memory_allocated() - base
     hidden = out["sequential_ms"] - out["prefetched_ms"]
     out["gather_time_hidden_frac"] = hidden / out["gathers_only_ms"]
+    out["gather_time_hidden_frac_high_priority"] = (
+        out["sequential_ms"] - out["prefetched_high_priority_ms"]) / out["gathers_only_ms"]
     return out
 
 

@@ -266,6 +266,7 @@ cudaError_t prepare_mode(TmaShape sh, int nd, int* blocks_per_sm)
 template <int MODE, class C>
 cudaError_t launch_mode(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s)
 {
+    // only the two instantiated shapes
     const void* f = a.b.ctrl ? pass_kernel<MODE, true, C>(sh) : pass_kernel<MODE, false, C>(sh);
     if (!f) return cudaErrorInvalidValue;
     const int smem = pass_smem<MODE, C>(sh, a.b.nd);

@@ -25,12 +25,15 @@ from . import _abi as A
 
 class LayerPrefetcher:
     def __init__(self, handle: int, ledger, stream: torch.cuda.Stream | None = None,
-                 device: torch.device | str = "cuda"):
+                 device: torch.device | str = "cuda", priority: int = 0):
+        """priority: of the side stream (lower is higher, see
+        torch.cuda.Stream); a high priority lets the gather's CTAs take SMs as
+        the caller's kernel frees them."""
         if ledger.n_units <= 0:
             raise ValueError("layer gathers need a stage-3 handle")
         self.h = handle
         self.stream = stream or torch.cuda.current_stream(device)
-        self.side = torch.cuda.Stream(device=self.stream.device)
+        self.side = torch.cuda.Stream(device=self.stream.device, priority=priority)
         n = max(ledger.transient_bytes // 2, 1)
         self.buffers = [torch.empty(n, dtype=torch.int16, device=self.stream.device) for _ in range(2)]
         self.peak_bytes = 2 * ledger.transient_bytes
