@@ -261,3 +261,32 @@ def test_bf16_set_state():
     c.step(c.grads(5))
     c.check("after a step from the restored state")
     c.close()
+
+
+def test_bf16_async_step_in_a_cuda_graph():
+    """The bfloat16 step without master, asynchronous and captured once in a
+    CUDA graph, replayed with fresh gradients (one overflowing)."""
+    c = Bf16Case(40_000, 4, 2, tensors=[(24_000, 0), (16_000, 0, NO_DECAY)], variant=TWO_TMA)
+    c.check("after init")
+    cap = torch.cuda.Stream()
+    with torch.cuda.stream(cap):
+        A.zero_async_begin(c.h, [g.data_ptr() for g in c.g_dev], A.zero_scaler(8.0, 2.0, 0.5, 2), 0.9, 0.999,
+                           cap.cuda_stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            A.zero_step_async(c.h, hyper(**c.hp), cap.cuda_stream)
+        scale, good = 8.0, 0
+        for s in range(5):
+            gs = c.grads(s)
+            if s == 2:
+                gs[0][39_999] = 0x7F80
+            c.upload(gs)
+            graph.replay()
+            sk = c.oracle_step(gs, scale)
+            scale, good = Z.scaler_update(scale, good, sk, 2.0, 0.5, 2)
+        st = A.zero_async_end(c.h, cap.cuda_stream)
+    torch.cuda.synchronize()
+    assert (st.t, st.skipped) == (c.t, 1) and st.loss_scale == np.float32(scale)
+    c.check("after graph replays")
+    del graph
+    c.close()

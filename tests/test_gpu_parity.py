@@ -607,3 +607,15 @@ def test_maximum_nd(stage, variant):
     tensors = [(3 * nd + 5, 0), (2 * nd + 32, 1)] if stage == 3 else None
     c = Case(psi, nd, stage, variant, tensors=tensors, hp=dict(lr=1e-2, weight_decay=0.01))
     assert _run(c, 2, inject=[(1, nd - 1, 0, 0x7C00)]) == [False, True]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("hp", [dict(lr=1e-2, beta1=0.0, beta2=0.0, weight_decay=0.0),
+                                dict(lr=1e-3, beta1=0.999999, beta2=0.5, weight_decay=0.0),
+                                dict(lr=0.0, weight_decay=0.1),
+                                dict(lr=1e-1, weight_decay=0.5, eps=1e-3)])
+def test_hyperparameter_corners(variant, hp):
+    """beta = 0 (bias corrections 1), beta close to 1 (tiny bias correction),
+    lr = 0 (master unchanged, moments move), large decoupled weight decay."""
+    _run(Case(70_001, 4, 2, variant, hp=hp), 3)
+    _run(Case(8 * 4 * 999, 4, 3, variant, tensors=[(8 * 4 * 500, 0), (8 * 4 * 499, 1)], hp=hp), 2)
