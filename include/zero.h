@@ -79,7 +79,7 @@ extern "C" {
  * Accelerator: tiles of the Nd gradient slices and of master/m/v are staged
  * into shared memory by bulk asynchronous copies while earlier tiles are
  * computed, and results leave by bulk stores. Same arithmetic, bytes and
- * workspace as ZERO_VARIANT_FUSED. Used when Nd <= 8 and every run's state
+ * workspace as ZERO_VARIANT_FUSED. Used when Nd <= 16 and every run's state
  * and output indices are in 16-byte phase with its gradient index; otherwise
  * the handle runs the ZERO_VARIANT_FUSED kernel. Its stage-3 layer gathers
  * copy through shared memory with bulk copies too (for units whose chunks are

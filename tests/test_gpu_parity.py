@@ -306,7 +306,7 @@ def test_workload_precision_stress(variant):
 
 
 @pytest.mark.parametrize("variant", TMA_VARIANTS)
-@pytest.mark.parametrize("nd", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("nd", [1, 2, 3, 4, 8, 12, 16])
 def test_tma_path_runs_and_matches(nd, variant):
     # sizes with whole tiles, partial tiles, and heads/tails around them; every
     # partition in 16-byte phase, so the TMA kernels are the ones that run
@@ -314,13 +314,13 @@ def test_tma_path_runs_and_matches(nd, variant):
         c = Case(psi, nd, 2, variant, hp=dict(weight_decay=0.01))
         assert c.uses_tma()
         assert _run(c, 2) == [False, False]
-    c = Case(4099, 9, 2, variant)  # Nd > 8: the plain kernels
+    c = Case(4099, 17, 2, variant)  # Nd > 16: the plain kernels
     assert not c.uses_tma()
     _run(c, 1)
 
 
 @pytest.mark.parametrize("variant", TMA_VARIANTS)
-@pytest.mark.parametrize("nd", [2, 4, 8])
+@pytest.mark.parametrize("nd", [2, 4, 8, 16])
 def test_tma_stage3_eligible_tensors(nd, variant):
     # tensor sizes that keep every chunk in 16-byte phase: multiples of 8 * nd
     rng = np.random.default_rng(nd)

@@ -130,7 +130,7 @@ struct TmaShape {
 constexpr TmaShape kTmaWide{31, 1, 31 * 32 * 4};
 constexpr TmaShape kTmaDeep{20, 2, 20 * 32 * 4};
 inline TmaShape tma_shape(int n_out) { return n_out >= 4 ? kTmaWide : kTmaDeep; }
-constexpr int kTmaMaxNd = 8;  // ranks whose tiles fit the stages
+constexpr int kTmaMaxNd = 16;  // ranks whose tiles fit the stages (deep shape at 16: 226,304 B)
 
 struct TmaArgs {
     StepArgs b;             // pointers, tables, constants, flag (segs unused)
