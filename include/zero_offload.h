@@ -36,10 +36,9 @@
  *     state_elems elements (ordinary host memory; 12 bytes per element);
  *   - host staging: page-locked memory (cudaHostAlloc or a pinned torch
  *     tensor) for the chunks in flight (host_staging_bytes).
- * The stage-3 layer gathers of zero.h have no counterpart here: the fp16
- * shards live in the device workspace of a zero.h handle only. Stage 3 here
- * keeps its fp16 shards in the caller's buffer param_bufs[0] (state order,
- * state_elems elements).
+ * Stage 3 keeps its fp16 shards in the caller's buffer param_bufs[0] (state
+ * order, state_elems elements); zero_offload_gather_layer rebuilds a layer
+ * unit from them as zero_gather_layer does.
  *
  * The library creates four CUDA streams and some events per handle (no device
  * memory); zero_offload_destroy releases them. Conventions of zero.h apply
@@ -112,6 +111,13 @@ int zero_offload_init(const zero_config* cfg, int64_t chunk_elems, void* device_
  * steps: the host state may be partly updated). */
 int zero_offload_step(zero_offload_handle* h, const uint16_t* const* grads, float loss_scale,
                       const zero_hyper* hp, void* stream);
+
+/* Stage 3: write layer unit `unit`'s full fp16 weights into `out` (device),
+ * exactly as zero_gather_layer (zero.h): the unit's tensors in tensor order,
+ * each rebuilt from the Nd ranks' chunks in the shard buffer. Ordered on
+ * `stream` (after a step when the step's work on that stream is). ZERO_OK,
+ * ZERO_ERR_STAGE (stage 1/2), ZERO_ERR_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA. */
+int zero_offload_gather_layer(zero_offload_handle* h, int32_t unit, uint16_t* out, void* stream);
 
 /* Checkpoint / resume: replace the host state with master, m, v (HOST
  * arrays of state_elems floats in state order, e.g. saved from

@@ -110,6 +110,12 @@ class OffloadCase:
             compare_f16(got[self.b0:self.e0], self.p16, f"partition {tag}")
         else:
             compare_f16(self.bufs[0].bits(), self.p16[self.perm], f"shards {tag}")
+            for u in range(A.zero_state_bytes(self.cfg).n_units):
+                fb, cnt = A.zero_unit_range(self.cfg, u)
+                out = GuardedF16(cnt)
+                A.zero_offload_gather_layer(self.h, u, out.ptr(), self.stream)
+                compare_f16(out.bits(), self.p16[fb:fb + cnt], f"gathered unit {u} {tag}")
+                assert out.guards_intact()
         for b in self.bufs:
             assert b.guards_intact()
 
@@ -232,3 +238,11 @@ def test_offload_checkpoint_resume():
     assert (b.state[:3 * E].view(np.uint32) == a.state[:3 * E].view(np.uint32)).all()
     a.close()
     b.close()
+
+
+def test_offload_gather_rejects_stage12():
+    c = OffloadCase(5000, 2, 2, chunk=1024)
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_offload_gather_layer(c.h, 0, GuardedF16(10).ptr(), c.stream)
+    assert ei.value.code == A.ZERO_ERR_STAGE
+    c.close()

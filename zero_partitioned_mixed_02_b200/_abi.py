@@ -143,6 +143,7 @@ def lib():
             "zero_offload_state": (C.c_int, [P, C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                              C.POINTER(C.c_int64)]),
             "zero_offload_set_state": (C.c_int, [P, P, P, P, C.c_int64, P]),
+            "zero_offload_gather_layer": (C.c_int, [P, C.c_int32, P, P]),
             "zero_offload_host_update": (C.c_int, [P, P, P, P, P, C.c_int64, C.POINTER(zero_hyper),
                                                    C.c_int64, C.c_int, C.c_int]),
             "zero_offload_destroy": (None, [P]),
@@ -344,6 +345,10 @@ def zero_offload_state(h: int) -> tuple[int, int, int, int]:
     _check(lib().zero_offload_state(h, C.byref(w), C.byref(m), C.byref(v), C.byref(t)),
            "zero_offload_state")
     return w.value, m.value, v.value, t.value
+
+
+def zero_offload_gather_layer(h: int, unit: int, out: int, stream: int) -> None:
+    _check(lib().zero_offload_gather_layer(h, unit, out, stream), "zero_offload_gather_layer")
 
 
 def zero_offload_set_state(h: int, master: int, m: int, v: int, t: int, stream: int) -> None:

@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(kBlock) off_bcast_kernel(const OffRun* runs, i
 struct OffLayout {
     int64_t E = 0, C = 0, n_chunks = 0;
     // device
-    int64_t d_flag = 0, d_grad_tab = 0, d_out_tab = 0, d_runs = 0, d_red[S] = {}, d_p16[S] = {}, d_total = 0;
+    int64_t d_flag = 0, d_grad_tab = 0, d_out_tab = 0, d_runs = 0, d_gather = 0, d_red[S] = {}, d_p16[S] = {},
+            d_total = 0;
     // host staging
     int64_t h_flag = 0, h_grad_tab = 0, h_out_tab = 0, h_red[S] = {}, h_p16[S] = {}, h_total = 0;
     // chunk tables
@@ -210,6 +211,8 @@ int off_layout(const zl::Layout& L, int64_t chunk_elems, OffLayout* O)
     off += up((int64_t)std::max(L.n_out, 1) * 8);
     O->d_runs = off;
     off += up((int64_t)std::max<size_t>(O->runs.size(), 1) * sizeof(OffRun));
+    O->d_gather = off;  // stage 3: the layer-gather run table (shard index -> unit index)
+    off += up((int64_t)L.gather_segs.size() * sizeof(zk::SegDesc));
     for (int s = 0; s < S; ++s) {
         O->d_red[s] = off;
         off += up(4 * O->C);
@@ -409,6 +412,9 @@ struct zero_offload_handle {
     float* h_red(int s) const { return reinterpret_cast<float*>(hst + O.h_red[s]); }
     uint16_t* h_p16(int s) const { return reinterpret_cast<uint16_t*>(hst + O.h_p16[s]); }
     const OffRun* d_runs() const { return reinterpret_cast<const OffRun*>(dws + O.d_runs); }
+    const zk::SegDesc* d_gather() const { return reinterpret_cast<const zk::SegDesc*>(dws + O.d_gather); }
+    uint16_t* shards = nullptr;  // stage 3: the fp16 shard buffer (param_bufs[0])
+    int occ_gather = 0;
     const uint16_t* const* d_grad_tab() const { return reinterpret_cast<const uint16_t* const*>(dws + O.d_grad_tab); }
     uint16_t* const* d_out_tab() const { return reinterpret_cast<uint16_t* const*>(dws + O.d_out_tab); }
     unsigned* d_flag() const { return reinterpret_cast<unsigned*>(dws + O.d_flag); }
@@ -630,6 +636,13 @@ ZERO_API int zero_offload_init(const zero_config* cfg, int64_t chunk_elems, void
     if (e == cudaSuccess && !O.runs.empty())
         e = cudaMemcpyAsync(h->dws + O.d_runs, O.runs.data(), O.runs.size() * sizeof(OffRun), cudaMemcpyHostToDevice,
                             h->s_bc);
+    if (e == cudaSuccess && !L.gather_segs.empty())
+        e = cudaMemcpyAsync(h->dws + O.d_gather, L.gather_segs.data(), L.gather_segs.size() * sizeof(zk::SegDesc),
+                            cudaMemcpyHostToDevice, h->s_bc);
+    if (e == cudaSuccess && L.stage == 3) {
+        h->shards = param_bufs[0];
+        e = zk::occupancy(zk::K_GATHER, 0, &h->occ_gather);
+    }
     if (e == cudaSuccess) e = cudaStreamSynchronize(h->s_bc);
 
     // host state in state order (each thread first-touches the pages it will
@@ -719,6 +732,31 @@ ZERO_API int zero_offload_step(zero_offload_handle* h, const uint16_t* const* gr
     e = cudaEventRecord(h->ev_end, h->s_bc);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, h->ev_end, 0);
     if (e != cudaSuccess) return fail(h, e);
+    return ZERO_OK;
+}
+
+ZERO_API int zero_offload_gather_layer(zero_offload_handle* h, int32_t unit, uint16_t* out, void* stream)
+{
+    if (!h) return ZERO_ERR_ARG;
+    const zl::Layout& L = h->L;
+    if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (unit < 0 || unit >= L.n_units || !out) return ZERO_ERR_ARG;
+    if (!al16(out)) return ZERO_ERR_ALIGN;
+    const zl::Unit& U = L.units[unit];
+    if (U.n_chunks == 0) return ZERO_OK;
+    zk::GatherArgs g{};
+    g.segs = h->d_gather() + U.seg0;
+    g.n_segs = (int)U.n_segs;
+    g.n_chunks = U.n_chunks;
+    g.src = h->shards;
+    g.dst = out;
+    const int64_t want = (U.n_chunks + zk::kThreads / 32 - 1) / (zk::kThreads / 32);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)h->sms * std::max(1, h->occ_gather)));
+    const cudaError_t e = zk::launch_gather(g, grid, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        h->last_cuda = (int)e;
+        return ZERO_ERR_CUDA;
+    }
     return ZERO_OK;
 }
 

@@ -171,6 +171,10 @@ class ZeroOffloadAdam:
         hp = A.zero_hyper(lr, betas[0], betas[1], eps, weight_decay)
         return A.zero_offload_step(self.h, ptrs, loss_scale, hp, self.stream.cuda_stream) == A.ZERO_SKIPPED
 
+    def gather_layer(self, unit: int, out: torch.Tensor) -> None:
+        """Stage 3: the unit's full fp16 weights into `out` (on this object's stream)."""
+        A.zero_offload_gather_layer(self.h, unit, out.data_ptr(), self.stream.cuda_stream)
+
     @property
     def t(self) -> int:
         return A.zero_offload_state(self.h)[3]
