@@ -12,7 +12,9 @@ import os
 from typing import Sequence
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libzero.so")
+# ZERO_LIBZERO selects another build of the library (the bounds-checked
+# libzero_bounds.so); it must exist like the default one
+LIB_PATH = os.environ.get("ZERO_LIBZERO") or os.path.join(PKG, "libzero.so")
 
 ZERO_OK = 0
 ZERO_SKIPPED = 1

@@ -1,5 +1,6 @@
 """Build the package's native libraries in-tree for sm_100a.
 
+  libzero_bounds.so   the same with the kernels' index ranges checked (debug)
   libzero.so          the ZeRO step library (csrc/*.cu and the host update
                       csrc/zero_host_adam.cpp; C ABI in include/zero.h and
                       include/zero_offload.h)
@@ -22,6 +23,10 @@ INCLUDE = os.path.join(ROOT, "include")
 SYNTH = os.path.join(PKG, "synth")
 
 LIBZERO = os.path.join(PKG, "libzero.so")
+# the same library with every kernel's global index ranges checked
+# (ZK_BOUNDS_CHECK): an access outside a buffer is skipped and reported as
+# ZERO_ERR_INTERNAL; load it with ZERO_LIBZERO=<path> to run a test suite on it
+LIBZERO_DEBUG = os.path.join(PKG, "libzero_bounds.so")
 LIBSYNTH = os.path.join(SYNTH, "libzsynth.so")
 PTXAS_LOG = os.path.join(PKG, "libzero.ptxas.txt")
 
@@ -82,11 +87,17 @@ def _host_objects() -> list[str]:
 
 
 def build(force: bool = False) -> None:
-    if force or _stale(LIBZERO, ZERO_DEPS):
+    stale = force or _stale(LIBZERO, ZERO_DEPS)
+    stale_debug = force or _stale(LIBZERO_DEBUG, ZERO_DEPS)
+    if stale or stale_debug:
         objs = _host_objects()
-        _nvcc(LIBZERO, ZERO_SOURCES + objs,
-              ["-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v"],
-              log=PTXAS_LOG)
+        if stale:
+            _nvcc(LIBZERO, ZERO_SOURCES + objs,
+                  ["-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v"],
+                  log=PTXAS_LOG)
+        if stale_debug:
+            _nvcc(LIBZERO_DEBUG, ZERO_SOURCES + objs,
+                  ["-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fvisibility=hidden", "-DZK_BOUNDS_CHECK"])
         for o in objs:
             os.remove(o)
     if force or _stale(LIBSYNTH, SYNTH_DEPS):

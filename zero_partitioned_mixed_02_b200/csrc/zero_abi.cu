@@ -13,6 +13,7 @@
 #include "zero.h"
 #include "zero_internal.h"
 #include "zero_layout.h"
+#include "zero_nvtx.h"
 
 #define ZERO_API extern "C" __attribute__((visibility("default")))
 
@@ -468,6 +469,31 @@ int grid_for(const zero_handle* h, zk::Kernel k, int64_t chunks)
     return (int)std::min(want, cap);
 }
 
+// The error word and the buffers' element extents every kernel argument
+// carries (checked by the bounds-checked build).
+void set_extents(const zero_handle* h, zk::StepArgs& a)
+{
+    const Layout& L = h->L;
+    a.err = h->d_flag + 1;
+    a.grad_len = L.grad_len;
+    a.state_len = L.state_elems;
+    a.out_len = L.stage == 3 ? L.state_elems : L.psi;
+}
+
+// The kernel-error word after a synchronising call (only the bounds-checked
+// build sets it outside the steps): ZERO_ERR_INTERNAL, cleared, if it is set.
+int check_error_word(zero_handle* h, cudaStream_t s)
+{
+    unsigned word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, h->d_flag + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    if (word == 0) return ZERO_OK;
+    e = cudaMemsetAsync(h->d_flag + 1, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? ZERO_ERR_INTERNAL : cuda_fail(h, e);
+}
+
 // (double)b^t as the t-fold product, continued from the previous call when
 // possible (same multiplications in the same order as a fresh loop).
 void bias_corrections(zero_handle* h, float b1, float b2, int64_t t, float* bc1, float* bc2)
@@ -573,6 +599,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
                        const float* master_init, uint16_t* const* param_bufs, void* stream,
                        zero_handle** out)
 {
+    const zk::NvtxRange nvtx_range("zero_init");
     if (!out) return ZERO_ERR_ARG;
     *out = nullptr;
     zero_handle* h = new (std::nothrow) zero_handle();
@@ -682,11 +709,17 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
         a.v_out = h->state(0, 2);
         a.master_init = master_init;
         a.flag = h->d_flag;
+        set_extents(h, a);
         e = zk::launch_step(zk::K_INIT, a, grid_for(h, zk::K_INIT, L.step_chunks), s, L.bf16);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) {
         rc = cuda_fail(h, e);
+        delete h;
+        return rc;
+    }
+    rc = check_error_word(h, s);
+    if (rc != ZERO_OK) {
         delete h;
         return rc;
     }
@@ -697,6 +730,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
 ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, float loss_scale,
                               const zero_hyper* hp, void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_step_launch");
     if (!h || !grads || !hp) return ZERO_ERR_ARG;
     if (h->pending || h->async) return ZERO_ERR_ARG;  // uncommitted launch, or an asynchronous run is open
     if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale)) return ZERO_ERR_ARG;
@@ -731,6 +765,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
     a.n_out = (int)h->out_tab.size();
     a.flag = h->d_flag;
     a.call_id = h->call_id;
+    set_extents(h, a);
     a.c.inv_scale = (float)(1.0 / (double)loss_scale);
     a.c.lr = hp->lr;
     a.c.b1 = hp->beta1;
@@ -774,6 +809,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
 
 ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
 {
+    const zk::NvtxRange nvtx_range("zero_step_commit");
     if (skipped) *skipped = 0;
     if (!h || !h->pending) return ZERO_ERR_ARG;
     h->pending = false;
@@ -878,6 +914,7 @@ ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, cons
 
 ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_step_async");
     if (!h || !hp || !h->async) return ZERO_ERR_ARG;
     if (hp->beta1 != h->async_b1 || hp->beta2 != h->async_b2) return ZERO_ERR_ARG;
     if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
@@ -894,7 +931,7 @@ ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
     a.nd = L.nd;
     a.n_out = (int)h->out_tab.size();
     a.flag = h->d_flag;
-    a.err = h->d_flag + 1;
+    set_extents(h, a);
     a.call_id = 1;  // the commit kernel clears the word after every step
     a.c.lr = hp->lr;
     a.c.b1 = hp->beta1;
@@ -963,6 +1000,7 @@ ZERO_API int zero_async_end(zero_handle* h, void* stream, zero_async_state* out)
 
 ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_gather_layer");
     if (!h || h->pending) return ZERO_ERR_ARG;
     const Layout& L = h->L;
     if (L.stage != 3) return ZERO_ERR_STAGE;
@@ -981,6 +1019,8 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
         g.err = h->d_flag + 1;
         g.wait_rounds = h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds;
         g.hold_tile = h->hold_tile;
+        g.src_len = L.state_elems;
+        g.dst_len = U.numel;
         h->hold_tile = -1;
         const int64_t want = std::max<int64_t>(1, std::max(U.tma_tiles, (U.tma_scal + 31) / 32));
         const int64_t cap = (int64_t)h->sms * h->occ_gather_tma;
@@ -993,6 +1033,9 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     g.n_chunks = U.n_chunks;
     g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
     g.dst = out;
+    g.err = h->d_flag + 1;
+    g.src_len = L.state_elems;
+    g.dst_len = U.numel;
     const cudaError_t e = zk::launch_gather(g, grid_for(h, zk::K_GATHER, U.n_chunks),
                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
@@ -1001,6 +1044,7 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
 ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m, const float* v, int64_t t,
                            void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_set_state");
     if (!h || h->pending || h->async || t < 0) return ZERO_ERR_ARG;
     const Layout& L = h->L;
     const size_t bytes = (size_t)L.state_elems * sizeof(float);
@@ -1026,10 +1070,13 @@ ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m,
         a.nd = L.nd;
         a.w_in = L.bf16 ? master : h->state(h->cur, 0);
         a.flag = h->d_flag;
+        set_extents(h, a);
         e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s, L.bf16);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(h, e);
+    const int rc = check_error_word(h, s);
+    if (rc != ZERO_OK) return rc;
     h->t = t;
     h->bc_t = -1;  // recompute the bias-correction products for the new t
     return ZERO_OK;

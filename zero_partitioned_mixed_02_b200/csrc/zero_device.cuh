@@ -18,6 +18,21 @@ __device__ __forceinline__ bool nonfinite(float x)
     return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
 }
 
+// The bounds-checked build (ZK_BOUNDS_CHECK): an access to elements
+// [i, i + n) of a buffer of len elements that is not inside it sets bit 32 of
+// the error word and is skipped (the host reports ZERO_ERR_INTERNAL). In the
+// normal build the check is the constant true and compiles away.
+#ifdef ZK_BOUNDS_CHECK
+__device__ __forceinline__ bool in_bounds(long long i, long long n, long long len, unsigned* err)
+{
+    if (i >= 0 && n >= 0 && i + n <= len) return true;
+    atomicOr(err, 32u);
+    return false;
+}
+#else
+__device__ __forceinline__ bool in_bounds(long long, long long, long long, unsigned*) { return true; }
+#endif
+
 __device__ __forceinline__ float h2f(unsigned short b) { return __half2float(__ushort_as_half(b)); }
 
 __device__ __forceinline__ unsigned short f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
@@ -300,6 +315,9 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, co
                                             bool& bad)
 {
     const long long gi = d.grad_begin + e, si = d.state_begin + e, oi = d.out_begin + e;
+    if (!(in_bounds(gi, 1, a.grad_len, a.err) & in_bounds(si, 1, a.state_len, a.err) &
+          in_bounds(oi, 1, a.out_len, a.err)))
+        return;
     float w = 0.0f, m = 0.0f, v = 0.0f, g = 0.0f;
     if (K == K_INIT) {
         w = __ldcs(a.master_init + gi);

@@ -88,6 +88,9 @@ struct StepArgs {
     const Ctrl* ctrl;
     float* st[2][3];
     unsigned* err;                 // kernel error word (roll-back condition)
+    // element extents of the buffers (grads and master_init; state arrays and
+    // red; outputs), checked by the bounds-checked build (ZK_BOUNDS_CHECK)
+    long long grad_len, state_len, out_len;
 };
 
 struct GatherArgs {
@@ -96,6 +99,8 @@ struct GatherArgs {
     long long n_chunks;
     const uint16_t* src;
     uint16_t* dst;
+    unsigned* err;                // error word (bounds-checked build)
+    long long src_len, dst_len;   // element extents (bounds-checked build)
 };
 
 // ---- the TMA-staged fused step ----
@@ -173,6 +178,7 @@ struct TmaGatherArgs {
     unsigned* err;
     unsigned wait_rounds;
     long long hold_tile;
+    long long src_len, dst_len;  // element extents (bounds-checked build)
 };
 
 // try_wait rounds (each may suspend about a microsecond) before a wait of the

@@ -47,6 +47,11 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const
     const long long sa = d.state_begin + p.ea, sb = d.state_begin + p.eb;
     const long long oa = d.out_begin + p.ea, ob = d.out_begin + p.eb;
     const bool hb = p.hb;
+    if (!(in_bounds(ga, 4, a.grad_len, a.err) & in_bounds(sa, 4, a.state_len, a.err) &
+          in_bounds(oa, 4, a.out_len, a.err) &
+          (!hb || (in_bounds(gb, 4, a.grad_len, a.err) & in_bounds(sb, 4, a.state_len, a.err) &
+                   in_bounds(ob, 4, a.out_len, a.err)))))
+        return;
     float w[8], m[8], v[8], g[8];
     if (K == K_INIT) {
         ld_pair(a.master_init, ga, gb, hb, w);
@@ -184,12 +189,19 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const GatherArgs a)
     walk(
         a.segs, a.n_segs, a.n_chunks,
         [&](const SegDesc& d, const Pair& p) {
+            if (!(in_bounds(d.grad_begin + p.ea, 4, a.src_len, a.err) &
+                  in_bounds(d.out_begin + p.ea, 4, a.dst_len, a.err) &
+                  (!p.hb || (in_bounds(d.grad_begin + p.eb, 4, a.src_len, a.err) &
+                             in_bounds(d.out_begin + p.eb, 4, a.dst_len, a.err)))))
+                return;
             const uint2 qa = ld_hq(a.src + d.grad_begin + p.ea);
             const uint2 qb = p.hb ? ld_hq(a.src + d.grad_begin + p.eb) : make_uint2(0u, 0u);
             st_hq(a.dst + d.out_begin + p.ea, qa);
             if (p.hb) st_hq(a.dst + d.out_begin + p.eb, qb);
         },
         [&](const SegDesc& d, long long e) {
+            if (!(in_bounds(d.grad_begin + e, 1, a.src_len, a.err) & in_bounds(d.out_begin + e, 1, a.dst_len, a.err)))
+                return;
             __stcs(reinterpret_cast<unsigned short*>(a.dst + d.out_begin + e),
                    __ldcs(reinterpret_cast<const unsigned short*>(a.src + d.grad_begin + e)));
         });

@@ -37,6 +37,7 @@
 #include "zero_host_adam.h"
 #include "zero_internal.h"
 #include "zero_layout.h"
+#include "zero_nvtx.h"
 #include "zero_offload.h"
 
 #define ZERO_API extern "C" __attribute__((visibility("default")))
@@ -665,6 +666,7 @@ ZERO_API int zero_offload_init(const zero_config* cfg, int64_t chunk_elems, void
 ZERO_API int zero_offload_step(zero_offload_handle* h, const uint16_t* const* grads, float loss_scale,
                                const zero_hyper* hp, void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_offload_step");
     if (!h || !grads || !hp) return ZERO_ERR_ARG;
     if (h->broken) return ZERO_ERR_CUDA;
     if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale)) return ZERO_ERR_ARG;
@@ -718,6 +720,7 @@ ZERO_API int zero_offload_step(zero_offload_handle* h, const uint16_t* const* gr
         e = cudaEventSynchronize(h->ev_d2h[s]);           // reduced gradient of chunk k on the host
         if (e == cudaSuccess) e = cudaEventSynchronize(h->ev_h2d[s]);  // host fp16 slot free
         if (e != cudaSuccess) return fail(h, e);
+        const zk::NvtxRange chunk_range("offload host update chunk");
         const int64_t c0 = h->chunk_begin(k);
         const float* g = h->h_red(s);
         uint16_t* p16 = h->h_p16(s);
@@ -737,6 +740,7 @@ ZERO_API int zero_offload_step(zero_offload_handle* h, const uint16_t* const* gr
 
 ZERO_API int zero_offload_gather_layer(zero_offload_handle* h, int32_t unit, uint16_t* out, void* stream)
 {
+    const zk::NvtxRange nvtx_range("zero_offload_gather_layer");
     if (!h) return ZERO_ERR_ARG;
     const zl::Layout& L = h->L;
     if (L.stage != 3) return ZERO_ERR_STAGE;
@@ -750,6 +754,9 @@ ZERO_API int zero_offload_gather_layer(zero_offload_handle* h, int32_t unit, uin
     g.n_chunks = U.n_chunks;
     g.src = h->shards;
     g.dst = out;
+    g.err = h->d_flag() + 1;
+    g.src_len = L.state_elems;
+    g.dst_len = U.numel;
     const int64_t want = (U.n_chunks + zk::kThreads / 32 - 1) / (zk::kThreads / 32);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)h->sms * std::max(1, h->occ_gather)));
     const cudaError_t e = zk::launch_gather(g, grid, static_cast<cudaStream_t>(stream));

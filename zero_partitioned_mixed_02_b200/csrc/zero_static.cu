@@ -118,7 +118,7 @@ ZERO_API int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* gr
     }
 
     // the array keeps the last call's contents: clear the overflow word
-    cudaError_t e = cudaMemsetAsync(base + kFlagOff, 0, sizeof(unsigned), s);
+    cudaError_t e = cudaMemsetAsync(base + kFlagOff, 0, 2 * sizeof(unsigned), s);  // overflow, error words
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(base + kGradTabOff, grad_tab, nd * sizeof(void*), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess)
@@ -143,6 +143,8 @@ ZERO_API int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* gr
     a.v_out = v;
     a.red = reinterpret_cast<float*>(base + kRedOff);
     a.flag = reinterpret_cast<unsigned*>(base + kFlagOff);
+    a.err = a.flag + 1;
+    a.grad_len = a.state_len = a.out_len = psi;
     a.call_id = 1;
     a.c.inv_scale = (float)(1.0 / (double)loss_scale);
     a.c.lr = hp->lr;
@@ -165,10 +167,12 @@ ZERO_API int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* gr
     const int g1 = (int)std::min<int64_t>(want, (int64_t)g_sms[dev] * std::max(1, g_occ[dev][1]));
     e = zk::launch_step(zk::K_REDUCE, a, g0, s);
     if (e == cudaSuccess) e = zk::launch_step(zk::K_UPDATE, a, g1, s);
-    unsigned flag = 0;
-    if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, base + kFlagOff, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    unsigned words[2] = {0, 0};  // overflow word, error word (bounds-checked build)
+    if (e == cudaSuccess) e = cudaMemcpyAsync(words, base + kFlagOff, sizeof(words), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    if (words[1] != 0) return ZERO_ERR_INTERNAL;
+    const unsigned flag = words[0];
     if (flag == a.call_id) {
         if (skipped) *skipped = 1;
         return ZERO_SKIPPED;

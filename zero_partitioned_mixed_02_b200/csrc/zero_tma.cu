@@ -87,6 +87,12 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
             d.decay = run.decay;
             char* sp = stage0 + st * stage_bytes;
             const unsigned full = full0 + 8 * st;
+            if (!(in_bounds(d.gi, n, b.grad_len, a.err) & in_bounds(d.si, n, b.state_len, a.err) &
+                  in_bounds(d.oi, n, b.out_len, a.err))) {
+                d.n = 0;  // bounds-checked build: an empty tile, the stage completes at once
+                mbar_expect_tx(full, 0u);
+                continue;
+            }
             mbar_expect_tx(full, (unsigned)n * (unsigned)(2 * nd + 12));
             for (int k = 0; k < nd; ++k)
                 bulk_g2s(smem_u32(sp + k * kTmaTile * 2), b.grads[k] + d.gi, 2u * n, full);
@@ -245,7 +251,10 @@ __global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
                 tiles[st].d = run.out_begin + e0;
                 tiles[st].bytes = 2u * n;
                 const unsigned full = full0 + 8 * st;
-                if (t != a.hold_tile) {  // test hook: leave this stage unarmed
+                if (!(in_bounds(tiles[st].s, n, a.src_len, a.err) & in_bounds(tiles[st].d, n, a.dst_len, a.err))) {
+                    tiles[st].bytes = 0;  // bounds-checked build: skip the tile
+                    mbar_expect_tx(full, 0u);
+                } else if (t != a.hold_tile) {  // test hook: leave this stage unarmed
                     mbar_expect_tx(full, 2u * n);
                     bulk_g2s(smem_u32(stage0 + st * kGatherTile * 2), a.src + tiles[st].s, 2u * n, full);
                 }
@@ -257,8 +266,10 @@ __global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
                 failed = true;
                 break;
             }
-            bulk_s2g(a.dst + tiles[st].d, smem_u32(stage0 + st * kGatherTile * 2), tiles[st].bytes);
-            bulk_commit();
+            if (tiles[st].bytes != 0) {
+                bulk_s2g(a.dst + tiles[st].d, smem_u32(stage0 + st * kGatherTile * 2), tiles[st].bytes);
+                bulk_commit();
+            }
         }
         // drain: issued loads must land, issued stores must finish, before exit
         for (long long i = issued - 1; i >= 0 && i >= issued - S; --i)
@@ -278,6 +289,8 @@ __global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
         const TmaRun& run = a.runs[r];
         const long long q = j - run.scal_begin;
         const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
+        if (!(in_bounds(run.grad_begin + e, 1, a.src_len, a.err) & in_bounds(run.out_begin + e, 1, a.dst_len, a.err)))
+            continue;
         __stcs(reinterpret_cast<unsigned short*>(a.dst + run.out_begin + e),
                __ldcs(reinterpret_cast<const unsigned short*>(a.src + run.grad_begin + e)));
     }

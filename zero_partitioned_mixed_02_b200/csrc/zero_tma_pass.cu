@@ -102,6 +102,12 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) pass_tma_kernel(const Tma
             d.decay = run.decay;
             char* sp = stage0 + st * stage_bytes;
             const unsigned full = full0 + 8 * st;
+            if (!(in_bounds(d.gi, n, b.grad_len, a.err) & in_bounds(d.si, n, b.state_len, a.err) &
+                  in_bounds(d.oi, n, b.out_len, a.err))) {
+                d.n = 0;  // bounds-checked build: an empty tile, the stage completes at once
+                mbar_expect_tx(full, 0u);
+                continue;
+            }
             mbar_expect_tx(full, (unsigned)n * (unsigned)pass_elem_bytes<MODE, C>(nd));
             if (MODE == kPassReduce) {
                 for (int k = 0; k < nd; ++k)
