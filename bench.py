@@ -64,7 +64,7 @@ def parse_args():
                    help="host threads of the offloaded update (0: every core this process may use)")
     p.add_argument("--offload-chunk", type=int, default=0,
                    help="elements per pipeline chunk of the offloaded step (0: the library default)")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -626,41 +626,72 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
                                f"ranks, {avail / 1e9:.1f} GB available"}
     s = torch.cuda.current_stream()
     side = torch.cuda.Stream()  # device->host reads of the result
+    up = torch.cuda.Stream()    # host->device uploads of the gradients
     host_g = [torch.empty(n_own, dtype=torch.int16, pin_memory=True) for _ in grads]
     for hg, g in zip(host_g, grads):
         hg.copy_(g)
     host_out = torch.empty(result.numel(), dtype=torch.int16, pin_memory=True)
+    # two device gradient sets: step k reads set k % 2 while the inputs of
+    # step k + 1 travel into the other one (every step's inputs still cross
+    # the link inside the timed region)
+    try:
+        sets = [grads, [torch.empty_like(g) for g in grads]]
+        pipelined = True
+    except torch.cuda.OutOfMemoryError:  # one set: each upload waits for the step before
+        sets = [grads, grads]
+        pipelined = False
+    ptrs = [[g.data_ptr() for g in x] for x in sets]
+    uploaded = [None, None]  # upload of each set done
+    used = [None, None]      # last step that read each set done
     read_done = None
 
-    def step():
-        # the gradient upload of this step overlaps the read-back of the last
-        # step's result; the step itself waits for that read-back to finish
+    def upload(k):
+        i = k % 2
+        if used[i] is not None:
+            up.wait_event(used[i])
+        with torch.cuda.stream(up):
+            for g, hg in zip(sets[i], host_g):
+                g.copy_(hg, non_blocking=True)
+        uploaded[i] = torch.cuda.Event()
+        uploaded[i].record(up)
+
+    def step(k, last):
+        # enqueue the next step's upload first: it runs while this step's
+        # kernels run and the last step's result is read back
         nonlocal read_done
-        for g, hg in zip(grads, host_g):
-            g.copy_(hg, non_blocking=True)
+        i = k % 2
+        if pipelined and k + 1 <= last:
+            upload(k + 1)
+        s.wait_event(uploaded[i])
         if read_done is not None:
-            s.wait_event(read_done)
-        rc = A.zero_step(h, gptrs, wl.loss_scale, hp, s.cuda_stream)
+            s.wait_event(read_done)  # the result buffer is free again
+        rc = A.zero_step(h, ptrs[i], wl.loss_scale, hp, s.cuda_stream)
         if rc != A.ZERO_OK:
             raise RuntimeError("unexpected skip")
         for u in order:
             A.zero_gather_layer(h, u, gather_out.data_ptr(), s.cuda_stream)
         done = torch.cuda.Event()
         done.record(s)
+        used[i] = done
         side.wait_event(done)
         with torch.cuda.stream(side):
             host_out.copy_(result, non_blocking=True)
         read_done = torch.cuda.Event()
         read_done.record(side)
+        if not pipelined and k + 1 <= last:
+            upload(k + 1)  # after the step: it overwrites the gradients the step read
 
-    step()
+    upload(0)
+    step(0, 0)  # warm-up
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(s)
-    for _ in range(args.e2e_steps):
-        step()
+    up.wait_event(a)
+    upload(0)
+    for k in range(args.e2e_steps):
+        step(k, args.e2e_steps - 1)
     s.wait_event(read_done)  # the last read-back is inside the timed region
     b.record(s)
     torch.cuda.synchronize()
@@ -668,7 +699,7 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
     n = L.state_elems
     return {"value": whole_job_value(n, args.e2e_steps, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": len(grads) * n_own * 2, "d2h_bytes_per_step": result.numel() * 2,
-            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
+            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps, "pipelined": pipelined}
 
 
 def host_copy_gbs(threads, n_bytes=1 << 31, reps=5):
