@@ -109,6 +109,31 @@ def algorithmic_bytes(wl, variant, bf16=False):
 
 
 # ---------------------------------------------------------------- environment
+def stream_copy_gbs(n_bytes=1 << 32, reps=10):
+    """This library's own copy kernel (zero_stream_copy) on n_bytes, read +
+    written bytes per second, median of reps: a same-run reference beside the
+    pool's measured peak."""
+    import torch
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+
+    src = torch.empty(n_bytes, dtype=torch.uint8, device="cuda")
+    dst = torch.empty_like(src)
+    s = torch.cuda.current_stream()
+    A.zero_stream_copy(dst.data_ptr(), src.data_ptr(), n_bytes, s.cuda_stream)
+    ms = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        A.zero_stream_copy(dst.data_ptr(), src.data_ptr(), n_bytes, s.cuda_stream)
+        b.record(s)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    del src, dst
+    torch.cuda.empty_cache()
+    return 2 * n_bytes / (sorted(ms)[len(ms) // 2] / 1e3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -509,6 +534,11 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
     }
+    # this library's copy kernel on 4 GB, after the timed region (context for
+    # the measured peak, which stays the denominator)
+    line["stream_copy"] = {"kernel": "zero_stream_copy", "bytes": 1 << 32, "gbs": stream_copy_gbs(),
+                           "frac_of_peak": None}
+    line["stream_copy"]["frac_of_peak"] = line["stream_copy"]["gbs"] / peak
     if gather_events:
         g_ms = statistics.mean(a.elapsed_time(b) for a, b in gather_events)
         line["gathers"] = {"per_step_ms": g_ms, "launches_per_step": len(order),
