@@ -10,7 +10,7 @@
  * so that every binary32 operation below is one IEEE-rounded operation in the
  * order written (no FMA contraction, no flush-to-zero, SSE arithmetic).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - Adam is the Kingma-Ba bias-corrected form, eps outside the square root,
  *    m-hat and v-hat formed by division; weight decay is decoupled and scaled
  *    by lr (AdamW).  [P2] "Where We Were" names Adam/AdamW without equations.

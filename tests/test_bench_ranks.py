@@ -62,9 +62,8 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
 
 def test_algorithmic_bytes_per_element():
     """The roofline's numerator: bytes per updated element of each workload,
-    variant and precision, from the step's definition (SURVEY's per-unit
-    figures: (24 + 4 Nd) for stage 1/2, (26 + 2 Nd) for stage 3, 154 per
-    element of the Nd = 64 rank view)."""
+    variant and precision, from the step's definition: (24 + 4 Nd) for stage
+    1/2, (26 + 2 Nd) for stage 3, 154 per element of the Nd = 64 rank view."""
     from zero_partitioned_mixed_02_b200.synth import workloads as W
     g = W.gpt2_1p5b()
     n, floor, per, gathers = bench.algorithmic_bytes(g, "fused-tma")
