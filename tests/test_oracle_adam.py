@@ -393,3 +393,47 @@ def test_masked_decay_is_elementwise_selection(seed):
         assert (out["masked"][k].view(np.uint8) == expect.view(np.uint8)).all()
         assert (out["ones"][k].view(np.uint8) == out["wd"][k].view(np.uint8)).all()
     assert (out["wd"][0] != out["nowd"][0]).any()
+
+
+# ---- ZeRO == DP on random sizes (beyond the brute-force grid) ---------------
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(psi=st.integers(1, 5000), nd=st.integers(1, 64), n_t=st.integers(1, 6), seed=st.integers(0, 10**6))
+def test_zero_stages_equal_dp_random(psi, nd, n_t, seed):
+    """Stage 1/2 and stage 3 (random tensor split) are bit-identical to the
+    plain data-parallel step, including empty partitions and chunks."""
+    rng = np.random.default_rng(seed)
+    n_t = min(n_t, psi)
+    cuts = np.sort(rng.choice(np.arange(1, psi), size=n_t - 1, replace=False)) if n_t > 1 else []
+    numel = [int(x) for x in np.diff(np.concatenate([[0], cuts, [psi]]))]
+    w0 = rng.uniform(-1, 1, psi).astype(np.float32)
+    gs = _grads(rng, nd, psi, sigma=1e-3, scale=256.0)
+    hp = Z.hyper(lr=1e-2, weight_decay=0.01)
+    w, m, v, p = w0.copy(), np.zeros(psi, np.float32), np.zeros(psi, np.float32), np.zeros(psi, np.uint16)
+    _, t = Z.dp_step(gs, w, m, v, p, 256.0, hp, 0)
+    # stage 1/2
+    parts = [Z.partition(psi, nd, r) for r in range(nd)]
+    ws = [w0[b:e].copy() for b, e in parts]
+    ms = [np.zeros(e - b, np.float32) for b, e in parts]
+    vs = [np.zeros(e - b, np.float32) for b, e in parts]
+    reps = [np.zeros(psi, np.uint16) for _ in range(nd)]
+    _, t12 = Z.zero12_step(psi, gs, ws, ms, vs, reps, 256.0, hp, 0)
+    assert t12 == t
+    assert (np.concatenate(ws).view(np.uint32) == w.view(np.uint32)).all()
+    assert all((r == p).all() for r in reps)
+    # stage 3
+    offs = np.concatenate([[0], np.cumsum(numel)])
+    w3 = [np.concatenate([w0[offs[i] + b: offs[i] + e] for i, n in enumerate(numel)
+                          for b, e in [Z.chunk(n, nd, r)]]).astype(np.float32) for r in range(nd)]
+    m3 = [np.zeros_like(x) for x in w3]
+    v3 = [np.zeros_like(x) for x in w3]
+    p3 = [np.zeros(x.size, np.uint16) for x in w3]
+    _, t3 = Z.zero3_step(numel, gs, w3, m3, v3, p3, 256.0, hp, 0)
+    assert t3 == t
+    units = list(range(len(numel)))
+    for u in units:
+        got = Z.zero3_gather(numel, units, nd, u, p3)
+        assert (got == p[offs[u]:offs[u + 1]]).all()
