@@ -145,3 +145,34 @@ def test_offload_object_equals_device_object():
     compare_f32(off.state()[0].numpy(), host_f32(dev.state()[0]), "master after load")
     dev.close()
     off.close()
+
+
+def test_zero_adam_bf16_object():
+    """ZeroAdam with precision=bf16 and the default variant runs the two-pass
+    TMA step; its state has no master; three steps equal the oracle."""
+    from zero_partitioned_mixed_02_b200 import ZeroAdam
+    psi, nd = 20_000, 4
+    w0 = S.host_f32(psi, 0, S.key(3, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
+    reps = [torch.zeros(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
+    opt = ZeroAdam(psi, nd, 2, torch.from_numpy(w0.copy()).cuda(), reps, precision=A.ZERO_PRECISION_BF16)
+    assert opt.cfg.c.variant == A.ZERO_VARIANT_TWO_PASS_TMA
+    w16 = Z.bf16_from_f32(w0)
+    m, v, t = np.zeros(psi, np.float32), np.zeros(psi, np.float32), 0
+    grads = [torch.empty(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
+    for s in range(3):
+        gs = [Z.bf16_from_f32(S.host_f32(psi, 0, S.key(3, S.STREAM_GRAD, s, k), S.normal(1e-3, 1.0)))
+              for k in range(nd)]
+        for g, x in zip(grads, gs):
+            g.copy_(torch.from_numpy(x.view(np.int16)))
+        assert opt.step(grads, 1.0, weight_decay=0.01) is False
+        _, t = Z.bf16_step(gs, w16, m, v, 1.0, Z.hyper(weight_decay=0.01), t)
+    gw, gm, gv = opt.state()
+    assert gw is None
+    compare_f32(host_f32(gm), m, "m")
+    compare_f32(host_f32(gv), v, "v")
+    for r in reps:
+        compare_f16(host_u16(r), w16, "bf16 replica")
+    sd = opt.state_dict()
+    assert sd["master"] is None and sd["t"] == 3
+    opt.load_state_dict(sd)
+    opt.close()

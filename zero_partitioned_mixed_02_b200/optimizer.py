@@ -28,7 +28,10 @@ class ZeroAdam:
                  stream: torch.cuda.Stream | None = None,
                  precision: int = A.ZERO_PRECISION_FP16):
         """precision = ZERO_PRECISION_BF16: bfloat16 gradients and parameters
-        without fp32 master weights (variant must be a two-pass one)."""
+        without fp32 master weights; only the two-pass variants exist for it,
+        so a fused variant is replaced by ZERO_VARIANT_TWO_PASS_TMA."""
+        if precision == A.ZERO_PRECISION_BF16 and variant in (A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_FUSED_TMA):
+            variant = A.ZERO_VARIANT_TWO_PASS_TMA
         self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors,
                             precision=precision)
         self.ledger = A.zero_state_bytes(self.cfg)
