@@ -1,11 +1,13 @@
 /* A plain C caller of libzero's host-only calls: the headers must compile as
  * C and the symbols link without C++ or CUDA on the caller's side. Prints the
- * ledger of the 7.5B-parameter, Nd = 64 running example ([P1] stage table)
- * and the offloaded step's residency for stage 2. */
+ * ledger of the 7.5B-parameter, Nd = 64 running example ([P1] stage table),
+ * the offloaded step's residency for stage 2, and the peer descriptor's
+ * size. */
 #include <stdio.h>
 
 #include "zero.h"
 #include "zero_offload.h"
+#include "zero_peer.h"
 
 int main(void)
 {
@@ -30,5 +32,7 @@ int main(void)
     printf("offload %lld %lld\n", (long long)O.host_state_bytes, (long long)O.device_state_bytes);
     cfg.nd = 0;
     printf("bad %d\n", zero_state_bytes(&cfg, &L));
+    zero_peer_desc d = {0};
+    printf("peer %u %d\n", (unsigned)sizeof d, zero_peer_open(&d, NULL));
     return 0;
 }

@@ -29,3 +29,4 @@ def test_c_caller(tmp_path):
     host, dev = (int(x) for x in out[2].split()[1:])
     assert host == 12 * 117187500 and dev == 2 * 7500000000 + 2 * 117187500
     assert out[3] == "bad -1"
+    assert out[4] == "peer 104 -1"

@@ -93,6 +93,16 @@ class zero_offload_ledger(C.Structure):
 ZERO_OFFLOAD_SLOTS = 3
 ZERO_OFFLOAD_DEFAULT_CHUNK = 1 << 22
 
+
+class zero_peer_desc(C.Structure):
+    _fields_ = [("magic", C.c_uint32), ("device", C.c_int32), ("process", C.c_uint64),
+                ("offset", C.c_uint64), ("bytes", C.c_uint64), ("address", C.c_uint64),
+                ("ipc", C.c_ubyte * 64)]
+
+
+ZERO_PEER_MAGIC = 0x5A505231
+ZERO_PEER_DESC_BYTES = 104
+
 _lib = None
 
 
@@ -149,6 +159,11 @@ def lib():
             "zero_offload_host_update": (C.c_int, [P, P, P, P, P, C.c_int64, C.POINTER(zero_hyper),
                                                    C.c_int64, C.c_int, C.c_int]),
             "zero_offload_destroy": (None, [P]),
+            "zero_peer_export": (C.c_int, [P, C.c_size_t, C.POINTER(zero_peer_desc)]),
+            "zero_peer_open": (C.c_int, [C.POINTER(zero_peer_desc), C.POINTER(P)]),
+            "zero_peer_close": (C.c_int, [C.POINTER(zero_peer_desc), P]),
+            "zero_peer_open_count": (C.c_int, []),
+            "zero_peer_last_cuda_error": (C.c_int, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -365,3 +380,39 @@ def zero_offload_host_update(g: int, w: int, m: int, v: int, p16: int, n: int, h
 
 def zero_offload_destroy(h: int) -> None:
     lib().zero_offload_destroy(h)
+
+
+# ---- peer buffers (include/zero_peer.h) ----
+
+def _peer_check(rc: int, where: str) -> int:
+    if rc < 0:
+        raise ZeroError(rc, where, lib().zero_peer_last_cuda_error())
+    return rc
+
+
+def _desc(desc: bytes) -> zero_peer_desc:
+    if len(desc) != C.sizeof(zero_peer_desc):
+        raise ZeroError(ZERO_ERR_ARG, "peer descriptor length")
+    return zero_peer_desc.from_buffer_copy(desc)
+
+
+def zero_peer_export(dev_ptr: int, nbytes: int) -> bytes:
+    """Descriptor (104 bytes) of the device buffer [dev_ptr, dev_ptr + nbytes)."""
+    d = zero_peer_desc()
+    _peer_check(lib().zero_peer_export(dev_ptr, int(nbytes), C.byref(d)), "zero_peer_export")
+    return bytes(d)
+
+
+def zero_peer_open(desc: bytes) -> int:
+    """This process's address of the buffer a descriptor names."""
+    p = C.c_void_p()
+    _peer_check(lib().zero_peer_open(C.byref(_desc(desc)), C.byref(p)), "zero_peer_open")
+    return p.value
+
+
+def zero_peer_close(desc: bytes, dev_ptr: int) -> None:
+    _peer_check(lib().zero_peer_close(C.byref(_desc(desc)), dev_ptr), "zero_peer_close")
+
+
+def zero_peer_open_count() -> int:
+    return lib().zero_peer_open_count()

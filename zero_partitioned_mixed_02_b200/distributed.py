@@ -13,6 +13,12 @@ and the commit the ranks reduce the handle's two flag words with MAX.
 
 flag_words(h) is a zero-copy torch view of the two words (int32), usable
 with torch.distributed.all_reduce on the NCCL backend.
+
+PeerBuffers exchanges descriptors of device buffers (include/zero_peer.h)
+across the group and maps every rank's buffers into this process; PeerRank
+is the whole per-rank job of stages 1 and 2 on top of it: this rank's
+gradient and parameter buffers shared with the others, one handle, and the
+step bracketed by device barriers.
 """
 from __future__ import annotations
 
@@ -50,5 +56,156 @@ def rank_step(h: int, grads: Sequence[int], loss_scale: float, hp: A.zero_hyper,
     step's stream, commit. Returns True if the step was skipped."""
     A.zero_step_launch(h, grads, loss_scale, hp, stream.cuda_stream)
     with torch.cuda.stream(stream):
-        agree_overflow(flag_words(h), group)
+        agree_overflow_any(flag_words(h, stream.device), group)
     return A.zero_step_commit(h, stream.cuda_stream) == A.ZERO_SKIPPED
+
+
+def _is_nccl(group=None) -> bool:
+    return dist.get_backend(group) == "nccl"
+
+
+def agree_overflow_any(words: torch.Tensor, group=None) -> torch.Tensor:
+    """agree_overflow on any backend: NCCL reduces the device words in stream
+    order; other backends (gloo) reduce a host copy, which waits for the
+    current stream."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return words
+    if _is_nccl(group) or words.device.type == "cpu":
+        return agree_overflow(words, group)
+    host = words.cpu()
+    dist.all_reduce(host, op=dist.ReduceOp.MAX, group=group)
+    words.copy_(host)
+    return words
+
+
+def device_barrier(stream: torch.cuda.Stream, group=None) -> None:
+    """Order the GPU work of every rank: work enqueued on `stream` after this
+    call starts only once every rank's work enqueued before its own call has
+    finished. NCCL: a one-word all-reduce on the stream (no host wait); other
+    backends: a stream synchronise and a host barrier."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return
+    if _is_nccl(group):
+        with torch.cuda.stream(stream):
+            dist.all_reduce(torch.zeros(1, dtype=torch.int32, device=stream.device), group=group)
+    else:
+        stream.synchronize()
+        dist.barrier(group=group)
+
+
+class _ApiPeers:
+    """The library's peer calls (include/zero_peer.h)."""
+    export = staticmethod(A.zero_peer_export)
+    open = staticmethod(A.zero_peer_open)
+    close = staticmethod(A.zero_peer_close)
+
+
+class PeerBuffers:
+    """Every rank's counterpart of some local device buffers, addressable
+    from this process. ptrs[k][j] is this process's address of rank k's j-th
+    buffer (its own buffers are returned unchanged). Collective: every rank of
+    the group constructs it with the same number of buffers, and close() is
+    collective too (it waits until no rank can still use a mapping, then
+    releases them)."""
+
+    def __init__(self, buffers: Sequence[tuple[int, int]], group=None, api=_ApiPeers):
+        """buffers: (device address, bytes) per local buffer."""
+        self._api = api
+        self._group = group
+        mine = [api.export(int(p), int(n)) for p, n in buffers]
+        world = dist.get_world_size(group)
+        rows: list = [None] * world
+        dist.all_gather_object(rows, mine, group=group)
+        if any(len(r) != len(mine) for r in rows):
+            raise ValueError("every rank must share the same number of buffers")
+        self.descs = rows
+        self.ptrs: list[list[int]] = []
+        try:
+            for row in rows:
+                self.ptrs.append([])
+                for d in row:
+                    self.ptrs[-1].append(api.open(d))
+        except Exception:
+            self._release()
+            raise
+
+    def _release(self) -> None:
+        for row, prow in zip(self.descs, self.ptrs):
+            for d, p in zip(row, prow):
+                self._api.close(d, p)
+        self.ptrs = []
+
+    def close(self, stream: torch.cuda.Stream | None = None) -> None:
+        if stream is not None:
+            stream.synchronize()
+        dist.barrier(group=self._group)  # nobody is still reading or writing through a mapping
+        self._release()
+        dist.barrier(group=self._group)  # nobody frees a buffer another rank still maps
+
+
+class PeerRank:
+    """Rank r of a real Nd-rank stage 1/2 job, one process per GPU (Nd = the
+    group's size). `grad` and `params` are this rank's full-length 16-bit
+    gradient and parameter buffers (torch tensors of psi elements); the handle
+    reads partition r of every rank's gradient and writes partition r of the
+    new parameters into every rank's `params` through peer mappings.
+
+    step(): a device barrier (every rank's gradient is written), the step
+    launch, the overflow agreement, the commit, and a second device barrier
+    (every rank's partition is in every parameter buffer)."""
+
+    def __init__(self, grad: torch.Tensor, params: torch.Tensor, master_init: torch.Tensor,
+                 stage: int = 2, variant: int = A.ZERO_VARIANT_FUSED_TMA,
+                 precision: int = A.ZERO_PRECISION_FP16, tensors=None, group=None,
+                 stream: torch.cuda.Stream | None = None):
+        """master_init: fp32 device tensor with this rank's partition of the
+        initial master weights (for bfloat16 without master: of the initial
+        weights)."""
+        if stage not in (1, 2):
+            raise ValueError("peer ranks run stage 1 or 2")
+        psi = params.numel()
+        if grad.numel() != psi or grad.element_size() != 2 or params.element_size() != 2:
+            raise ValueError("grad and params: 16-bit tensors of the same length")
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.stream = stream or torch.cuda.current_stream(params.device)
+        self.cfg = A.Config(psi, self.world, stage, rank_view=self.rank, variant=variant, tensors=tensors,
+                            precision=precision, view_outputs=self.world)
+        L = A.zero_state_bytes(self.cfg)
+        P = L.partition_len
+        self.begin = min(self.rank * P, psi)
+        self.end = min(self.begin + P, psi)
+        if master_init.numel() != self.end - self.begin or master_init.dtype != torch.float32:
+            raise ValueError(f"master_init: {self.end - self.begin} fp32 elements of partition {self.rank}")
+        self.peers = PeerBuffers([(grad.data_ptr(), 2 * psi), (params.data_ptr(), 2 * psi)], group)
+        self.workspace = torch.empty(L.workspace_bytes, dtype=torch.uint8, device=params.device)
+        self.grad_ptrs = [row[0] + 2 * self.begin for row in self.peers.ptrs]
+        self.h = None
+        try:
+            self.h = A.zero_init(self.cfg, self.workspace.data_ptr(), L.workspace_bytes,
+                                 master_init.data_ptr(), [row[1] for row in self.peers.ptrs],
+                                 self.stream.cuda_stream)
+        finally:
+            # every rank's initial partition is in every parameter buffer (or
+            # every rank learns here that one of them failed: the barrier ends)
+            device_barrier(self.stream, group)
+        self._grads = grad
+        self._params = params
+
+    def step(self, loss_scale: float, hp: A.zero_hyper) -> bool:
+        device_barrier(self.stream, self.group)
+        skipped = rank_step(self.h, self.grad_ptrs, loss_scale, hp, self.stream, self.group)
+        device_barrier(self.stream, self.group)
+        return skipped
+
+    def state(self) -> tuple[int, int, int, int]:
+        """Device addresses of this rank's master, m, v and t."""
+        return A.zero_current_state(self.h)
+
+    def close(self) -> None:
+        self.stream.synchronize()
+        if self.h is not None:
+            A.zero_destroy(self.h)
+            self.h = None
+        self.peers.close(self.stream)
