@@ -78,46 +78,65 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _grads(psi, step, rank):
-    g = S.host_f16_bits(psi, 0, S.key(4, S.STREAM_GRAD, step, rank), S.normal(1e-3, SCALE))
-    return g
+CASES = {
+    # stage 2, fp16 gradients and parameters with fp32 master, every variant
+    "fp16": dict(stage=2, precision=A.ZERO_PRECISION_FP16, tensors=None, inf=0x7C00,
+                 variants=[A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA,
+                           A.ZERO_VARIANT_TWO_PASS_TMA]),
+    # stage 1, bfloat16 without master, a tensor excluded from weight decay
+    "bf16": dict(stage=1, precision=A.ZERO_PRECISION_BF16, inf=0x7F80,
+                 tensors=[(5000, 0), (10999, 0, A.ZERO_TENSOR_NO_DECAY)],
+                 variants=[A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_TWO_PASS_TMA]),
+}
 
 
-def _inject(g, step, rank, world):
+def _scale(case):
+    return 1.0 if case["precision"] == A.ZERO_PRECISION_BF16 else SCALE
+
+
+def _grads(case, psi, step, rank, world):
+    key = S.key(4, S.STREAM_GRAD, step, rank)
+    if case["precision"] == A.ZERO_PRECISION_BF16:
+        g = Z.bf16_from_f32(S.host_f32(psi, 0, key, S.normal(1e-3, 1.0)))
+    else:
+        g = S.host_f16_bits(psi, 0, key, S.normal(1e-3, SCALE))
     # step 1: an inf on the last rank, in partition 0 (owned by rank 0)
     if step == 1 and rank == world - 1:
-        g[0] = 0x7C00
+        g[0] = case["inf"]
     return g
 
 
-def _worker(rank, world, port, variants, psi, steps, q):
+def _worker(rank, world, port, name, psi, steps, q):
     from datetime import timedelta
 
     import torch.distributed as dist
     from zero_partitioned_mixed_02_b200.distributed import PeerRank
 
+    case = CASES[name]
+    bf16 = case["precision"] == A.ZERO_PRECISION_BF16
     torch.cuda.set_device(0)
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
                             timeout=timedelta(seconds=90))
     out = {}
     try:
         w0 = S.host_f32(psi, 0, S.key(4, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
-        for variant in variants:
+        for variant in case["variants"]:
             grad = torch.zeros(psi, dtype=torch.int16, device="cuda")
             params = torch.zeros(psi, dtype=torch.int16, device="cuda")
             P = -(-psi // world)
             b, e = min(rank * P, psi), min(rank * P + P, psi)
-            job = PeerRank(grad, params, torch.from_numpy(w0[b:e].copy()).cuda(), stage=2, variant=variant)
+            job = PeerRank(grad, params, torch.from_numpy(w0[b:e].copy()).cuda(), stage=case["stage"],
+                           variant=variant, precision=case["precision"], tensors=case["tensors"])
             assert (job.begin, job.end) == (b, e)
             res = []
             for step in range(steps):
-                g = _inject(_grads(psi, step, rank), step, rank, world)
-                grad.copy_(torch.from_numpy(g.view(np.int16)))
-                skipped = job.step(SCALE, hyper(**HP))
-                wp, _, _, t = job.state()
+                grad.copy_(torch.from_numpy(_grads(case, psi, step, rank, world).view(np.int16)))
+                skipped = job.step(_scale(case), hyper(**HP))
+                wp, mp, _, t = job.state()
+                src = mp if bf16 else wp  # no master in bfloat16: check the first moment
                 base = job.workspace.data_ptr()
-                w = job.workspace[wp - base: wp - base + 4 * (e - b)].view(torch.float32).cpu().numpy().copy()
-                res.append((skipped, t, params.cpu().numpy().view(np.uint16).copy(), w))
+                x = job.workspace[src - base: src - base + 4 * (e - b)].view(torch.float32).cpu().numpy().copy()
+                res.append((skipped, t, params.cpu().numpy().view(np.uint16).copy(), x))
             mapped = A.zero_peer_open_count()
             job.close()
             out[variant] = (b, e, res, mapped, A.zero_peer_open_count())
@@ -129,16 +148,15 @@ def _worker(rank, world, port, variants, psi, steps, q):
         q.put((rank, out))
 
 
-VARIANTS = [A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_TWO_PASS, A.ZERO_VARIANT_FUSED_TMA, A.ZERO_VARIANT_TWO_PASS_TMA]
-
-
-def test_two_ranks_through_ipc_mappings():
+@pytest.mark.parametrize("name", list(CASES))
+def test_two_ranks_through_ipc_mappings(name):
+    case = CASES[name]
     world, steps = 2, 3
     psi = 8000 * world - (world - 1)  # 16-byte aligned partitions, a ragged last one
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, VARIANTS, psi, steps, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, name, psi, steps, q)) for r in range(world)]
     for p in procs:
         p.start()
     got = {}
@@ -157,23 +175,29 @@ def test_two_ranks_through_ipc_mappings():
     assert [p.exitcode for p in procs] == [0] * world
 
     # the oracle: plain data-parallel mixed-precision Adam on the summed gradients
+    bf16 = case["precision"] == A.ZERO_PRECISION_BF16
+    tensors = case["tensors"]
+    mask = Z.decay_mask([x[0] for x in tensors], [len(x) > 2 for x in tensors]) if tensors else None
     w0 = S.host_f32(psi, 0, S.key(4, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
     w, m, v = w0.copy(), np.zeros(psi, np.float32), np.zeros(psi, np.float32)
-    p16 = Z.f16_from_f32(w)
+    p16 = Z.bf16_from_f32(w) if bf16 else Z.f16_from_f32(w)
     t = 0
     want = []
     for step in range(steps):
-        gs = [_inject(_grads(psi, step, k), step, k, world) for k in range(world)]
-        sk, t = Z.dp_step(gs, w, m, v, p16, SCALE, Z.hyper(**HP), t)
-        want.append((sk, t, p16.copy(), w.copy()))
+        gs = [_grads(case, psi, step, k, world) for k in range(world)]
+        if bf16:
+            sk, t = Z.bf16_step(gs, p16, m, v, _scale(case), Z.hyper(**HP), t, decay=mask)
+        else:
+            sk, t = Z.dp_step(gs, w, m, v, p16, _scale(case), Z.hyper(**HP), t, decay=mask)
+        want.append((sk, t, p16.copy(), (m if bf16 else w).copy()))
     assert [x[0] for x in want] == [False, True, False]
 
-    for variant in VARIANTS:
+    for variant in case["variants"]:
         for rank in range(world):
             b, e, res, mapped, after = got[rank][variant]
             assert mapped in (1, 2) and after == 0, (variant, rank, mapped, after)
-            for step, ((sk, tt, params, wpart), (wsk, wt, wp16, ww)) in enumerate(zip(res, want)):
-                what = f"variant {variant}, rank {rank}, step {step}"
+            for step, ((sk, tt, params, x), (wsk, wt, wp16, wx)) in enumerate(zip(res, want)):
+                what = f"{name}, variant {variant}, rank {rank}, step {step}"
                 assert sk == wsk and tt == wt, what
                 compare_f16(params, wp16, f"parameters of {what}")
-                compare_f32(wpart, ww[b:e], f"master of {what}")
+                compare_f32(x, wx[b:e], f"{'m' if bf16 else 'master'} of {what}")
