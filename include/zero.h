@@ -136,8 +136,13 @@ typedef struct zero_config {
     int64_t psi;       /* number of parameters of the flat vector */
     int32_t nd;        /* virtual data-parallel ranks, 1 .. ZERO_MAX_ND */
     int32_t stage;     /* ZeRO stage 1, 2 or 3 */
-    int32_t rank_view; /* -1: emulate all Nd ranks; r >= 0 (stage 1/2 only):
-                          act as rank r alone, owning partition r */
+    int32_t rank_view; /* -1: emulate all Nd ranks; r >= 0: act as rank r
+                          alone, owning partition r (stage 1/2) or shard r
+                          (stage 3: rank r of a real job; grads are the Nd
+                          ranks' full-length gradients, master_init the full
+                          flat master, the fp16 shard stays in the workspace
+                          at zero_ledger.off_shard16, and layer units are
+                          gathered with zero_gather_layer_ranks) */
     int32_t variant;   /* ZERO_VARIANT_FUSED, _TWO_PASS, _FUSED_TMA or _TWO_PASS_TMA */
     int32_t n_tensors; /* 0 allowed for stage 1/2 (one flat tensor) */
     int32_t precision; /* ZERO_PRECISION_FP16 (0) or ZERO_PRECISION_BF16 */
@@ -147,7 +152,8 @@ typedef struct zero_config {
                              written, 0 or 1 = one buffer, nd = every rank's
                              replica (rank r of a real Nd-rank job: param_bufs
                              are all ranks' replicas, e.g. peer-mapped; see
-                             zero_flag_words) */
+                             zero_flag_words); stage 3: 0 or 1, the
+                             output is the rank's own shard */
     int32_t reserved;     /* must be 0 */
 } zero_config;
 
@@ -255,7 +261,8 @@ int zero_step_commit(zero_handle* h, void* stream, int* skipped);
  * rank's reduced gradient overflows ([P1] "The part that sounds too good:
  * communication": the ranks reduce-scatter, update their slices, all-gather;
  * one overflow decision for the step). When each rank of a real Nd-rank job
- * runs its own single-rank-view handle (view_outputs = nd), the ranks agree by
+ * runs its own single-rank-view handle (view_outputs = nd on stage 1/2; any
+ * stage-3 rank view), the ranks agree by
  * reducing these two words with MAX across ranks on `stream` between
  * zero_step_launch and zero_step_commit (for instance ncclAllReduce with
  * ncclMax on ncclUint32, count 2); the words hold the handle's step call id on
@@ -314,6 +321,21 @@ int zero_async_end(zero_handle* h, void* stream, zero_async_state* out);
  * reverse for backward ([P1] "communication": parameters are gathered on demand
  * in the forward and backward passes, then discarded). ZERO_ERR_STAGE on 1/2. */
 int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream);
+
+/* Stage-3 layer gather of rank r of a real Nd-rank job (a handle with
+ * rank_view = r): the fp16 values of layer unit `unit` in flat order, copied
+ * from the Nd ranks' fp16 shards ([P1] "The part that sounds too good:
+ * communication": stage 3 all-gathers each layer's parameters when the
+ * forward or the backward pass needs them). shards[k]: device address of
+ * rank k's shard (the region at zero_ledger.off_shard16 of rank k's
+ * workspace, shard_len(k) elements; peer-mapped for k != r, see zero_peer.h;
+ * may be NULL for an empty shard); out: device buffer of the unit's numel
+ * elements (zero_unit_range). Every rank's step must have finished before the
+ * gather reads its shard (the caller's barrier). Returns ZERO_ERR_STAGE on
+ * stage 1/2, ZERO_ERR_ARG for a handle that emulates all ranks (use
+ * zero_gather_layer) or a bad unit, ZERO_ERR_ALIGN for unaligned buffers. */
+int zero_gather_layer_ranks(zero_handle* h, int32_t unit, const uint16_t* const* shards, uint16_t* out,
+                            void* stream);
 
 /* Current state: device pointers to the live master/m/v arrays (the fused
  * variant alternates between two buffers) and the step count t. Any output

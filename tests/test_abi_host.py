@@ -136,8 +136,8 @@ def test_workspace_layout():
 @pytest.mark.parametrize("kw", [
     dict(psi=0, nd=1, stage=1), dict(psi=10, nd=0, stage=1), dict(psi=10, nd=2, stage=4),
     dict(psi=10, nd=2, stage=3),  # stage 3 needs a tensor list
-    dict(psi=10, nd=2, stage=2, rank_view=2), dict(psi=10, nd=2, stage=3, rank_view=0,
-                                                   tensors=[(10, 0)]),
+    dict(psi=10, nd=2, stage=2, rank_view=2), dict(psi=10, nd=2, stage=3, rank_view=0, view_outputs=2,
+                                                   tensors=[(10, 0)]),  # a stage-3 rank has one output
     dict(psi=10, nd=2, stage=2, variant=7), dict(psi=10, nd=2, stage=2, tensors=[(4, 0), (5, 0)]),
     dict(psi=10, nd=2, stage=3, tensors=[(4, 1), (6, 1)]),  # units must start at 0
     dict(psi=10, nd=2, stage=3, tensors=[(4, 0), (6, 2)]),  # units must be contiguous

@@ -201,3 +201,119 @@ def test_two_ranks_through_ipc_mappings(name):
                 assert sk == wsk and tt == wt, what
                 compare_f16(params, wp16, f"parameters of {what}")
                 compare_f32(x, wx[b:e], f"{'m' if bf16 else 'master'} of {what}")
+
+
+# stage 3: each rank keeps its shard in its workspace; after every step each
+# rank gathers every layer unit from both ranks' shards through the mappings
+TENSORS3 = [(8192, 0), (4096, 0), (40001, 1), (2048, 1), (777, 2), (5000, 3)]
+
+
+def _shards(x, numel, nd, r):
+    out, off = [], 0
+    for n in numel:
+        b, e = Z.chunk(n, nd, r)
+        out.append(x[off + b: off + e])
+        off += n
+    return np.concatenate(out)
+
+
+def _worker3(rank, world, port, variants, steps, q):
+    from datetime import timedelta
+
+    import torch.distributed as dist
+    from zero_partitioned_mixed_02_b200.distributed import PeerRank
+
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=90))
+    out = {}
+    try:
+        psi = sum(t[0] for t in TENSORS3)
+        n_units = TENSORS3[-1][1] + 1
+        w0 = S.host_f32(psi, 0, S.key(6, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
+        for variant in variants:
+            grad = torch.zeros(psi, dtype=torch.int16, device="cuda")
+            job = PeerRank(grad, None, torch.from_numpy(w0.copy()).cuda(), stage=3, variant=variant,
+                           tensors=TENSORS3)
+            n = A.zero_state_bytes(job.cfg).state_elems
+            res = []
+            for step in range(steps):
+                g = S.host_f16_bits(psi, 0, S.key(6, S.STREAM_GRAD, step, rank), S.normal(1e-3, SCALE))
+                if step == 1 and rank == 0:
+                    g[psi - 1] = 0xFC00  # -inf on rank 0, in the last tensor's last chunk (rank 1's)
+                grad.copy_(torch.from_numpy(g.view(np.int16)))
+                skipped = job.step(SCALE, hyper(**HP))
+                wp, _, _, t = job.state()
+                base = job.workspace.data_ptr()
+                w = job.workspace[wp - base: wp - base + 4 * n].view(torch.float32).cpu().numpy().copy()
+                units = []
+                for u in range(n_units):
+                    buf = torch.empty(job.unit_range(u)[1], dtype=torch.int16, device="cuda")
+                    job.gather(u, buf)
+                    units.append(buf.cpu().numpy().view(np.uint16).copy())
+                res.append((skipped, t, w, units))
+            mapped = A.zero_peer_open_count()
+            job.close()
+            out[variant] = (res, mapped, A.zero_peer_open_count())
+            del job, grad
+    except Exception as exc:  # reported to the parent, which fails the test
+        out = {"error": repr(exc)}
+    finally:
+        dist.destroy_process_group()
+        q.put((rank, out))
+
+
+def test_stage3_ranks_through_ipc_mappings():
+    world, steps = 2, 3
+    variants = CASES["fp16"]["variants"]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker3, args=(r, world, port, variants, steps, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    try:
+        for _ in range(world):
+            rank, out = q.get(timeout=300)
+            got[rank] = out
+    finally:
+        for p in procs:
+            p.join(120)
+        for p in procs:  # only the processes started here, if they outlived the wait
+            if p.is_alive():
+                p.kill()
+                p.join(30)
+    assert all("error" not in out for out in got.values()), got
+    assert [p.exitcode for p in procs] == [0] * world
+
+    numel = [t[0] for t in TENSORS3]
+    unit_of = [t[1] for t in TENSORS3]
+    psi = sum(numel)
+    w0 = S.host_f32(psi, 0, S.key(6, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
+    w_sh = [_shards(w0, numel, world, r).copy() for r in range(world)]
+    m_sh = [np.zeros_like(x) for x in w_sh]
+    v_sh = [np.zeros_like(x) for x in w_sh]
+    p_sh = [Z.f16_from_f32(x) for x in w_sh]
+    t = 0
+    want = []
+    for step in range(steps):
+        gs = [S.host_f16_bits(psi, 0, S.key(6, S.STREAM_GRAD, step, k), S.normal(1e-3, SCALE))
+              for k in range(world)]
+        if step == 1:
+            gs[0][psi - 1] = 0xFC00
+        sk, t = Z.zero3_step(numel, gs, w_sh, m_sh, v_sh, p_sh, SCALE, Z.hyper(**HP), t)
+        units = [Z.zero3_gather(numel, unit_of, world, u, p_sh) for u in range(unit_of[-1] + 1)]
+        want.append((sk, t, [x.copy() for x in w_sh], units))
+    assert [x[0] for x in want] == [False, True, False]
+
+    for variant in variants:
+        for rank in range(world):
+            res, mapped, after = got[rank][variant]
+            assert mapped in (1, 2) and after == 0, (variant, rank, mapped, after)
+            for step, ((sk, tt, w, units), (wsk, wt, ww, wunits)) in enumerate(zip(res, want)):
+                what = f"stage 3, variant {variant}, rank {rank}, step {step}"
+                assert sk == wsk and tt == wt, what
+                compare_f32(w, ww[rank], f"master shard of {what}")
+                for u, (x, y) in enumerate(zip(units, wunits)):
+                    compare_f16(x, y, f"unit {u} of {what}")

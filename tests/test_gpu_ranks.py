@@ -147,3 +147,124 @@ def test_rank_handles_refuse_asynchronous_steps():
         A.zero_async_begin(h, [g.data_ptr() for g in G], A.zero_scaler(1.0, 2.0, 0.5, 10), 0.9, 0.999, s)
     assert ei.value.code == A.ZERO_ERR_ARG
     A.zero_destroy(h)
+
+
+# stage 3: rank r of a real job keeps shard r; layer units are gathered from
+# the Nd ranks' shards (zero_gather_layer_ranks). Tensor lists: chunks in
+# 16-byte phase with runs of several gather tiles, and chunks out of phase
+# with a ragged tail.
+SHAPES3 = {
+    "aligned": [(8192, 0), (4096, 0), (65536, 1), (64, 1), (16384, 2)],
+    "ragged": [(4000, 0), (1601, 0), (40001, 1), (2048, 1), (777, 2), (5000, 3)],
+}
+
+
+def _shards(x, numel, nd, r):
+    """Rank r's chunks of every tensor, concatenated (the oracle's shard)."""
+    out, off = [], 0
+    for n in numel:
+        b, e = Z.chunk(n, nd, r)
+        out.append(x[off + b: off + e])
+        off += n
+    return np.concatenate(out) if out else x[:0]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("nd", [2, 4])
+@pytest.mark.parametrize("shape", list(SHAPES3))
+def test_stage3_ranks_as_handles(shape, nd, variant):
+    tensors = SHAPES3[shape]
+    numel = [t[0] for t in tensors]
+    unit_of = [t[1] for t in tensors]
+    n_units = unit_of[-1] + 1
+    psi = sum(numel)
+    s = torch.cuda.current_stream()
+    w0 = S.host_f32(psi, 0, S.key(5, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
+    m_init = torch.from_numpy(w0.copy()).cuda()
+    G = [torch.empty(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
+    handles, wss, Ls = [], [], []
+    for r in range(nd):
+        cfg = A.Config(psi, nd, 3, rank_view=r, variant=variant, tensors=tensors)
+        L = A.zero_state_bytes(cfg)
+        assert L.state_elems == Z.shard_len(numel, nd, r) and L.grad_len == psi
+        ws = torch.empty(L.workspace_bytes, dtype=torch.uint8, device="cuda")
+        handles.append(A.zero_init(cfg, ws.data_ptr(), L.workspace_bytes, m_init.data_ptr(), None, s.cuda_stream))
+        wss.append(ws)
+        Ls.append(L)
+    shard_ptrs = [wss[k].data_ptr() + Ls[k].off_shard16 for k in range(nd)]
+    w_sh = [_shards(w0, numel, nd, r).copy() for r in range(nd)]
+    m_sh = [np.zeros_like(x) for x in w_sh]
+    v_sh = [np.zeros_like(x) for x in w_sh]
+    p_sh = [Z.f16_from_f32(x) for x in w_sh]
+    hp = dict(lr=1e-2, weight_decay=0.05)
+    t = 0
+    skips = []
+    for step in range(3):
+        gs = [S.host_f16_bits(psi, 0, S.key(5, S.STREAM_GRAD, step, k), S.normal(1e-3, 1024.0))
+              for k in range(nd)]
+        if step == 1:
+            gs[nd - 1][psi - 1] = 0x7E00  # a NaN on the last rank, in the last rank's last chunk
+        for k in range(nd):
+            G[k].copy_(torch.from_numpy(gs[k].view(np.int16)))
+        for h in handles:
+            A.zero_step_launch(h, [g.data_ptr() for g in G], 1024.0, hyper(**hp), s.cuda_stream)
+        words = [flag_words(h) for h in handles]
+        agreed = torch.stack(words).max(dim=0).values
+        for x in words:
+            x.copy_(agreed)
+        rcs = [A.zero_step_commit(h, s.cuda_stream) for h in handles]
+        assert len(set(rcs)) == 1
+        sk, t = Z.zero3_step(numel, gs, w_sh, m_sh, v_sh, p_sh, 1024.0, Z.hyper(**hp), t)
+        assert (rcs[0] == A.ZERO_SKIPPED) == sk
+        skips.append(sk)
+        for r, h in enumerate(handles):
+            wp, mp, _, tt = A.zero_current_state(h)
+            assert tt == t
+            n = Ls[r].state_elems
+            base = wss[r].data_ptr()
+            compare_f32(wss[r][wp - base: wp - base + 4 * n].view(torch.float32).cpu().numpy(), w_sh[r],
+                        f"rank {r} master shard, step {step}")
+            compare_f32(wss[r][mp - base: mp - base + 4 * n].view(torch.float32).cpu().numpy(), m_sh[r],
+                        f"rank {r} m shard, step {step}")
+            o = Ls[r].off_shard16
+            compare_f16(wss[r][o: o + 2 * n].view(torch.int16).cpu().numpy().view(np.uint16), p_sh[r],
+                        f"rank {r} fp16 shard, step {step}")
+        for u in range(n_units):
+            want = Z.zero3_gather(numel, unit_of, nd, u, p_sh)
+            out = GuardedF16(len(want))
+            A.zero_gather_layer_ranks(handles[u % nd], u, shard_ptrs, out.ptr(), s.cuda_stream)
+            compare_f16(out.bits(), want, f"unit {u} gathered by rank {u % nd}, step {step}")
+            assert out.guards_intact()
+        torch.cuda.synchronize()
+    assert skips == [False, True, False]
+    # the errors a rank's gather reports (before any launch)
+    spare = GuardedF16(max(numel))
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_gather_layer(handles[0], 0, spare.ptr(), s.cuda_stream)
+    assert ei.value.code == A.ZERO_ERR_ARG
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_gather_layer_ranks(handles[0], n_units, shard_ptrs, spare.ptr(), s.cuda_stream)
+    assert ei.value.code == A.ZERO_ERR_ARG
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_gather_layer_ranks(handles[0], 0, [p + 2 for p in shard_ptrs], spare.ptr(), s.cuda_stream)
+    assert ei.value.code == A.ZERO_ERR_ALIGN
+    torch.cuda.synchronize()
+    assert spare.guards_intact()
+    for h in handles:
+        A.zero_destroy(h)
+
+
+def test_stage3_rank_refuses_asynchronous_steps():
+    tensors = SHAPES3["aligned"]
+    psi = sum(t[0] for t in tensors)
+    cfg = A.Config(psi, 2, 3, rank_view=1, tensors=tensors)
+    L = A.zero_state_bytes(cfg)
+    ws = torch.empty(L.workspace_bytes, dtype=torch.uint8, device="cuda")
+    m0 = torch.zeros(psi, dtype=torch.float32, device="cuda")
+    G = [torch.zeros(psi, dtype=torch.int16, device="cuda") for _ in range(2)]
+    s = torch.cuda.current_stream().cuda_stream
+    h = A.zero_init(cfg, ws.data_ptr(), L.workspace_bytes, m0.data_ptr(), None, s)
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_async_begin(h, [g.data_ptr() for g in G], A.zero_scaler(1.0, 2.0, 0.5, 10), 0.9, 0.999, s)
+    assert ei.value.code == A.ZERO_ERR_ARG
+    A.zero_destroy(h)

@@ -74,3 +74,35 @@ def test_layout_invariants(c):
         o = A.zero_offload_bytes(cfg, 256)
         assert o.state_elems == psi and o.host_state_bytes == 12 * psi
         assert o.n_chunks == -(-psi // o.chunk_elems)
+
+
+@settings(max_examples=200, deadline=None)
+@given(configs(), st.integers(0, 39))
+def test_stage3_rank_view(c, r):
+    """Rank r of a real stage-3 job: its state is shard r (the oracle's shard
+    length), gradients stay full length, the ledger is the job's, and the
+    workspace holds the shard plus the gather tables; an offloaded stage-3
+    rank and a stage-3 rank with Nd outputs are refused."""
+    nd, tensors, _, variant, bf16 = c
+    r = r % nd
+    psi = sum(t[0] for t in tensors)
+    prec = A.ZERO_PRECISION_BF16 if bf16 else A.ZERO_PRECISION_FP16
+    job = A.zero_state_bytes(A.Config(psi, nd, 3, variant=variant, tensors=tensors, precision=prec))
+    cfg = A.Config(psi, nd, 3, rank_view=r, variant=variant, tensors=tensors, precision=prec)
+    L = A.zero_state_bytes(cfg)
+    assert L.state_elems == Z.shard_len([t[0] for t in tensors], nd, r) == A.zero_rank_shard(cfg, r)[1]
+    assert L.grad_len == psi
+    assert list(L.exact_bytes) == list(job.exact_bytes) and L.transient_bytes == job.transient_bytes
+    assert L.off_shard16 > 0 and L.off_shard16 + 2 * L.state_elems <= L.workspace_bytes
+    if nd > 1:
+        try:
+            A.zero_state_bytes(A.Config(psi, nd, 3, rank_view=r, variant=variant, tensors=tensors,
+                                        precision=prec, view_outputs=nd))
+            raise AssertionError("a stage-3 rank with Nd outputs was accepted")
+        except A.ZeroError as e:
+            assert e.code == A.ZERO_ERR_ARG
+    try:
+        A.zero_offload_bytes(A.Config(psi, nd, 3, rank_view=r, tensors=tensors))
+        raise AssertionError("an offloaded stage-3 rank was accepted")
+    except A.ZeroError as e:
+        assert e.code == A.ZERO_ERR_ARG

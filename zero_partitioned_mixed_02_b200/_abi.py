@@ -129,6 +129,7 @@ def lib():
             "zero_step_launch": (C.c_int, [P, C.POINTER(P), C.c_float, C.POINTER(zero_hyper), P]),
             "zero_step_commit": (C.c_int, [P, P, C.POINTER(C.c_int)]),
             "zero_gather_layer": (C.c_int, [P, C.c_int32, P, P]),
+            "zero_gather_layer_ranks": (C.c_int, [P, C.c_int32, C.POINTER(P), P, P]),
             "zero_async_begin": (C.c_int, [P, C.POINTER(P), C.POINTER(zero_scaler), C.c_float,
                                            C.c_float, P]),
             "zero_step_async": (C.c_int, [P, C.POINTER(zero_hyper), P]),
@@ -278,6 +279,12 @@ def zero_async_end(h: int, stream: int) -> zero_async_state:
 
 def zero_gather_layer(h: int, unit: int, out: int, stream: int) -> None:
     _check(lib().zero_gather_layer(h, unit, out, stream), "zero_gather_layer", h)
+
+
+def zero_gather_layer_ranks(h: int, unit: int, shards: Sequence[int], out: int, stream: int) -> None:
+    """Stage-3 rank of a real job: gather a layer unit from the Nd ranks'
+    fp16 shards (shards[k]: rank k's shard, peer-mapped for other ranks)."""
+    _check(lib().zero_gather_layer_ranks(h, unit, _ptr_array(shards), out, stream), "zero_gather_layer_ranks", h)
 
 
 def zero_current_state(h: int) -> tuple[int, int, int, int]:

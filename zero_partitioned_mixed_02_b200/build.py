@@ -38,11 +38,12 @@ COMMON = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-fmad=false", "-f
 ZERO_SOURCES = [os.path.join(CSRC, "zero_abi.cu"), os.path.join(CSRC, "zero_kernels.cu"),
                 os.path.join(CSRC, "zero_static.cu"), os.path.join(CSRC, "zero_tma.cu"),
                 os.path.join(CSRC, "zero_offload.cu"), os.path.join(CSRC, "zero_tma_pass.cu"),
-                os.path.join(CSRC, "zero_peer.cu")]
+                os.path.join(CSRC, "zero_peer.cu"), os.path.join(CSRC, "zero_gather_ranks.cu")]
 HOST_ADAM = os.path.join(CSRC, "zero_host_adam.cpp")
 ZERO_DEPS = ZERO_SOURCES + [HOST_ADAM, os.path.join(CSRC, "zero_host_adam.h"),
                             os.path.join(CSRC, "zero_internal.h"), os.path.join(CSRC, "zero_device.cuh"),
                             os.path.join(CSRC, "zero_layout.h"), os.path.join(CSRC, "zero_tma.cuh"),
+                            os.path.join(CSRC, "zero_gather_ranks.h"),
                             os.path.join(INCLUDE, "zero.h"),
                             os.path.join(INCLUDE, "zero_offload.h"), os.path.join(INCLUDE, "zero_peer.h")]
 # the host update is built twice: AVX2 + F16C, and the baseline instruction set

@@ -73,7 +73,8 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
     // without a master nothing can be rolled back: the two-pass step only
     if (cfg->precision == ZERO_PRECISION_BF16 && is_fused(cfg->variant)) return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
-    if (cfg->rank_view >= 0 && cfg->stage == 3) return ZERO_ERR_ARG;
+    // a stage-3 rank writes only its own fp16 shard
+    if (cfg->rank_view >= 0 && cfg->stage == 3 && cfg->view_outputs > 1) return ZERO_ERR_ARG;
     if (cfg->reserved != 0) return ZERO_ERR_ARG;
     if (cfg->rank_view < 0 ? cfg->view_outputs != 0
                            : (cfg->view_outputs != 0 && cfg->view_outputs != 1 && cfg->view_outputs != cfg->nd))
@@ -161,7 +162,10 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
         }
     } else {
         // stage 3: every tensor split per rank; rank r's shard is its chunks
-        // in tensor order, shards back to back in rank order
+        // in tensor order, shards back to back in rank order. The single-rank
+        // view (rank r of a real job) keeps rank r's runs only, its state and
+        // shard indexed from 0; gradients stay full-length (flat index).
+        const int view = cfg->rank_view;
         int64_t pos = 0;
         for (int r = 0; r < nd; ++r) {
             L->shard_begin[r] = pos;
@@ -169,14 +173,17 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             for (size_t t = 0; t < L->numel.size(); ++t) {
                 int64_t b, e;
                 split(L->numel[t], nd, r, &b, &e);
-                add_run(L->step_segs, &L->step_chunks, off + b, pos + q, pos + q, e - b, L->decay_of[t]);
+                if (view < 0)
+                    add_run(L->step_segs, &L->step_chunks, off + b, pos + q, pos + q, e - b, L->decay_of[t]);
+                else if (r == view)
+                    add_run(L->step_segs, &L->step_chunks, off + b, q, q, e - b, L->decay_of[t]);
                 q += e - b;
                 off += L->numel[t];
             }
             L->shard_len[r] = q;
             pos += q;
         }
-        L->state_elems = cfg->psi;
+        L->state_elems = view < 0 ? cfg->psi : L->shard_len[view];
         L->grad_len = cfg->psi;
         L->n_out = 1;  // the fp16 shard array
 
@@ -201,20 +208,33 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             U.seg0 = (int64_t)L->gather_segs.size();
             U.flat_begin = tensor_off[t];
             int64_t chunks = 0;
+            U.rank_run0 = (int64_t)L->rank_gather.size();
             while (t < L->numel.size() && L->unit_of[t] == u) {
                 for (int r = 0; r < nd; ++r) {
                     int64_t b, e;
                     split(L->numel[t], nd, r, &b, &e);
-                    add_run(L->gather_segs, &chunks, chunk_pos[t * nd + r],
-                            0, tensor_off[t] - U.flat_begin + b, e - b);
+                    if (view < 0) {
+                        add_run(L->gather_segs, &chunks, chunk_pos[t * nd + r],
+                                0, tensor_off[t] - U.flat_begin + b, e - b);
+                    } else if (e > b) {
+                        zg::Run g{};
+                        g.src_begin = chunk_pos[t * nd + r] - L->shard_begin[r];
+                        g.out_begin = tensor_off[t] - U.flat_begin + b;
+                        g.len = e - b;
+                        g.tile_begin = U.rank_tiles;
+                        g.rank = r;
+                        U.rank_tiles += zg::tiles_of(e - b);
+                        L->rank_gather.push_back(g);
+                    }
                 }
                 U.numel += L->numel[t];
                 ++t;
             }
             U.n_segs = (int64_t)L->gather_segs.size() - U.seg0;
             U.n_chunks = chunks;
+            U.rank_n_runs = (int64_t)L->rank_gather.size() - U.rank_run0;
             L->transient_elems = std::max(L->transient_elems, U.numel);
-            if (is_tma(cfg->variant)) {
+            if (is_tma(cfg->variant) && view < 0) {
                 bool ok = U.n_segs > 0;
                 for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
                     const zk::SegDesc& g = L->gather_segs[i];
@@ -311,6 +331,13 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
         L->off_tma_gather = off;
         off += align_up((int64_t)L->tma_gather.size() * sizeof(zk::TmaRun));
     }
+    if (cfg->stage == 3 && cfg->rank_view >= 0) {
+        // the Nd shard addresses, then the Nd shard lengths
+        L->off_shard_tab = off;
+        off += align_up((int64_t)nd * 16);
+        L->off_rank_gather = off;
+        off += align_up((int64_t)std::max<size_t>(L->rank_gather.size(), 1) * sizeof(zg::Run));
+    }
     const int n_buf = is_fused(cfg->variant) ? 2 : 1;
     for (int b = 0; b < n_buf; ++b)
         for (int k = 0; k < 3; ++k) {
@@ -404,6 +431,13 @@ struct zero_handle {
     int occ_tma_r = 0;
     zk::TmaRun* d_tma_gather = nullptr;
     int occ_gather_tma = 0;
+    // stage-3 rank view: the gather from the Nd ranks' shards
+    const uint16_t** d_shard_tab = nullptr;
+    int64_t* d_shard_len = nullptr;
+    zg::Run* d_rank_gather = nullptr;
+    int occ_gather_ranks = 0;
+    std::vector<const uint16_t*> shard_tab;  // host copy of what d_shard_tab holds
+    bool shard_tab_valid = false;
     int64_t hold_tile = -1;  // test hook for the bounded waits (zero_test_hold_tile)
     unsigned hold_rounds = 0;
     bool async = false;      // between zero_async_begin and zero_async_end
@@ -453,7 +487,12 @@ cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_
 // zero_step_commit. A two-pass step updates in place, so its update pass must
 // wait for that agreement: zero_step_launch enqueues the reduce pass only and
 // zero_step_commit the update pass.
-bool defers_update(const Layout& L) { return L.view >= 0 && L.n_out > 1 && !is_fused(L.variant); }
+// a rank of a real job: its outputs are the other ranks' replicas (stage 1/2)
+// or its shard of a sharded job (stage 3); it agrees with the other ranks on
+// overflow between launch and commit
+bool real_rank(const Layout& L) { return L.view >= 0 && (L.n_out > 1 || L.stage == 3); }
+
+bool defers_update(const Layout& L) { return real_rank(L) && !is_fused(L.variant); }
 
 int cuda_fail(zero_handle* h, cudaError_t e)
 {
@@ -672,6 +711,17 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
             return rc;
         }
     }
+    if (L.off_shard_tab >= 0) {
+        h->d_shard_tab = reinterpret_cast<const uint16_t**>(h->ws + L.off_shard_tab);
+        h->d_shard_len = reinterpret_cast<int64_t*>(h->ws + L.off_shard_tab + 8 * (int64_t)L.nd);
+        h->d_rank_gather = reinterpret_cast<zg::Run*>(h->ws + L.off_rank_gather);
+        e = zg::occupancy(&h->occ_gather_ranks);
+        if (e != cudaSuccess) {
+            rc = cuda_fail(h, e);
+            delete h;
+            return rc;
+        }
+    }
     if (L.stage <= 2)
         h->out_tab.assign(param_bufs, param_bufs + L.n_out);
     else
@@ -696,6 +746,11 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     if (e == cudaSuccess && !L.gather_segs.empty())
         e = cudaMemcpyAsync(h->d_gather_segs, L.gather_segs.data(),
                             L.gather_segs.size() * sizeof(zk::SegDesc), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && h->d_shard_len)
+        e = cudaMemcpyAsync(h->d_shard_len, L.shard_len.data(), L.nd * sizeof(int64_t), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !L.rank_gather.empty())
+        e = cudaMemcpyAsync(h->d_rank_gather, L.rank_gather.data(), L.rank_gather.size() * sizeof(zg::Run),
+                            cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && L.step_chunks > 0) {
         zk::StepArgs a{};
         a.segs = h->d_step_segs;
@@ -869,7 +924,7 @@ ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, cons
 {
     if (!h || !grads || !sc || h->pending || h->async) return ZERO_ERR_ARG;
     // a rank of a real job agrees with the other ranks through launch/commit
-    if (h->L.view >= 0 && h->L.n_out > 1) return ZERO_ERR_ARG;
+    if (real_rank(h->L)) return ZERO_ERR_ARG;
     if (!(sc->init_scale > 0.0f) || !std::isfinite(sc->init_scale) || !(sc->growth_factor >= 1.0f) ||
         !std::isfinite(sc->growth_factor) || !(sc->backoff_factor > 0.0f) || !(sc->backoff_factor <= 1.0f) ||
         sc->growth_interval < 1 || !std::isfinite(beta1) || !std::isfinite(beta2))
@@ -1004,6 +1059,7 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     if (!h || h->pending) return ZERO_ERR_ARG;
     const Layout& L = h->L;
     if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (L.view >= 0) return ZERO_ERR_ARG;  // a rank's handle gathers with zero_gather_layer_ranks
     if (unit < 0 || unit >= L.n_units || !out) return ZERO_ERR_ARG;
     if (!aligned16(out)) return ZERO_ERR_ALIGN;
     const Unit& U = L.units[unit];
@@ -1038,6 +1094,45 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     g.dst_len = U.numel;
     const cudaError_t e = zk::launch_gather(g, grid_for(h, zk::K_GATHER, U.n_chunks),
                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+}
+
+ZERO_API int zero_gather_layer_ranks(zero_handle* h, int32_t unit, const uint16_t* const* shards, uint16_t* out,
+                                    void* stream)
+{
+    const zk::NvtxRange nvtx_range("zero_gather_layer_ranks");
+    if (!h || h->pending) return ZERO_ERR_ARG;
+    const Layout& L = h->L;
+    if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (L.view < 0 || !h->d_shard_tab) return ZERO_ERR_ARG;  // emulated ranks: zero_gather_layer
+    if (unit < 0 || unit >= L.n_units || !out || !shards) return ZERO_ERR_ARG;
+    if (!aligned16(out)) return ZERO_ERR_ALIGN;
+    for (int k = 0; k < L.nd; ++k) {
+        if (!shards[k] && L.shard_len[k] > 0) return ZERO_ERR_ARG;
+        if (!aligned16(shards[k])) return ZERO_ERR_ALIGN;
+    }
+    const Unit& U = L.units[unit];
+    if (U.rank_tiles == 0) return ZERO_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!h->shard_tab_valid || !std::equal(shards, shards + L.nd, h->shard_tab.begin())) {
+        h->shard_tab.assign(shards, shards + L.nd);
+        const cudaError_t e = cudaMemcpyAsync(h->d_shard_tab, h->shard_tab.data(), L.nd * sizeof(uint16_t*),
+                                              cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+        h->shard_tab_valid = true;
+    }
+    zg::Args g{};
+    g.runs = h->d_rank_gather + U.rank_run0;
+    g.n_runs = (int)U.rank_n_runs;
+    g.nd = L.nd;
+    g.n_tiles = U.rank_tiles;
+    g.shards = h->d_shard_tab;
+    g.shard_len = h->d_shard_len;
+    g.dst = out;
+    g.dst_len = U.numel;
+    g.err = h->d_flag + 1;
+    const int64_t cap = (int64_t)h->sms * std::max(h->occ_gather_ranks, 1);
+    const cudaError_t e = zg::launch(g, (int)std::min(U.rank_tiles, cap), s);
     return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
 }
 

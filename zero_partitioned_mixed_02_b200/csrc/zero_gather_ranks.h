@@ -1,0 +1,48 @@
+// Layer gather of rank r of a real stage-3 job ([P1] "The part that sounds too
+// good: communication": stage 3 all-gathers each layer's parameters on demand,
+// forward and backward; [P2] "ZeRO and the Memory Tricks" -- "The
+// Breakthrough"): the fp16 chunks of one layer unit are copied from the Nd
+// ranks' shards (this rank's own and the others', peer-mapped) into one
+// contiguous buffer in tensor order. Internal to libzero.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace zg {
+
+// One rank's chunk of one tensor of a unit. Runs are listed in the unit's
+// output order; tiles of kTile elements are numbered across the unit's runs.
+struct Run {
+    int64_t src_begin;   // element offset in the source rank's shard
+    int64_t out_begin;   // element offset in the gathered unit
+    int64_t len;         // elements, > 0
+    int64_t tile_begin;  // the run's first tile
+    int32_t rank;        // source rank
+    int32_t pad[3];
+};
+static_assert(sizeof(Run) == 48, "run layout");
+
+constexpr int64_t kTile = 8192;  // elements per tile (16 KB of fp16)
+constexpr int kThreads = 256;
+
+struct Args {
+    const Run* runs;
+    int n_runs;
+    int nd;
+    int64_t n_tiles;
+    const uint16_t* const* shards;  // device table: Nd shard addresses
+    const int64_t* shard_len;       // device table: Nd shard lengths (elements)
+    uint16_t* dst;
+    int64_t dst_len;
+    unsigned* err;                  // kernel-error word (bounds-checked build)
+};
+
+// Tiles of `n` elements of a run: ceil(n / kTile).
+inline int64_t tiles_of(int64_t n) { return (n + kTile - 1) / kTile; }
+
+cudaError_t occupancy(int* blocks_per_sm);
+cudaError_t launch(const Args& a, int grid, cudaStream_t s);
+
+}  // namespace zg

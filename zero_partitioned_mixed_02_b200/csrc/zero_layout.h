@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "zero.h"
+#include "zero_gather_ranks.h"
 #include "zero_internal.h"
 
 namespace zl {
@@ -32,6 +33,10 @@ struct Unit {
     int64_t tma_n_runs = 0;
     int64_t tma_tiles = 0;
     int64_t tma_scal = 0;
+    // stage-3 rank view: the unit's runs from the Nd ranks' shards
+    int64_t rank_run0 = 0;
+    int64_t rank_n_runs = 0;
+    int64_t rank_tiles = 0;
 };
 
 // Everything that follows from a configuration: partitions, run tables,
@@ -51,6 +56,7 @@ struct Layout {
     std::vector<zk::SegDesc> gather_segs;
     std::vector<zk::TmaRun> tma_gather;  // TMA variant: bulk-copy gather runs of all units
     std::vector<Unit> units;
+    std::vector<zg::Run> rank_gather;  // stage-3 rank view: gather runs of all units
     std::vector<zk::TmaRun> tma_runs;  // TMA variants, when every run is eligible
     bool tma_ok = false;
     zk::TmaShape tma_shape = zk::kTmaDeep;
@@ -61,7 +67,7 @@ struct Layout {
     int64_t tma_tiles_r = 0, tma_scal_r = 0;
     int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
             off_gather_segs = 0, off_tma_runs = -1, off_tma_runs_r = -1, off_tma_gather = -1, off_reduced = -1,
-            off_shard16 = -1,
+            off_shard16 = -1, off_shard_tab = -1, off_rank_gather = -1,
             total = 0;
     int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};
     int64_t transient_elems = 0;

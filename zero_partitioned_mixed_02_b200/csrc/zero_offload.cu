@@ -165,6 +165,7 @@ struct OffLayout {
 int off_layout(const zl::Layout& L, int64_t chunk_elems, OffLayout* O)
 {
     if (L.bf16) return ZERO_ERR_ARG;  // the offloaded step keeps an fp32 master
+    if (L.stage == 3 && L.view >= 0) return ZERO_ERR_ARG;  // no offloaded stage-3 rank of a real job
     O->E = L.state_elems;
     if (chunk_elems == 0) {
         // at most ZERO_OFFLOAD_DEFAULT_CHUNK, and at least 8 chunks for

@@ -144,51 +144,77 @@ class PeerBuffers:
 
 
 class PeerRank:
-    """Rank r of a real Nd-rank stage 1/2 job, one process per GPU (Nd = the
-    group's size). `grad` and `params` are this rank's full-length 16-bit
+    """Rank r of a real Nd-rank job, one process per GPU (Nd = the group's
+    size), on peer buffers.
+
+    Stages 1 and 2: `grad` and `params` are this rank's full-length 16-bit
     gradient and parameter buffers (torch tensors of psi elements); the handle
     reads partition r of every rank's gradient and writes partition r of the
-    new parameters into every rank's `params` through peer mappings.
+    new parameters into every rank's `params`; master_init holds partition r
+    of the initial master weights.
+
+    Stage 3: no parameter buffer (params=None): the handle reads chunk r of
+    every tensor from every rank's gradient and keeps shard r of the fp16
+    parameters in its workspace; gather(unit, out) assembles a layer unit from
+    the Nd ranks' shards; master_init is the full flat master (every rank
+    starts from the same weights) and `tensors` is required.
 
     step(): a device barrier (every rank's gradient is written), the step
     launch, the overflow agreement, the commit, and a second device barrier
-    (every rank's partition is in every parameter buffer)."""
+    (every rank's new parameters, or shard, are complete)."""
 
-    def __init__(self, grad: torch.Tensor, params: torch.Tensor, master_init: torch.Tensor,
+    def __init__(self, grad: torch.Tensor, params: torch.Tensor | None, master_init: torch.Tensor,
                  stage: int = 2, variant: int = A.ZERO_VARIANT_FUSED_TMA,
                  precision: int = A.ZERO_PRECISION_FP16, tensors=None, group=None,
                  stream: torch.cuda.Stream | None = None):
-        """master_init: fp32 device tensor with this rank's partition of the
-        initial master weights (for bfloat16 without master: of the initial
-        weights)."""
-        if stage not in (1, 2):
-            raise ValueError("peer ranks run stage 1 or 2")
-        psi = params.numel()
-        if grad.numel() != psi or grad.element_size() != 2 or params.element_size() != 2:
-            raise ValueError("grad and params: 16-bit tensors of the same length")
+        if stage not in (1, 2, 3):
+            raise ValueError("stage 1, 2 or 3")
+        psi = grad.numel()
+        if grad.element_size() != 2:
+            raise ValueError("grad: a 16-bit tensor")
+        if stage <= 2:
+            if params is None or params.numel() != psi or params.element_size() != 2:
+                raise ValueError("params: a 16-bit tensor as long as grad")
+        elif params is not None:
+            raise ValueError("stage 3 keeps the parameters in shards: params=None")
         self.group = group
+        self.stage = stage
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
-        self.stream = stream or torch.cuda.current_stream(params.device)
-        self.cfg = A.Config(psi, self.world, stage, rank_view=self.rank, variant=variant, tensors=tensors,
-                            precision=precision, view_outputs=self.world)
+        self.stream = stream or torch.cuda.current_stream(grad.device)
+        cfg_of = lambda r: A.Config(psi, self.world, stage, rank_view=r, variant=variant, tensors=tensors,
+                                    precision=precision, view_outputs=self.world if stage <= 2 else 0)
+        self.cfg = cfg_of(self.rank)
         L = A.zero_state_bytes(self.cfg)
-        P = L.partition_len
-        self.begin = min(self.rank * P, psi)
-        self.end = min(self.begin + P, psi)
+        if stage <= 2:
+            P = L.partition_len
+            self.begin = min(self.rank * P, psi)
+            self.end = min(self.begin + P, psi)
+        else:
+            self.begin, self.end = 0, psi
         if master_init.numel() != self.end - self.begin or master_init.dtype != torch.float32:
-            raise ValueError(f"master_init: {self.end - self.begin} fp32 elements of partition {self.rank}")
-        self.peers = PeerBuffers([(grad.data_ptr(), 2 * psi), (params.data_ptr(), 2 * psi)], group)
-        self.workspace = torch.empty(L.workspace_bytes, dtype=torch.uint8, device=params.device)
-        self.grad_ptrs = [row[0] + 2 * self.begin for row in self.peers.ptrs]
+            raise ValueError(f"master_init: {self.end - self.begin} fp32 elements")
+        self.workspace = torch.empty(L.workspace_bytes, dtype=torch.uint8, device=grad.device)
+        second = params if stage <= 2 else self.workspace
+        self.peers = PeerBuffers([(grad.data_ptr(), 2 * psi),
+                                  (second.data_ptr(), second.numel() * second.element_size())], group)
+        if stage <= 2:
+            self.grad_ptrs = [row[0] + 2 * self.begin for row in self.peers.ptrs]
+            outs = [row[1] for row in self.peers.ptrs]
+            self.shard_ptrs = None
+        else:
+            self.grad_ptrs = [row[0] for row in self.peers.ptrs]
+            outs = None
+            # rank k's shard sits at its own layout's offset in its workspace
+            self.shard_ptrs = [row[1] + A.zero_state_bytes(cfg_of(k)).off_shard16
+                               for k, row in enumerate(self.peers.ptrs)]
         self.h = None
         try:
             self.h = A.zero_init(self.cfg, self.workspace.data_ptr(), L.workspace_bytes,
-                                 master_init.data_ptr(), [row[1] for row in self.peers.ptrs],
-                                 self.stream.cuda_stream)
+                                 master_init.data_ptr(), outs, self.stream.cuda_stream)
         finally:
-            # every rank's initial partition is in every parameter buffer (or
-            # every rank learns here that one of them failed: the barrier ends)
+            # every rank's initial parameters are in place (or every rank
+            # learns here that one of them failed: the barrier ends)
             device_barrier(self.stream, group)
         self._grads = grad
         self._params = params
@@ -198,6 +224,22 @@ class PeerRank:
         skipped = rank_step(self.h, self.grad_ptrs, loss_scale, hp, self.stream, self.group)
         device_barrier(self.stream, self.group)
         return skipped
+
+    def unit_range(self, unit: int) -> tuple[int, int]:
+        """Flat offset and length of a layer unit (stage 3)."""
+        return A.zero_unit_range(self.cfg, unit)
+
+    def gather(self, unit: int, out: torch.Tensor) -> torch.Tensor:
+        """Stage 3: layer unit `unit` from the Nd ranks' shards into `out` (a
+        16-bit tensor of the unit's length), on this rank's stream. Local: the
+        shards it reads were completed by the step's closing barrier."""
+        if self.stage != 3:
+            raise ValueError("gather: stage 3 only")
+        _, n = self.unit_range(unit)
+        if out.numel() < n or out.element_size() != 2:
+            raise ValueError(f"out: at least {n} 16-bit elements")
+        A.zero_gather_layer_ranks(self.h, unit, self.shard_ptrs, out.data_ptr(), self.stream.cuda_stream)
+        return out
 
     def state(self) -> tuple[int, int, int, int]:
         """Device addresses of this rank's master, m, v and t."""
