@@ -16,9 +16,10 @@ with torch.distributed.all_reduce on the NCCL backend.
 
 PeerBuffers exchanges descriptors of device buffers (include/zero_peer.h)
 across the group and maps every rank's buffers into this process; PeerRank
-is the whole per-rank job of stages 1 and 2 on top of it: this rank's
-gradient and parameter buffers shared with the others, one handle, and the
-step bracketed by device barriers.
+is the whole per-rank job on top of it: this rank's gradient and parameter
+buffers (stage 1/2) or gradient and shard-holding workspace (stage 3) shared
+with the others, one handle, the step bracketed by device barriers, and on
+stage 3 the layer gather from every rank's shard.
 """
 from __future__ import annotations
 
