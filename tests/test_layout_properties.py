@@ -90,7 +90,10 @@ def test_stage3_rank_view(c, r):
     job = A.zero_state_bytes(A.Config(psi, nd, 3, variant=variant, tensors=tensors, precision=prec))
     cfg = A.Config(psi, nd, 3, rank_view=r, variant=variant, tensors=tensors, precision=prec)
     L = A.zero_state_bytes(cfg)
-    assert L.state_elems == Z.shard_len([t[0] for t in tensors], nd, r) == A.zero_rank_shard(cfg, r)[1]
+    assert L.state_elems == Z.shard_len([t[0] for t in tensors], nd, r)
+    # the handle holds shard r alone, from 0
+    assert [A.zero_rank_shard(cfg, k) for k in range(nd)] == [(0, L.state_elems if k == r else 0)
+                                                             for k in range(nd)]
     assert L.grad_len == psi
     assert list(L.exact_bytes) == list(job.exact_bytes) and L.transient_bytes == job.transient_bytes
     assert L.off_shard16 > 0 and L.off_shard16 + 2 * L.state_elems <= L.workspace_bytes

@@ -616,6 +616,11 @@ ZERO_API int zero_rank_shard(const zero_config* cfg, int32_t rank, int64_t* stat
     const int rc = build_layout(cfg, &L);
     if (rc != ZERO_OK) return rc;
     if (rank < 0 || rank >= L.nd) return ZERO_ERR_ARG;
+    if (L.view >= 0) {  // the handle holds the viewed rank's shard alone, from 0
+        *state_begin = 0;
+        *len = rank == L.view ? L.state_elems : 0;
+        return ZERO_OK;
+    }
     *state_begin = L.shard_begin[rank];
     *len = L.shard_len[rank];
     return ZERO_OK;
