@@ -337,6 +337,26 @@ int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
 int zero_gather_layer_ranks(zero_handle* h, int32_t unit, const uint16_t* const* shards, uint16_t* out,
                             void* stream);
 
+/* One copy of a stage-3 layer gather: `len` fp16 elements from offset
+ * src_begin of rank src_rank's shard to offset out_begin of the unit. */
+typedef struct zero_gather_run {
+    int64_t src_begin;
+    int64_t out_begin;
+    int64_t len;      /* > 0 */
+    int32_t src_rank;
+    int32_t reserved; /* 0 */
+} zero_gather_run;
+
+/* The copies that gather layer unit `unit` of a stage-3 configuration (any
+ * rank_view): one per non-empty chunk, tensor by tensor in the unit, ranks in
+ * order within a tensor, so out_begin increases and the runs tile the unit.
+ * What zero_gather_layer_ranks executes, for callers that move the chunks
+ * with a transport of their own. *n_runs receives the count; runs may be NULL
+ * to ask for it, else it must hold cap >= *n_runs entries. Host only.
+ * ZERO_ERR_STAGE on stage 1/2, ZERO_ERR_ARG for a bad unit or a short cap. */
+int zero_gather_plan(const zero_config* cfg, int32_t unit, zero_gather_run* runs, int64_t cap,
+                     int64_t* n_runs);
+
 /* Current state: device pointers to the live master/m/v arrays (the fused
  * variant alternates between two buffers) and the step count t. Any output
  * pointer may be NULL. ZERO_ERR_ARG while an asynchronous run is open. */

@@ -109,3 +109,47 @@ def test_stage3_rank_view(c, r):
         raise AssertionError("an offloaded stage-3 rank was accepted")
     except A.ZeroError as e:
         assert e.code == A.ZERO_ERR_ARG
+
+
+@settings(max_examples=200, deadline=None)
+@given(configs(), st.integers(-1, 39))
+def test_gather_plan_against_the_oracles_chunks(c, view):
+    """The stage-3 gather plan (zero_gather_plan: what the rank gather runs)
+    copies, for every tensor of a unit and every rank in order, the oracle's
+    chunk of that tensor from the rank's shard: the source offset is the
+    rank's earlier chunks, the destination the chunk's place in the unit, and
+    the runs tile the unit."""
+    nd, tensors, _, variant, _ = c
+    view = view % nd if view >= 0 else -1
+    numel = [t[0] for t in tensors]
+    unit_of = [t[1] for t in tensors]
+    psi = sum(numel)
+    cfg = A.Config(psi, nd, 3, rank_view=view, variant=variant, tensors=tensors)
+    def chunk_len(t, r):
+        b, e = Z.chunk(numel[t], nd, r)
+        return e - b
+
+    def in_shard(t, r):  # rank r's chunks of the tensors before t
+        return sum(chunk_len(k, r) for k in range(t))
+
+    for u in range(unit_of[-1] + 1):
+        flat0 = A.zero_unit_range(cfg, u)[0]
+        want = []
+        for t in (k for k in range(len(numel)) if unit_of[k] == u):
+            for r in range(nd):
+                b, e = Z.chunk(numel[t], nd, r)
+                if e > b:
+                    want.append((r, in_shard(t, r), sum(numel[:t]) - flat0 + b, e - b))
+        plan = A.zero_gather_plan(cfg, u)
+        assert plan == want
+        # tiling, and every source range inside its rank's shard
+        assert sum(x[3] for x in plan) == A.zero_unit_range(cfg, u)[1]
+        pos = 0
+        for r, sb, ob, n in plan:
+            assert ob == pos and n > 0 and 0 <= sb and sb + n <= Z.shard_len(numel, nd, r)
+            pos += n
+    try:
+        A.zero_gather_plan(A.Config(psi, nd, 2, variant=variant, tensors=tensors), 0)
+        raise AssertionError("a stage-2 plan was given")
+    except A.ZeroError as e:
+        assert e.code == A.ZERO_ERR_STAGE

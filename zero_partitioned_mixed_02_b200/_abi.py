@@ -94,6 +94,11 @@ ZERO_OFFLOAD_SLOTS = 3
 ZERO_OFFLOAD_DEFAULT_CHUNK = 1 << 22
 
 
+class zero_gather_run(C.Structure):
+    _fields_ = [("src_begin", C.c_int64), ("out_begin", C.c_int64), ("len", C.c_int64),
+                ("src_rank", C.c_int32), ("reserved", C.c_int32)]
+
+
 class zero_peer_desc(C.Structure):
     _fields_ = [("magic", C.c_uint32), ("device", C.c_int32), ("process", C.c_uint64),
                 ("offset", C.c_uint64), ("bytes", C.c_uint64), ("address", C.c_uint64),
@@ -130,6 +135,8 @@ def lib():
             "zero_step_commit": (C.c_int, [P, P, C.POINTER(C.c_int)]),
             "zero_gather_layer": (C.c_int, [P, C.c_int32, P, P]),
             "zero_gather_layer_ranks": (C.c_int, [P, C.c_int32, C.POINTER(P), P, P]),
+            "zero_gather_plan": (C.c_int, [C.POINTER(zero_config), C.c_int32, C.POINTER(zero_gather_run),
+                                           C.c_int64, C.POINTER(C.c_int64)]),
             "zero_async_begin": (C.c_int, [P, C.POINTER(P), C.POINTER(zero_scaler), C.c_float,
                                            C.c_float, P]),
             "zero_step_async": (C.c_int, [P, C.POINTER(zero_hyper), P]),
@@ -285,6 +292,15 @@ def zero_gather_layer_ranks(h: int, unit: int, shards: Sequence[int], out: int, 
     """Stage-3 rank of a real job: gather a layer unit from the Nd ranks'
     fp16 shards (shards[k]: rank k's shard, peer-mapped for other ranks)."""
     _check(lib().zero_gather_layer_ranks(h, unit, _ptr_array(shards), out, stream), "zero_gather_layer_ranks", h)
+
+
+def zero_gather_plan(cfg: Config, unit: int) -> list[tuple[int, int, int, int]]:
+    """The copies of a stage-3 layer gather: (src_rank, src_begin, out_begin, len)."""
+    n = C.c_int64()
+    _check(lib().zero_gather_plan(cfg.byref(), unit, None, 0, C.byref(n)), "zero_gather_plan")
+    runs = (zero_gather_run * max(n.value, 1))()
+    _check(lib().zero_gather_plan(cfg.byref(), unit, runs, n.value, C.byref(n)), "zero_gather_plan")
+    return [(r.src_rank, r.src_begin, r.out_begin, r.len) for r in runs[:n.value]]
 
 
 def zero_current_state(h: int) -> tuple[int, int, int, int]:

@@ -213,10 +213,12 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
                 for (int r = 0; r < nd; ++r) {
                     int64_t b, e;
                     split(L->numel[t], nd, r, &b, &e);
-                    if (view < 0) {
+                    if (view < 0)
                         add_run(L->gather_segs, &chunks, chunk_pos[t * nd + r],
                                 0, tensor_off[t] - U.flat_begin + b, e - b);
-                    } else if (e > b) {
+                    // the same copies by source rank (the rank gather's
+                    // table, and the plan zero_gather_plan reports)
+                    if (e > b) {
                         zg::Run g{};
                         g.src_begin = chunk_pos[t * nd + r] - L->shard_begin[r];
                         g.out_begin = tensor_off[t] - U.flat_begin + b;
@@ -626,6 +628,30 @@ ZERO_API int zero_rank_shard(const zero_config* cfg, int32_t rank, int64_t* stat
     return ZERO_OK;
 }
 
+ZERO_API int zero_gather_plan(const zero_config* cfg, int32_t unit, zero_gather_run* runs, int64_t cap,
+                             int64_t* n_runs)
+{
+    if (!n_runs) return ZERO_ERR_ARG;
+    Layout L;
+    const int rc = build_layout(cfg, &L);
+    if (rc != ZERO_OK) return rc;
+    if (L.stage != 3) return ZERO_ERR_STAGE;
+    if (unit < 0 || unit >= L.n_units) return ZERO_ERR_ARG;
+    const Unit& U = L.units[unit];
+    *n_runs = U.rank_n_runs;
+    if (!runs) return ZERO_OK;
+    if (cap < U.rank_n_runs) return ZERO_ERR_ARG;
+    for (int64_t i = 0; i < U.rank_n_runs; ++i) {
+        const zg::Run& g = L.rank_gather[U.rank_run0 + i];
+        runs[i].src_begin = g.src_begin;
+        runs[i].out_begin = g.out_begin;
+        runs[i].len = g.len;
+        runs[i].src_rank = g.rank;
+        runs[i].reserved = 0;
+    }
+    return ZERO_OK;
+}
+
 ZERO_API int zero_unit_range(const zero_config* cfg, int32_t unit, int64_t* flat_begin, int64_t* numel)
 {
     if (!flat_begin || !numel) return ZERO_ERR_ARG;
@@ -753,7 +779,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
                             L.gather_segs.size() * sizeof(zk::SegDesc), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && h->d_shard_len)
         e = cudaMemcpyAsync(h->d_shard_len, L.shard_len.data(), L.nd * sizeof(int64_t), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && !L.rank_gather.empty())
+    if (e == cudaSuccess && h->d_rank_gather && !L.rank_gather.empty())
         e = cudaMemcpyAsync(h->d_rank_gather, L.rank_gather.data(), L.rank_gather.size() * sizeof(zg::Run),
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && L.step_chunks > 0) {
