@@ -82,7 +82,8 @@ class ZeroAdam:
         return self._view_f32(w), self._view_f32(m), self._view_f32(v)
 
     def shard16(self) -> torch.Tensor:
-        """Stage 3: the fp16 parameter shards of all ranks (state order), as int16 bits."""
+        """Stage 3: the fp16 parameter shards (state order: every rank's when
+        emulating all ranks, this rank's alone for a rank view), as int16 bits."""
         off = self.ledger.off_shard16
         if off < 0:
             raise ValueError("only stage 3 keeps fp16 shards")
