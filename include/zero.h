@@ -219,8 +219,10 @@ int zero_unit_range(const zero_config* cfg, int32_t unit, int64_t* flat_begin, i
  *   workspace     device, >= ledger.workspace_bytes, owned by the caller and
  *                 used by the handle until zero_destroy.
  *   master_init   device fp32: the initial master weights of the elements this
- *                 handle owns, in flat order (psi values; the single-rank view
- *                 takes the P_r values of partition r; NULL if that is empty).
+ *                 handle owns, in flat order (psi values; the stage 1/2
+ *                 single-rank view takes the P_r values of partition r, NULL
+ *                 if that is empty; a stage-3 rank view takes all psi values
+ *                 and keeps its chunks).
  *   param_bufs    host array of device fp16 buffers that receive the all-
  *                 gathered parameters: stage 1/2 with all ranks: Nd replicas
  *                 of psi values each; single-rank view: one full psi-value
@@ -235,8 +237,9 @@ int zero_init(const zero_config* cfg, void* workspace, size_t workspace_bytes,
 /* One optimizer step.
  *   grads       host array of Nd device fp16 gradient buffers, rank order.
  *               All ranks: each holds psi values (the rank's full gradient).
- *               Single-rank view: each holds rank k's P_r gradients of the
- *               viewed partition r.
+ *               Stage 1/2 single-rank view: each holds rank k's P_r
+ *               gradients of the viewed partition r. Stage-3 rank view: each
+ *               holds rank k's full gradient (psi values).
  *   loss_scale  > 0 and finite; gradients are multiplied by 1/loss_scale.
  *   skipped     optional out: 1 if the step was skipped for overflow.
  * Returns ZERO_OK, or ZERO_SKIPPED when some unscaled reduced gradient is inf
