@@ -117,3 +117,54 @@ def test_argument_errors_without_cuda():
         A.zero_peer_open(bytes(d))
     assert e.value.code == A.ZERO_ERR_ARG
     assert A.zero_peer_open_count() == 0
+
+
+class _FakeStream:
+    def __init__(self):
+        self.synced = 0
+
+    def synchronize(self):
+        self.synced += 1
+
+
+def _barrier_worker(rank, world, port, q):
+    import time
+
+    import torch
+    import torch.distributed as dist
+    from zero_partitioned_mixed_02_b200.distributed import agree_overflow_any, device_barrier
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        s = _FakeStream()
+        if rank == 1:
+            time.sleep(1.0)  # the other rank must wait here for this one
+        t0 = time.monotonic()
+        device_barrier(s, None)
+        waited = time.monotonic() - t0
+        words = torch.tensor([0, 0] if rank == 0 else [5, 0], dtype=torch.int32)
+        agree_overflow_any(words)
+        q.put((rank, s.synced, waited, words.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_device_barrier_and_agreement_gloo():
+    """The gloo branch of the per-rank step's host side: device_barrier
+    synchronises the stream and holds every rank until all have arrived;
+    the overflow words are MAX-reduced (rank 1 overflowed on call 5)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_barrier_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(2):
+        rank, synced, waited, words = q.get(timeout=120)
+        got[rank] = (synced, waited, words)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    assert got[0][0] == got[1][0] == 1
+    assert got[0][1] > 0.5  # rank 0 waited for the late rank
+    assert got[0][2] == got[1][2] == [5, 0]
