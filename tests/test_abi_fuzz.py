@@ -1,6 +1,7 @@
 """Host-side robustness of the boundary (no GPU): arbitrary, mostly invalid
 configurations are either accepted with a consistent ledger or rejected
 with ZERO_ERR_ARG — never a crash."""
+import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
 
@@ -29,3 +30,36 @@ def test_state_bytes_accepts_or_rejects(psi, nd, stage, view, variant, precision
         assert L.state_elems == psi
     if tensors:
         assert sum(t[0] for t in tensors) == psi
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
+# host-side validation only: where a GPU is present, random IPC handles would
+# reach the driver, which this test has no reason to probe
+@pytest.mark.skipif(_has_gpu(), reason="host-side validation test; not run where a GPU is present")
+@settings(max_examples=300, deadline=None)
+@given(raw=st.binary(min_size=104, max_size=104), magic=st.booleans(), offset=st.integers(0, 1 << 40),
+       nbytes=st.integers(0, 1 << 40), address=st.integers(0, (1 << 64) - 1))
+def test_peer_descriptors_from_the_wire(raw, magic, offset, nbytes, address):
+    """zero_peer_open/close take descriptors received from other processes:
+    any 104 bytes are refused with an error code (ZERO_ERR_ARG, or
+    ZERO_ERR_CUDA where no device can map them), never a crash."""
+    d = A.zero_peer_desc.from_buffer_copy(raw)
+    if magic:
+        d.magic = A.ZERO_PEER_MAGIC
+        d.offset, d.bytes, d.address = offset, nbytes, address
+    desc = bytes(d)
+    try:
+        ptr = A.zero_peer_open(desc)
+    except A.ZeroError as e:
+        assert e.code in (A.ZERO_ERR_ARG, A.ZERO_ERR_CUDA)
+    else:  # only a descriptor naming this very process opens without a device
+        assert ptr == d.address
+    try:
+        A.zero_peer_close(desc, 16)
+    except A.ZeroError as e:
+        assert e.code in (A.ZERO_ERR_ARG, A.ZERO_ERR_CUDA)
+    assert A.zero_peer_open_count() == 0
