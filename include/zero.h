@@ -31,6 +31,14 @@
  * on-demand gather of one layer's full fp16 weights ([P1] "communication",
  * stage 3; [P3] "Partitioned parameters still have to participate").
  *
+ * A handle with rank_view = r acts as rank r alone. With one process per GPU
+ * it is rank r of a real job: on stage 1/2 with view_outputs = Nd its step
+ * reads partition r of every rank's gradient and writes partition r into
+ * every rank's parameter buffer; on stage 3 it keeps shard r and
+ * zero_gather_layer_ranks gathers layers from every rank's shard; in both
+ * cases the ranks agree on overflow through zero_flag_words. The other
+ * ranks' buffers are mapped with zero_peer.h.
+ *
  * Conventions for every call:
  *   - fp16 values are IEEE binary16 bit patterns (uint16_t).
  *   - "device" pointers are CUDA global-memory addresses on the current device;
