@@ -1,15 +1,19 @@
-"""zero_step_static, the allocation-free step, against the existing entry point.
+"""zero_step_static, the allocation-free step, against the existing entry point
+and against the oracle.
 
 zero_step_static is for callers that cannot allocate device memory for a
 workspace (their device memory belongs to another allocator, or they cannot
 afford cudaMalloc's cost and implicit synchronisation inside a step): its
 scratch lives in a fixed array inside the library. Here it is called through
-the C ABI on caller-owned state and checked, on two calls in a row, against
+the C ABI on caller-owned state and checked, call after call, against
 zero_step on a handle with the two-pass variant (the same arithmetic) fed the
-same gradients: master/m/v within the tests' tolerance (and bit for bit),
-fp16 replicas within 1 ulp (and bit for bit), the same step count. A third
-call with an inf gradient must skip on both paths. Sizes beyond the array's
-limits are rejected.
+same gradients, and against the oracle's data-parallel step (the definition
+of the result): master/m/v within the tests' tolerance (and bit for bit),
+fp16 replicas within 1 ulp (and bit for bit), the same step count. Four calls:
+two ordinary ones, one with an inf gradient that must skip on every path, and
+an ordinary one after the skip (the overflow word is cleared between calls).
+The sizes include ones where some ranks own empty partitions. Sizes beyond the
+array's limits are rejected.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process.
@@ -20,15 +24,19 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import zero_ref as Z
 from zero_partitioned_mixed_02_b200 import _abi as A
 from zero_partitioned_mixed_02_b200 import synth as S
 
-from gpu_common import compare_f16, compare_f32, host_f32, host_u16, hyper
+from gpu_common import compare_f16, compare_f32, dev_u16, host_f32, host_u16, hyper
 
 pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a GPU", allow_module_level=True)
+
+HP = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+SCALE = 1024.0
 
 
 def _state_view(ws: torch.Tensor, ptr: int, n: int) -> torch.Tensor:
@@ -36,12 +44,13 @@ def _state_view(ws: torch.Tensor, ptr: int, n: int) -> torch.Tensor:
     return ws[off: off + 4 * n].view(torch.float32)
 
 
-@pytest.mark.parametrize("psi,nd", [(A.ZERO_STATIC_MAX_PSI, 4), (70001, 5), (4099, 64), (1, 1)])
-def test_static_step_matches_handle_step(psi, nd):
+@pytest.mark.parametrize("psi,nd", [(A.ZERO_STATIC_MAX_PSI, 4), (70001, 5), (4099, 64), (1, 1),
+                                    (3, 8), (17, 64)])
+def test_static_step_matches_handle_step_and_oracle(psi, nd):
     s = torch.cuda.current_stream().cuda_stream
     w0 = S.host_f32(psi, 0, S.key(0, S.STREAM_MASTER, 0, 0), S.uniform(-0.1, 0.1))
-    gdist = S.normal(1e-3, 1024.0)
-    hp = hyper(lr=1e-3, weight_decay=0.01)
+    gdist = S.normal(1e-3, SCALE)
+    hp = hyper(**HP)
 
     # the existing entry point: a handle with its workspace
     cfg = A.Config(psi, nd, 2, variant=A.ZERO_VARIANT_TWO_PASS)
@@ -59,25 +68,36 @@ def test_static_step_matches_handle_step(psi, nd):
     reps_s = [torch.zeros(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
     t = 0
 
-    grads = [torch.empty(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
-    gp = [g.data_ptr() for g in grads]
-    for step in range(3):
-        for k in range(nd):
-            S.fill_f16(gp[k], psi, 0, S.key(0, S.STREAM_GRAD, step, k), gdist, s)
-        if step == 2:  # an inf on the last rank: both paths must skip
-            grads[nd - 1][psi // 2] = 0x7C00
-        rc_h = A.zero_step(h, gp, 1024.0, hp, s)
+    # the oracle: the plain data-parallel step on the CPU
+    ow, om, ov = w0.copy(), np.zeros(psi, np.float32), np.zeros(psi, np.float32)
+    op16 = Z.f16_from_f32(w0)
+    ot = 0
+    ohp = Z.hyper(**HP)
+
+    for step in range(4):
+        gs = [S.host_f16_bits(psi, 0, S.key(0, S.STREAM_GRAD, step, k), gdist) for k in range(nd)]
+        if step == 2:  # an inf on the last rank: every path must skip
+            gs[nd - 1][psi // 2] = 0x7C00
+        grads = [dev_u16(g) for g in gs]
+        gp = [g.data_ptr() for g in grads]
+        rc_h = A.zero_step(h, gp, SCALE, hp, s)
         rc_s, t = A.zero_step_static(psi, gp, master.data_ptr(), m.data_ptr(), v.data_ptr(),
-                                     [r.data_ptr() for r in reps_s], 1024.0, hp, t, s)
+                                     [r.data_ptr() for r in reps_s], SCALE, hp, t, s)
+        skipped, ot = Z.dp_step(gs, ow, om, ov, op16, SCALE, ohp, ot)
         want_rc = A.ZERO_SKIPPED if step == 2 else A.ZERO_OK
-        assert rc_h == want_rc and rc_s == want_rc
+        assert rc_h == want_rc and rc_s == want_rc and skipped == (step == 2)
         wp, mp, vp, th = A.zero_current_state(h)
-        assert th == t == min(step + 1, 2)
-        compare_f32(host_f32(master), host_f32(_state_view(ws, wp, psi)), f"master, call {step}")
-        compare_f32(host_f32(m), host_f32(_state_view(ws, mp, psi)), f"m, call {step}")
-        compare_f32(host_f32(v), host_f32(_state_view(ws, vp, psi)), f"v, call {step}")
+        assert th == t == ot == (step + 1 if step < 2 else step)
+        got = {"master": host_f32(master), "m": host_f32(m), "v": host_f32(v)}
+        handle = {"master": host_f32(_state_view(ws, wp, psi)), "m": host_f32(_state_view(ws, mp, psi)),
+                  "v": host_f32(_state_view(ws, vp, psi))}
+        oracle = {"master": ow, "m": om, "v": ov}
+        for name in got:
+            compare_f32(got[name], oracle[name], f"{name} vs oracle, call {step}")
+            compare_f32(got[name], handle[name], f"{name} vs zero_step, call {step}")
         for k in range(nd):
-            compare_f16(host_u16(reps_s[k]), host_u16(reps_h[k]), f"replica {k}, call {step}")
+            compare_f16(host_u16(reps_s[k]), op16, f"replica {k} vs oracle, call {step}")
+            compare_f16(host_u16(reps_s[k]), host_u16(reps_h[k]), f"replica {k} vs zero_step, call {step}")
     A.zero_destroy(h)
 
 

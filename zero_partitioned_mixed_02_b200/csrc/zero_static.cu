@@ -38,6 +38,44 @@ int g_sms[kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// beta^n as the n-fold double product 1.0 * beta * ... * beta, the same
+// definition as the handle path's bias corrections. The caller passes t, so
+// the products are kept between calls: a call continues from the last one's
+// products when its betas are the same and its n has not gone backwards, and
+// starts again from 1.0 otherwise. The loop also ends as soon as neither
+// product changes any more (a beta of 1, a product of 0, or the smallest
+// subnormal on which a beta below one settles), which bounds a large first t
+// to a few million multiplications; the values are those of the plain loop.
+struct Powers {
+    double b1 = -1.0, b2 = -1.0;
+    int64_t n = 0;
+    double p1 = 1.0, p2 = 1.0;
+};
+Powers g_pow;  // guarded by g_mu
+
+void beta_powers(double b1, double b2, int64_t n, double* p1, double* p2)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    Powers& c = g_pow;
+    if (c.b1 != b1 || c.b2 != b2 || c.n > n) {
+        c = Powers{};
+        c.b1 = b1;
+        c.b2 = b2;
+    }
+    while (c.n < n) {
+        const double q1 = c.p1 * b1, q2 = c.p2 * b2;
+        if (q1 == c.p1 && q2 == c.p2) {  // a fixed point: every further factor leaves both unchanged
+            c.n = n;
+            break;
+        }
+        c.p1 = q1;
+        c.p2 = q2;
+        ++c.n;
+    }
+    *p1 = c.p1;
+    *p2 = c.p2;
+}
+
 // The host-side name of a __device__ array is not its device address; the
 // address is looked up once per device, with that device current.
 cudaError_t setup(int dev, void** scratch)
@@ -86,7 +124,7 @@ ZERO_API int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* gr
 {
     if (skipped) *skipped = 0;
     if (psi < 1 || psi > ZERO_STATIC_MAX_PSI || nd < 1 || nd > ZERO_STATIC_MAX_ND) return ZERO_ERR_ARG;
-    if (!grads || !master || !m || !v || !replicas || !hp || !t || *t < 0) return ZERO_ERR_ARG;
+    if (!grads || !master || !m || !v || !replicas || !hp || !t || *t < 0 || *t == INT64_MAX) return ZERO_ERR_ARG;
     if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale)) return ZERO_ERR_ARG;
     if (!std::isfinite(hp->lr) || !std::isfinite(hp->beta1) || !std::isfinite(hp->beta2) ||
         !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
@@ -154,11 +192,8 @@ ZERO_API int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* gr
     a.c.omb2 = 1.0f - hp->beta2;
     a.c.eps = hp->eps;
     a.c.wd = hp->weight_decay;
-    double p1 = 1.0, p2 = 1.0;  // beta^t as the t-fold double product
-    for (int64_t k = 0; k < *t + 1; ++k) {
-        p1 = p1 * (double)hp->beta1;
-        p2 = p2 * (double)hp->beta2;
-    }
+    double p1, p2;  // beta^(t+1) as the (t+1)-fold double product
+    beta_powers((double)hp->beta1, (double)hp->beta2, *t + 1, &p1, &p2);
     a.c.bc1 = (float)(1.0 - p1);
     a.c.bc2 = (float)(1.0 - p2);
 
