@@ -40,6 +40,7 @@ CSRC = os.path.join(ROOT, "zero_partitioned_mixed_02_b200", "csrc")
 WORKLOADS = {
     "flat-1m": 1, "stress-16m": 2, "gpt2-1.5b": 3, "7.5b-rank-view": 4, "llama-2.7b": 5,
 }
+PROFILE_WORKLOADS = ("flat-64m", "llama-block")
 
 
 def parse_args():
@@ -48,7 +49,16 @@ def parse_args():
     p.add_argument("--steps", type=int, default=60)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2-1.5b")
+    p.add_argument("--mode", choices=["zero", "replicas"], default=None,
+                   help="with --gpus N > 1: 'zero' (default) runs the real job, Nd = N ranks, one "
+                        "partition per GPU over peer memory; 'replicas' runs N independent copies of the "
+                        "one-GPU emulation")
+    p.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
+                   help="process-group backend of the real job (gloo: ranks may share one GPU; "
+                        "no NCCL comparison)")
+    p.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PROFILE_WORKLOADS), default="gpt2-1.5b",
+                   help="the five configurations, or a small profiling case of their kernels "
+                        "(flat-64m: the stage-2 step at psi = 2^26; llama-block: one Llama block, stage 3)")
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass", "two-pass-tma"], default="fused-tma")
     p.add_argument("--precision", choices=["fp16", "bf16"], default="fp16",
                    help="bf16: bfloat16 gradients and parameters without fp32 master weights "
@@ -66,6 +76,9 @@ def parse_args():
                    help="elements per pipeline chunk of the offloaded step (0: the library default)")
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="time only --workload (by default a one-GPU fp16 synchronous run of a workload "
+                        "with psi >= 1B also times the other two under per_config)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
@@ -74,6 +87,8 @@ def parse_args():
 
 def workload(name):
     from zero_partitioned_mixed_02_b200.synth import workloads as W
+    if name in W.PROFILE:
+        return W.PROFILE[name]()
     return W.ALL[WORKLOADS[name]]()
 
 
@@ -376,13 +391,16 @@ def config_of(wl, variant):
 
 
 # ---------------------------------------------------------------- GPU leg
+SPEC_HBM_GBS = 8000.0  # the B200's HBM3e specification (context beside the measured peak)
+# the configurations with psi >= 1B that a default single-GPU run also times,
+# beside the headline workload
+PER_CONFIG = ("7.5b-rank-view", "llama-2.7b")
+PER_CONFIG_E2E_STEPS = 3
+
+
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
-
-    from zero_partitioned_mixed_02_b200 import _abi as A
-    from zero_partitioned_mixed_02_b200 import synth as S
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -393,13 +411,52 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    wl = workload(args.workload)
+    line, wl, bf16 = measure(args, args.workload, args.variant, args.e2e_steps, world, rank, local,
+                             prefetch=args.prefetch)
+    if (world == 1 and not args.no_per_config and args.precision == "fp16" and not args.async_steps
+            and args.workload in PER_CONFIG + ("gpt2-1.5b",)):
+        # the other large configurations, one after the other in the same run
+        # (each allocates its own buffers after the previous one's are freed)
+        line["per_config"] = {}
+        for name in PER_CONFIG:
+            if name == args.workload:
+                continue
+            torch.cuda.empty_cache()
+            if hasattr(torch._C, "_host_emptyCache"):
+                torch._C._host_emptyCache()  # the previous end-to-end leg's pinned buffers
+            sub, _, _ = measure(args, name, args.variant, min(args.e2e_steps, PER_CONFIG_E2E_STEPS), world,
+                                rank, local, prefetch=False, with_stream_copy=False)
+            line["per_config"][name] = {k: sub[k] for k in (
+                "value", "unit", "ms_per_step", "config", "hbm_gbs", "roofline", "gpu_launches", "clocks",
+                "gathers", "e2e") if k in sub}
+            torch.cuda.empty_cache()
+
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, bf16)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure(args, wl_name, variant_name, e2e_steps, world, rank, local, prefetch=False, with_stream_copy=True):
+    """Time one workload on this GPU: warm-up steps, then args.steps timed
+    steps (and on stage 3 the forward + backward layer gathers of each step),
+    the dominant kernel's roofline, and the end-to-end leg. Every buffer is
+    freed when it returns. Returns (line, workload, bf16)."""
+    import torch
+    import torch.distributed as dist
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+    from zero_partitioned_mixed_02_b200 import synth as S
+
+    wl = workload(wl_name)
     bf16 = args.precision == "bf16"
-    if bf16 and args.variant in ("fused", "fused-tma"):
-        args.variant = "two-pass-tma"  # without a master only the two-pass step exists
+    if bf16 and variant_name in ("fused", "fused-tma"):
+        variant_name = "two-pass-tma"  # without a master only the two-pass step exists
     variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
-               "fused-tma": A.ZERO_VARIANT_FUSED_TMA, "two-pass-tma": A.ZERO_VARIANT_TWO_PASS_TMA}[args.variant]
-    two_pass = args.variant.startswith("two-pass")
+               "fused-tma": A.ZERO_VARIANT_FUSED_TMA, "two-pass-tma": A.ZERO_VARIANT_TWO_PASS_TMA}[variant_name]
+    two_pass = variant_name.startswith("two-pass")
     cfg = A.Config(wl.psi, wl.nd, wl.stage, rank_view=wl.rank_view, variant=variant,
                    tensors=wl.tensors,
                    precision=A.ZERO_PRECISION_BF16 if bf16 else A.ZERO_PRECISION_FP16)
@@ -498,7 +555,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
 
-    n, floor, per_launch, gathers = algorithmic_bytes(wl, args.variant, bf16)
+    n, floor, per_launch, gathers = algorithmic_bytes(wl, variant_name, bf16)
     launches_per_step = (2 if two_pass else 1) + len(order)
     if args.async_steps:  # + the conditional roll-back (fused variants) and the commit kernel
         launches_per_step += 1 if two_pass else 2
@@ -509,7 +566,7 @@ def run_ours(args):
     k_s = statistics.mean(kern_ms) / 1e3
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
-    traffic = recorded_traffic(args.workload, args.variant + ("-bf16" if bf16 else ""))
+    traffic = recorded_traffic(wl_name, variant_name + ("-bf16" if bf16 else ""))
     codec = ",bf16" if bf16 else ""
     if two_pass and A.zero_uses_tma(h):
         kname = f"pass_tma_kernel<reduce{codec}>+<update{codec}>"
@@ -524,41 +581,38 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": config_of(wl, args.variant),
+        "config": config_of(wl, variant_name),
         "hbm_gbs": (floor + gathers) / step_s / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": kname,
                      "algorithmic_bytes_per_launch": dom_bytes,
-                     "kernel_ms": statistics.mean(kern_ms), "peak_source": peak_src},
+                     "kernel_ms": statistics.mean(kern_ms), "peak_source": peak_src,
+                     "spec_gbs": SPEC_HBM_GBS, "spec_frac": achieved / SPEC_HBM_GBS},
         "mode": "async" if args.async_steps else "sync",
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
     }
     # this library's copy kernel on 4 GB, after the timed region (context for
     # the measured peak, which stays the denominator)
-    line["stream_copy"] = {"kernel": "zero_stream_copy", "bytes": 1 << 32, "gbs": stream_copy_gbs(),
-                           "frac_of_peak": None}
-    line["stream_copy"]["frac_of_peak"] = line["stream_copy"]["gbs"] / peak
+    if with_stream_copy:
+        line["stream_copy"] = {"kernel": "zero_stream_copy", "bytes": 1 << 32, "gbs": stream_copy_gbs(),
+                               "frac_of_peak": None}
+        line["stream_copy"]["frac_of_peak"] = line["stream_copy"]["gbs"] / peak
     if gather_events:
         g_ms = statistics.mean(a.elapsed_time(b) for a, b in gather_events)
+        g_gbs = gathers / (g_ms / 1e3) / 1e9
         line["gathers"] = {"per_step_ms": g_ms, "launches_per_step": len(order),
-                           "bytes_per_step": gathers, "achieved_gbs": gathers / (g_ms / 1e3) / 1e9,
-                           "frac": gathers / (g_ms / 1e3) / 1e9 / peak}
+                           "bytes_per_step": gathers, "achieved_gbs": g_gbs,
+                           "frac": g_gbs / peak, "spec_frac": g_gbs / SPEC_HBM_GBS}
 
-    if args.prefetch and wl.stage == 3:
+    if prefetch and wl.stage == 3:
         line["prefetch"] = prefetch_demo(h, L, order, gather_out)
 
     # ---- end to end through the public API from pinned host buffers ----
-    if not args.no_e2e and args.e2e_steps > 0:
-        line["e2e"] = e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world)
+    if not args.no_e2e and e2e_steps > 0:
+        line["e2e"] = e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world, e2e_steps)
     A.zero_destroy(h)
-
-    if rank == 0 and not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, bf16)
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return line, wl, bf16
 
 
 def prefetch_demo(h, L, order, gather_out, reps=5):
@@ -629,7 +683,7 @@ def prefetch_demo(h, L, order, gather_out, reps=5):
     return out
 
 
-def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
+def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world, steps):
     import psutil
     import torch
     import torch.distributed as dist
@@ -637,7 +691,10 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
     from zero_partitioned_mixed_02_b200 import _abi as A
 
     n_own = grads[0].numel()
-    if wl.stage <= 2:
+    if wl.stage <= 2 and wl.rank_view >= 0:
+        b0, e0 = owned_range(wl)
+        result = bufs[0][b0:e0]  # the step's result: the new fp16 partition of this rank
+    elif wl.stage <= 2:
         result = bufs[0]  # the step's result: one rank's all-gathered fp16 parameters
     else:
         result = ws[L.off_shard16: L.off_shard16 + 2 * L.state_elems].view(torch.int16)
@@ -720,16 +777,227 @@ def e2e(args, wl, h, grads, gptrs, bufs, ws, L, hp, order, gather_out, world):
     a.record(s)
     up.wait_event(a)
     upload(0)
-    for k in range(args.e2e_steps):
-        step(k, args.e2e_steps - 1)
+    for k in range(steps):
+        step(k, steps - 1)
     s.wait_event(read_done)  # the last read-back is inside the timed region
     b.record(s)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), "cuda")
     n = L.state_elems
-    return {"value": whole_job_value(n, args.e2e_steps, world, ms), "unit": UNIT,
+    return {"value": whole_job_value(n, steps, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": len(grads) * n_own * 2, "d2h_bytes_per_step": result.numel() * 2,
-            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps, "pipelined": pipelined}
+            "steps": steps, "ms_per_step": ms / steps, "pipelined": pipelined}
+
+
+# ---------------------------------------------------------------- the real job
+NVLINK_PEER_GBS = 770.0  # measured peer copy on this machine, per direction per GPU (nominal 900)
+
+
+def zero_job_bytes(psi: int, world: int, stage: int, n_units_elems: int = 0) -> dict:
+    """Bytes one rank of the real Nd = world job moves per step, for the
+    slowest (first, full-length) partition P = ceil(psi / world). Stage 1/2:
+    it pulls partition r of the other ranks' fp16 gradients over NVLink and
+    stores the new fp16 partition into the other ranks' parameter buffers;
+    its own HBM serves its gradient slice to every rank, its state, and every
+    rank's store into its parameter buffer. Stage 3: the same pull of the
+    gradient chunks, the fp16 shard stays local; each layer gather pulls the
+    other ranks' chunks of the unit (n_units_elems: elements gathered per step
+    over all units, forward and backward)."""
+    P = -(-psi // world)
+    remote = world - 1
+    out = {"partition": P, "nvlink_in": 2 * P * remote, "nvlink_out": 0, "hbm": 0}
+    if stage <= 2:
+        out["nvlink_out"] = 2 * P * remote
+        out["hbm"] = 2 * P * world + 24 * P + 2 * P * world
+    else:
+        out["hbm"] = 2 * P * world + 24 * P + 2 * P
+        # gathers: (world - 1)/world of every unit's elements come from peers
+        out["nvlink_in_gathers"] = 2 * n_units_elems * remote // world
+    return out
+
+
+def run_zero_job(args):
+    """The real Nd = N job (SURVEY's multi-GPU design): one process per GPU,
+    rank r owns partition r (stage 1/2) or chunk r of every tensor (stage 3)
+    of the workload's parameter list; its step pulls the other ranks'
+    gradients of that partition through peer mappings, sums them in rank order
+    and runs Adam, then stores the new fp16 partition into every rank's
+    parameter buffer (stage 1/2; distributed.PeerRank); the overflow decision
+    is MAX-reduced between launch and commit. Timed with CUDA events on each
+    rank's stream, max over ranks; whole-job Gparams/s = psi per step. Beside
+    it: NCCL reduce-scatter + all-gather of the same fp16 bytes (NCCL backend
+    only)."""
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    from zero_partitioned_mixed_02_b200 import _abi as A
+    from zero_partitioned_mixed_02_b200 import synth as S
+    from zero_partitioned_mixed_02_b200.distributed import PeerRank, device_barrier
+
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = local % max(torch.cuda.device_count(), 1)
+    torch.cuda.set_device(dev)
+    if args.backend == "nccl":
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", dev))
+    else:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+    wl = workload(args.workload)
+    if wl.rank_view >= 0:
+        raise SystemExit("the real job runs a full-model workload (not the rank view)")
+    variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
+               "fused-tma": A.ZERO_VARIANT_FUSED_TMA, "two-pass-tma": A.ZERO_VARIANT_TWO_PASS_TMA}[args.variant]
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    psi, stage = wl.psi, wl.stage
+    grad = torch.empty(psi, dtype=torch.int16, device="cuda")
+    S.fill_f16(grad.data_ptr(), psi, 0, S.key(wl.seed, S.STREAM_GRAD, 0, rank), wl.grad, s)
+    P = -(-psi // world)
+    b, e = (min(rank * P, psi), min(rank * P + P, psi)) if stage <= 2 else (0, psi)
+    m_init = torch.empty(e - b, dtype=torch.float32, device="cuda")
+    S.fill_f32(m_init.data_ptr(), e - b, b, S.key(wl.seed, S.STREAM_MASTER, 0, 0), wl.master, s)
+    params = torch.empty(psi, dtype=torch.int16, device="cuda") if stage <= 2 else None
+    job = PeerRank(grad, params, m_init, stage=stage, variant=variant, tensors=wl.tensors, stream=stream)
+    del m_init
+    hp = A.zero_hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay)
+    order, gather_out, gathered = [], None, 0
+    if stage == 3:
+        L = A.zero_state_bytes(job.cfg)
+        order = list(range(L.n_units)) + list(reversed(range(L.n_units)))
+        gather_out = torch.empty(L.transient_bytes // 2, dtype=torch.int16, device="cuda")
+        gathered = sum(job.unit_range(u)[1] for u in order)
+
+    step_ev, gather_ev = [], []
+
+    def one_step(timed):
+        if timed:
+            a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        if job.step(wl.loss_scale, hp):
+            raise RuntimeError("unexpected skip in the benchmark workload")
+        if timed:
+            c.record(stream)
+            step_ev.append((a, c))
+        if order:
+            if timed:
+                g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                g0.record(stream)
+            for u in order:
+                job.gather(u, gather_out)
+            if timed:
+                g1.record(stream)
+                gather_ev.append((g0, g1))
+
+    for _ in range(args.warmup):
+        one_step(False)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(dev) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        one_step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop() if clocks else None
+    dev_str = "cuda" if args.backend == "nccl" else "cpu"
+    total_ms = max_over_ranks(t0.elapsed_time(t1), dev_str)
+    step_ms = max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in step_ev), dev_str)
+    g_ms = max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in gather_ev), dev_str) if gather_ev else None
+
+    by = zero_job_bytes(psi, world, stage, gathered)
+    nv_dir = max(by["nvlink_in"], by["nvlink_out"])
+    nv_gbs = nv_dir / (step_ms / 1e3) / 1e9
+    peak, peak_src = measured_peak()
+    line = {
+        "metric": METRIC, "value": psi * args.steps / (total_ms / 1e3) / 1e9, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "psi": psi, "nd": world, "stage": stage, "variant": args.variant,
+                   "elements_updated": psi, "partition": P, "loss_scale": wl.loss_scale,
+                   "weight_decay": wl.weight_decay, "backend": args.backend,
+                   "l2": "inputs larger than L2, no flush",
+                   "parallelism": f"zero-dp{world}: one partition per GPU, the reduce-scatter and "
+                                  f"all-gather fused into the step over peer memory"},
+        "roofline": {"bound": "nvlink", "achieved": nv_gbs, "peak": NVLINK_PEER_GBS, "unit": "GB/s",
+                     "frac": nv_gbs / NVLINK_PEER_GBS, "traffic": None, "kernel": "rank step",
+                     "algorithmic_bytes_per_launch": nv_dir, "kernel_ms": step_ms,
+                     "peak_source": "measured peer copy on this pool, per direction",
+                     "hbm_bytes_per_rank": by["hbm"],
+                     "hbm_gbs": by["hbm"] / (step_ms / 1e3) / 1e9, "hbm_peak": peak,
+                     "hbm_peak_source": peak_src},
+        "gpu_launches": ((2 if args.variant.startswith("two-pass") else 1) + len(order)) * args.steps,
+        "clocks": clock_info,
+    }
+    if g_ms is not None:
+        line["gathers"] = {"per_step_ms": g_ms, "launches_per_step": len(order),
+                           "nvlink_in_bytes_per_rank": by["nvlink_in_gathers"],
+                           "nvlink_gbs": by["nvlink_in_gathers"] / (g_ms / 1e3) / 1e9}
+
+    if args.backend == "nccl" and stage <= 2:
+        # NCCL's reduce-scatter + all-gather of the same fp16 bytes (no Adam,
+        # fp16 sums in NCCL's order): what the fused step replaces
+        pad = P * world
+        g16 = torch.zeros(pad, dtype=torch.float16, device="cuda")
+        g16[:psi].copy_(grad.view(torch.float16))
+        part = torch.empty(P, dtype=torch.float16, device="cuda")
+        full = torch.empty(pad, dtype=torch.float16, device="cuda")
+
+        def rs_ag():
+            dist.reduce_scatter_tensor(part, g16)
+            dist.all_gather_into_tensor(full, part)
+
+        for _ in range(max(args.warmup, 1)):
+            rs_ag()
+        torch.cuda.synchronize()
+        dist.barrier()
+        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            rs_ag()
+        c.record(stream)
+        torch.cuda.synchronize()
+        n_ms = max_over_ranks(a.elapsed_time(c) / args.steps, "cuda")
+        line["nccl_rs_ag"] = {"ms_per_step": n_ms, "bytes_per_rank_per_direction": 2 * P * (world - 1),
+                              "gbs_per_direction": 2 * P * (world - 1) / (n_ms / 1e3) / 1e9,
+                              "vs_rank_step": n_ms / step_ms}
+        del g16, part, full
+
+    if not args.no_e2e and args.e2e_steps > 0:
+        # end to end: every step uploads this rank's gradient from pinned host
+        # memory and reads back the step's result (this rank's new fp16
+        # partition, or its shard)
+        host_g = torch.empty(psi, dtype=torch.int16, pin_memory=True)
+        host_g.copy_(grad)
+        res = params[b:e] if stage <= 2 else job.workspace[
+            A.zero_state_bytes(job.cfg).off_shard16:].view(torch.int16)[: A.zero_state_bytes(job.cfg).state_elems]
+        host_out = torch.empty(res.numel(), dtype=torch.int16, pin_memory=True)
+        device_barrier(stream)
+        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            grad.copy_(host_g, non_blocking=True)
+            if job.step(wl.loss_scale, hp):
+                raise RuntimeError("unexpected skip")
+            for u in order:
+                job.gather(u, gather_out)
+            host_out.copy_(res, non_blocking=True)
+        c.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(c), dev_str)
+        line["e2e"] = {"value": psi * args.e2e_steps / (e_ms / 1e3) / 1e9, "unit": UNIT,
+                       "h2d_bytes_per_step": 2 * psi, "d2h_bytes_per_step": 2 * res.numel(),
+                       "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
+                       "per_rank": True}
+    job.close()
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def host_copy_gbs(threads, n_bytes=1 << 31, reps=5):
@@ -850,10 +1118,13 @@ def run_offload(args):
 
 def main():
     args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         run_reference(args)
     elif args.offload:
         run_offload(args)
+    elif world > 1 and (args.mode or "zero") == "zero":
+        run_zero_job(args)
     else:
         run_ours(args)
 

@@ -109,3 +109,39 @@ def test_overflow_agreement_gloo():
         assert p.exitcode == 0
     got = dict(q.get() for _ in range(2))
     assert got == {0: [7, 0], 1: [7, 0]}
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_real_job_bytes(world):
+    """The real job's per-rank byte counts: the NVLink bytes are the
+    reduce-scatter and all-gather volumes of the pages' accounting for one
+    rank ((Nd - 1) / Nd of 2 psi each way), and the rank's HBM bytes are the
+    one-GPU step's (24 + 4 Nd) per partition element."""
+    psi = 1_557_611_200
+    P = -(-psi // world)
+    b = bench.zero_job_bytes(psi, world, 2)
+    assert b["partition"] == P
+    assert b["nvlink_in"] == b["nvlink_out"] == 2 * P * (world - 1)
+    assert b["hbm"] == (24 + 4 * world) * P
+    b3 = bench.zero_job_bytes(psi, world, 3, n_units_elems=2 * psi)
+    assert b3["nvlink_in"] == 2 * P * (world - 1) and b3["nvlink_out"] == 0
+    assert b3["hbm"] == (26 + 2 * world) * P
+    assert b3["nvlink_in_gathers"] == 2 * (2 * psi) * (world - 1) // world
+
+
+def test_real_job_is_the_default_for_several_gpus(monkeypatch):
+    """bench.py --gpus N under torchrun (WORLD_SIZE > 1) runs the real job
+    unless --mode replicas asks for independent copies of the emulation."""
+    calls = []
+    monkeypatch.setattr(bench, "run_zero_job", lambda a: calls.append("zero"))
+    monkeypatch.setattr(bench, "run_ours", lambda a: calls.append("replicas"))
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    for argv, want in ((["bench.py", "--gpus", "2"], "zero"),
+                       (["bench.py", "--gpus", "2", "--mode", "replicas"], "replicas")):
+        monkeypatch.setattr("sys.argv", argv)
+        bench.main()
+        assert calls[-1] == want
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr("sys.argv", ["bench.py"])
+    bench.main()
+    assert calls[-1] == "replicas"

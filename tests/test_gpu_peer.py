@@ -317,3 +317,34 @@ def test_stage3_ranks_through_ipc_mappings():
                 compare_f32(w, ww[rank], f"master shard of {what}")
                 for u, (x, y) in enumerate(zip(units, wunits)):
                     compare_f16(x, y, f"unit {u} of {what}")
+
+
+@pytest.mark.parametrize("workload", ["stress-16m", "llama-block"])
+def test_bench_real_job_two_ranks(workload):
+    """bench.py's real-job mode (the default for --gpus N > 1), launched like
+    the multi-GPU benchmark (torchrun, one process per rank), here with two
+    ranks on this one GPU over gloo: peer mappings of the same device instead
+    of NVLink peers, no NCCL comparison. It must exit 0 and print one line
+    describing the Nd = 2 job (stage 2, and stage 3 with the rank gathers)."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = ["timeout", "-k", "60", "600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(root, "bench.py"), "--gpus", "2", "--backend", "gloo", "--workload", workload,
+           "--steps", "3", "--warmup", "3", "--e2e-steps", "2"]
+    out = subprocess.run(cmd, capture_output=True, text=True, cwd=root)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-4000:]
+    lines = [x for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["config"]["nd"] == 2 and line["scaling"] == "strong"
+    assert line["steps"] == 3 and line["value"] > 0 and line["gpu_launches"] > 0
+    assert line["roofline"]["bound"] == "nvlink" and line["roofline"]["kernel_ms"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 2 * line["config"]["psi"]
+    assert "nccl_rs_ag" not in line  # gloo: no NCCL leg
+    if workload == "llama-block":
+        assert line["config"]["stage"] == 3 and line["gathers"]["launches_per_step"] == 6

@@ -106,3 +106,32 @@ def llama_2p7b() -> Workload:
 
 
 ALL = {1: flat_1m, 2: stress_16m, 3: gpt2_1p5b, 4: running_example_7p5b, 5: llama_2p7b}
+
+
+# Small cases of the large workloads' kernels for profiler captures: inputs
+# well above the 126 MB L2, a few GB on the device in all.
+def flat_64m() -> Workload:
+    """The GPT-2 workload's stage-2 step at psi = 2^26 (one tensor, same value
+    distributions and Nd): about 3.6 GB on the device, 3.8 GB moved per step,
+    so the lines still dirty in L2 when a kernel ends are ~1-2 % of its bytes."""
+    return Workload("flat-64M-nd8-stage2", psi=1 << 26, nd=8, stage=2, steps=5,
+                    loss_scale=4096.0, grad=normal(1e-3, 4096.0), master=uniform(-0.1, 0.1),
+                    weight_decay=0.01)
+
+
+def llama_block() -> Workload:
+    """One block of the Llama-shaped 2.7B list (d = 2560, ffn 6912: 79.3M
+    parameters, 158.6 MB of fp16) between a 1024-row embedding (unit 0) and the
+    final norm + a 1024-row head (unit 2), Nd = 8, stage 3: the block's layer
+    gather has the full model's tensor and chunk shapes; about 3.7 GB on the
+    device."""
+    d, ffn = 2560, 6912
+    t = [(1024 * d, 0)]
+    t += [(d, 1), (d * d, 1), (d * d, 1), (d * d, 1), (d * d, 1), (d, 1), (ffn * d, 1), (ffn * d, 1), (d * ffn, 1)]
+    t += [(d, 2), (1024 * d, 2)]
+    return Workload("llama-block-nd8-stage3", psi=sum(n for n, _ in t), nd=8, stage=3, steps=3,
+                    loss_scale=1024.0, grad=normal(1e-3, 1024.0), master=uniform(-0.1, 0.1),
+                    tensors=t)
+
+
+PROFILE = {"flat-64m": flat_64m, "llama-block": llama_block}
