@@ -71,6 +71,14 @@ extern "C" {
 #define ZERO_ERR_INTERNAL (-6)  /* internal consistency check failed, or a bounded
                                    wait inside a kernel gave up; the step is then
                                    rolled back like a skipped one */
+#define ZERO_ERR_PARTIAL (-7)   /* a bounded wait of the in-place update pass of
+                                   ZERO_VARIANT_TWO_PASS_TMA gave up: some elements
+                                   of the master (without one: the 16-bit weights),
+                                   m, v and the parameters hold this step's values,
+                                   the others the previous step's; t did not
+                                   advance. Nothing can be rolled back: restore a
+                                   saved state with zero_set_state, which rewrites
+                                   the parameters too */
 
 /* ---- step variants ---- */
 /* One pass: reads the gradients and the current master/m/v, writes the next
@@ -89,10 +97,7 @@ extern "C" {
  * computed, and results leave by bulk stores. Same arithmetic, bytes and
  * workspace as ZERO_VARIANT_FUSED. Used when Nd <= 16 and every run's state
  * and output indices are in 16-byte phase with its gradient index; otherwise
- * the handle runs the ZERO_VARIANT_FUSED kernel. Its stage-3 layer gathers
- * copy through shared memory with bulk copies too (for units whose chunks are
- * in 16-byte phase with their place in the output); a gather whose bounded
- * wait gave up is reported by the next zero_step as ZERO_ERR_INTERNAL. */
+ * the handle runs the ZERO_VARIANT_FUSED kernel. */
 #define ZERO_VARIANT_FUSED_TMA 2
 /* The two passes of ZERO_VARIANT_TWO_PASS with their loads done by the Tensor
  * Memory Accelerator (bulk copies of gradient, reduced-gradient, moment and
@@ -100,8 +105,10 @@ extern "C" {
  * arithmetic, bytes and workspace as ZERO_VARIANT_TWO_PASS, under the same
  * eligibility rule as ZERO_VARIANT_FUSED_TMA (otherwise the plain two-pass
  * kernels run). Valid with both precisions. The update pass writes in place:
- * should one of its bounded waits give up (ZERO_ERR_INTERNAL), part of the
- * state may already be updated. */
+ * should one of its bounded waits give up, the step returns ZERO_ERR_PARTIAL
+ * (part of the state is already updated; restore it with zero_set_state). A
+ * wait of the reduce pass that gives up is rolled back (ZERO_ERR_INTERNAL):
+ * the update pass then writes nothing. */
 #define ZERO_VARIANT_TWO_PASS_TMA 3
 
 #define ZERO_MAX_ND 1024
@@ -323,14 +330,22 @@ int zero_async_begin(zero_handle* h, const uint16_t* const* grads, const zero_sc
 int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream);
 /* Close the run: synchronise `stream`, return the device-side counters and
  * hand t and the live buffer back to the host. Returns ZERO_ERR_INTERNAL if a
- * kernel gave up a bounded wait during the run (those steps were skipped). */
+ * kernel gave up a bounded wait during the run (those steps, and every later
+ * one of the run, were skipped), or ZERO_ERR_PARTIAL if that kernel was the
+ * in-place update pass of ZERO_VARIANT_TWO_PASS_TMA (part of the state holds
+ * that step's values: restore a saved state with zero_set_state). */
 int zero_async_end(zero_handle* h, void* stream, zero_async_state* out);
 
 /* Stage 3: write layer unit `unit`'s full fp16 weights into `out` (device,
  * >= the numel zero_unit_range reports): its tensors in tensor order, each whole
  * and contiguous, back to back. Call it per unit in forward order and again in
  * reverse for backward ([P1] "communication": parameters are gathered on demand
- * in the forward and backward passes, then discarded). ZERO_ERR_STAGE on 1/2. */
+ * in the forward and backward passes, then discarded). ZERO_ERR_STAGE on 1/2.
+ * Every variant gathers with the same copy kernel as zero_gather_layer_ranks
+ * (16-byte loads and stores, each block copying 16 KB tiles of one rank's
+ * chunk in turn), launched as a programmatic dependent of the previous kernel
+ * on `stream`: its blocks may be scheduled while that kernel finishes, but it
+ * touches no memory before that kernel has completed. */
 int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream);
 
 /* Stage-3 layer gather of rank r of a real Nd-rank job (a handle with
@@ -401,8 +416,14 @@ int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);
  *   master, m, v  device fp32, psi values each, updated in place (the caller
  *              initialises them: m = v = 0 before the first step)
  *   replicas   host array of nd device fp16 parameter buffers, psi values each
- *   t          host in/out step count (t-fold bias-correction products; it
- *              advances by one on a step that is not skipped)
+ *   t          host in/out step count, 0 <= t < INT64_MAX (the bias
+ *              corrections use the (t+1)-fold products of the betas; it
+ *              advances by one on a step that is not skipped). The library
+ *              keeps the last products and continues from them while the
+ *              betas stay the same and t does not go backwards, so a run
+ *              pays one multiplication per step; a large first t costs at
+ *              most a few million (the products stop changing at 0 or the
+ *              smallest subnormal).
  * The arithmetic and the result are those of zero_step with
  * ZERO_VARIANT_TWO_PASS on the same state. Returns ZERO_OK or ZERO_SKIPPED
  * (nothing changed), ZERO_ERR_ARG when psi > ZERO_STATIC_MAX_PSI or
@@ -415,8 +436,11 @@ int zero_stream_copy(void* dst, const void* src, size_t bytes, void* stream);
  * device address; make that first call before any stream capture. All calls
  * on a device share the array and it keeps the last call's contents (the
  * overflow word is cleared by each call): calls that overlap on the GPU, for
- * example on two streams, race with each other and must not be issued. The
- * call synchronises `stream` once to read the overflow word. */
+ * example on two streams, race with each other and must not be issued. Calls
+ * from two host threads at the same time race as well, even on one stream,
+ * because one call's table uploads can land between the other call's uploads
+ * and its kernels: serialise them. The call synchronises `stream` once to
+ * read the overflow word. */
 #define ZERO_STATIC_MAX_PSI 1048576
 #define ZERO_STATIC_MAX_ND 64
 int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* grads, float* master,
@@ -428,14 +452,21 @@ int zero_step_static(int64_t psi, int32_t nd, const uint16_t* const* grads, floa
 int zero_uses_tma(const zero_handle* h);
 
 /* Test hook for the bounded waits of the TMA kernels, which fail without any
- * GPU fault: the next TMA step or TMA layer gather on this handle leaves its
- * tile number `tile` unarmed, so the waits on it give up after `wait_rounds`
- * try_wait rounds (each suspends about a microsecond). The kernel sets its
- * error word and drains its own copies; the step is rolled back like a
- * skipped one and returns ZERO_ERR_INTERNAL (a gather's failure is reported,
- * and its step rolled back, by the next zero_step). The hook applies once.
- * Has no effect on handles that do not run the TMA kernels. */
+ * GPU fault: the next TMA step on this handle leaves its tile number `tile`
+ * unarmed, so the waits on it give up after `wait_rounds` try_wait rounds
+ * (each suspends about a microsecond). The kernel sets its error word and
+ * drains its own copies; the step is rolled back like a skipped one and
+ * returns ZERO_ERR_INTERNAL. The hook applies once.
+ * Has no effect on handles that do not run the TMA kernels. For
+ * ZERO_VARIANT_TWO_PASS_TMA the tile is one of the reduce pass. */
 int zero_test_hold_tile(zero_handle* h, int64_t tile, uint32_t wait_rounds);
+
+/* The same test hook for the update pass of ZERO_VARIANT_TWO_PASS_TMA: the
+ * next step's update pass leaves its tile number `tile` unarmed, its waits on
+ * it give up after `wait_rounds` rounds, the other tiles are updated in place,
+ * and the step returns ZERO_ERR_PARTIAL. Applies once; ZERO_ERR_ARG on a
+ * handle of another variant, or one that does not run the TMA kernels. */
+int zero_test_hold_update_tile(zero_handle* h, int64_t tile, uint32_t wait_rounds);
 
 /* The cudaError_t of the last failed CUDA call made through `h` (0 if none). */
 int zero_last_cuda_error(const zero_handle* h);

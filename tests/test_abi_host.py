@@ -174,7 +174,7 @@ def test_init_validation_before_device_work():
 
 
 def test_error_strings():
-    for code in (0, 1, -1, -2, -3, -4, -5, -6):
+    for code in (0, 1, -1, -2, -3, -4, -5, -6, -7):
         assert A.error_string(code) and A.error_string(code) != "unknown error code"
 
 

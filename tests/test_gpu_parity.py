@@ -365,31 +365,6 @@ def test_tma_wait_that_gives_up_is_reported_and_rolled_back(variant):
         c.close()
 
 
-@pytest.mark.parametrize("variant", TMA_VARIANTS)
-def test_tma_gather_wait_that_gives_up_is_reported(variant):
-    nd = 4
-    sizes = [8 * nd * 700, 8 * nd * 300, 8 * nd * 1200]
-    c = Case(sum(sizes), nd, 3, variant, tensors=list(zip(sizes, [0, 1, 1])))
-    assert c.uses_tma()
-    c.step(c.grads(0))
-    c.check("after step 0")
-    A.zero_test_hold_tile(c.h, 0, 1 << 14)
-    fb, cnt = A.zero_unit_range(c.cfg, 1)
-    out = GuardedF16(cnt)
-    A.zero_gather_layer(c.h, 1, out.ptr(), c.stream)  # its failure shows at the next step
-    n = c.e0 - c.b0
-    gs = c.grads(1)
-    for k in range(c.nd):
-        c.g_dev[k][:n].copy_(torch.from_numpy(gs[k].view(np.int16)))
-    with pytest.raises(A.ZeroError) as ei:
-        A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], c.loss_scale, hyper(), c.stream)
-    assert ei.value.code == A.ZERO_ERR_INTERNAL
-    c.check("after the reported failure: unchanged")  # gathers re-checked inside
-    assert c.step(c.grads(2)) is False
-    c.check("after the next step")
-    c.close()
-
-
 def _async_case(stage, variant, nd=4):
     if stage == 3:
         sizes = [8 * nd * 500, 8 * nd * 37, 8 * nd * 900]

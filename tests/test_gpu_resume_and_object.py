@@ -176,3 +176,91 @@ def test_zero_adam_bf16_object():
     assert sd["master"] is None and sd["t"] == 3
     opt.load_state_dict(sd)
     opt.close()
+
+
+@pytest.mark.parametrize("precision", [A.ZERO_PRECISION_FP16, A.ZERO_PRECISION_BF16])
+def test_partial_update_is_reported_and_restored(precision):
+    """The two-pass TMA step updates in place. A bounded wait of its update
+    pass that gives up (a tile left unarmed by the test hook: no fault) leaves
+    the state partly updated; ZeroAdam raises ZeroPartialUpdateError, the state
+    saved before the step restores master/m/v, t and the parameters exactly,
+    and the same step run again equals the oracle's."""
+    from zero_partitioned_mixed_02_b200 import ZeroAdam
+    from zero_partitioned_mixed_02_b200.optimizer import ZeroPartialUpdateError
+    bf16 = precision == A.ZERO_PRECISION_BF16
+    psi, nd = 200_000, 4
+    w0 = S.host_f32(psi, 0, S.key(5, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
+    reps = [torch.zeros(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
+    opt = ZeroAdam(psi, nd, 2, torch.from_numpy(w0.copy()).cuda(), reps,
+                   variant=A.ZERO_VARIANT_TWO_PASS_TMA, precision=precision)
+    assert A.zero_uses_tma(opt.h)
+    hp = Z.hyper(weight_decay=0.01)
+    if bf16:
+        w16, w = Z.bf16_from_f32(w0), None
+    else:
+        w, w16 = w0.copy(), Z.f16_from_f32(w0)
+    m, v, t = np.zeros(psi, np.float32), np.zeros(psi, np.float32), 0
+    grads = [torch.empty(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
+
+    def grads_of(s):
+        if bf16:
+            gs = [Z.bf16_from_f32(S.host_f32(psi, 0, S.key(5, S.STREAM_GRAD, s, k), S.normal(1e-3, 1.0)))
+                  for k in range(nd)]
+        else:
+            gs = [S.host_f16_bits(psi, 0, S.key(5, S.STREAM_GRAD, s, k), S.normal(1e-3, 1024.0))
+                  for k in range(nd)]
+        for g, x in zip(grads, gs):
+            g.copy_(torch.from_numpy(x.view(np.int16)))
+        return gs
+
+    scale = 1.0 if bf16 else 1024.0
+
+    def oracle_step(gs):
+        nonlocal t
+        if bf16:
+            _, t = Z.bf16_step(gs, w16, m, v, scale, hp, t)
+        else:
+            _, t = Z.dp_step(gs, w, m, v, w16, scale, hp, t)
+
+    def check(what):
+        gw, gm, gv = opt.state()
+        if not bf16:
+            compare_f32(host_f32(gw), w, f"master, {what}")
+        compare_f32(host_f32(gm), m, f"m, {what}")
+        compare_f32(host_f32(gv), v, f"v, {what}")
+        for r in reps:
+            compare_f16(host_u16(r), w16, f"parameters, {what}")
+        assert opt.t == t
+
+    gs = grads_of(0)
+    assert opt.step(grads, scale, weight_decay=0.01) is False
+    oracle_step(gs)
+    check("after step 0")
+    sd = opt.state_dict()
+
+    gs = grads_of(1)
+    A.zero_test_hold_update_tile(opt.h, 3, 1 << 14)
+    with pytest.raises(ZeroPartialUpdateError) as ei:
+        opt.step(grads, scale, weight_decay=0.01)
+    assert ei.value.code == A.ZERO_ERR_PARTIAL
+    assert opt.t == 1  # t did not advance
+    _, gm, _ = opt.state()
+    changed = int((host_f32(gm).view(np.uint32) != m.view(np.uint32)).sum())
+    assert 0 < changed < psi  # the other tiles were updated in place, the held one not
+
+    opt.load_state_dict(sd)
+    check("restored")
+    assert opt.step(grads, scale, weight_decay=0.01) is False
+    oracle_step(gs)
+    check("after the step run again")
+    opt.close()
+
+
+def test_update_hold_hook_refuses_other_variants():
+    psi, nd = 10_000, 2
+    for variant in (A.ZERO_VARIANT_FUSED_TMA, A.ZERO_VARIANT_TWO_PASS):
+        c = Case(psi, nd, 2, variant)
+        with pytest.raises(A.ZeroError) as ei:
+            A.zero_test_hold_update_tile(c.h, 0, 1 << 10)
+        assert ei.value.code == A.ZERO_ERR_ARG
+        c.close()

@@ -24,6 +24,7 @@ ZERO_ERR_STAGE = -3
 ZERO_ERR_WORKSPACE = -4
 ZERO_ERR_CUDA = -5
 ZERO_ERR_INTERNAL = -6
+ZERO_ERR_PARTIAL = -7
 
 ZERO_TENSOR_NO_DECAY = 1
 ZERO_PRECISION_FP16 = 0
@@ -152,6 +153,7 @@ def lib():
             "zero_uses_tma": (C.c_int, [P]),
             "zero_flag_words": (C.c_int, [P, C.POINTER(P)]),
             "zero_test_hold_tile": (C.c_int, [P, C.c_int64, C.c_uint32]),
+            "zero_test_hold_update_tile": (C.c_int, [P, C.c_int64, C.c_uint32]),
             "zero_error_string": (C.c_char_p, [C.c_int]),
             "zero_destroy": (None, [P]),
             "zero_offload_bytes": (C.c_int, [C.POINTER(zero_config), C.c_int64,
@@ -338,6 +340,10 @@ def zero_step_static(psi: int, grads: Sequence[int], master: int, m: int, v: int
 
 def zero_test_hold_tile(h: int, tile: int, wait_rounds: int) -> None:
     _check(lib().zero_test_hold_tile(h, tile, wait_rounds), "zero_test_hold_tile")
+
+
+def zero_test_hold_update_tile(h: int, tile: int, wait_rounds: int) -> None:
+    _check(lib().zero_test_hold_update_tile(h, tile, wait_rounds), "zero_test_hold_update_tile")
 
 
 def zero_flag_words(h: int) -> int:

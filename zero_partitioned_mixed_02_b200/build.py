@@ -43,7 +43,7 @@ HOST_ADAM = os.path.join(CSRC, "zero_host_adam.cpp")
 ZERO_DEPS = ZERO_SOURCES + [HOST_ADAM, os.path.join(CSRC, "zero_host_adam.h"),
                             os.path.join(CSRC, "zero_internal.h"), os.path.join(CSRC, "zero_device.cuh"),
                             os.path.join(CSRC, "zero_layout.h"), os.path.join(CSRC, "zero_tma.cuh"),
-                            os.path.join(CSRC, "zero_gather_ranks.h"),
+                            os.path.join(CSRC, "zero_gather_ranks.h"), os.path.join(CSRC, "zero_pdl.cuh"),
                             os.path.join(INCLUDE, "zero.h"),
                             os.path.join(INCLUDE, "zero_offload.h"), os.path.join(INCLUDE, "zero_peer.h")]
 # the host update is built twice: AVX2 + F16C, and the baseline instruction set

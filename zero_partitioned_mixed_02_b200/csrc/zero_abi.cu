@@ -236,35 +236,6 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             U.n_chunks = chunks;
             U.rank_n_runs = (int64_t)L->rank_gather.size() - U.rank_run0;
             L->transient_elems = std::max(L->transient_elems, U.numel);
-            if (is_tma(cfg->variant) && view < 0) {
-                bool ok = U.n_segs > 0;
-                for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
-                    const zk::SegDesc& g = L->gather_segs[i];
-                    if ((g.out_begin - g.grad_begin) % 8 != 0) ok = false;
-                }
-                if (ok) {
-                    U.tma_ok = true;
-                    U.tma_run0 = (int64_t)L->tma_gather.size();
-                    for (int64_t i = U.seg0; i < U.seg0 + U.n_segs; ++i) {
-                        const zk::SegDesc& g = L->gather_segs[i];
-                        zk::TmaRun t{};
-                        t.grad_begin = g.grad_begin;
-                        t.out_begin = g.out_begin;
-                        t.len = g.len;
-                        int64_t head = (zk::kLineElems - g.grad_begin % zk::kLineElems) % zk::kLineElems;
-                        if (head > g.len) head = g.len;
-                        const int64_t body = (g.len - head) / 8 * 8;
-                        t.head = (int)head;
-                        t.tail = (int)(g.len - head - body);
-                        t.tile_begin = U.tma_tiles;
-                        t.scal_begin = U.tma_scal;
-                        U.tma_tiles += (body + zk::kGatherTile - 1) / zk::kGatherTile;
-                        U.tma_scal += t.head + t.tail;
-                        L->tma_gather.push_back(t);
-                    }
-                    U.tma_n_runs = (int64_t)L->tma_gather.size() - U.tma_run0;
-                }
-            }
         }
     }
 
@@ -319,8 +290,6 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
     off += align_up((int64_t)std::max(L->n_out, 1) * 8);
     L->off_step_segs = off;
     off += align_up((int64_t)std::max<size_t>(L->step_segs.size(), 1) * sizeof(zk::SegDesc));
-    L->off_gather_segs = off;
-    off += align_up((int64_t)L->gather_segs.size() * sizeof(zk::SegDesc));
     if (L->tma_ok) {
         L->off_tma_runs = off;
         off += align_up((int64_t)L->tma_runs.size() * sizeof(zk::TmaRun));
@@ -329,12 +298,9 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
             off += align_up((int64_t)L->tma_runs_r.size() * sizeof(zk::TmaRun));
         }
     }
-    if (!L->tma_gather.empty()) {
-        L->off_tma_gather = off;
-        off += align_up((int64_t)L->tma_gather.size() * sizeof(zk::TmaRun));
-    }
-    if (cfg->stage == 3 && cfg->rank_view >= 0) {
-        // the Nd shard addresses, then the Nd shard lengths
+    if (cfg->stage == 3) {
+        // the Nd shard addresses, then the Nd shard lengths (a rank of a real
+        // job: the ranks' shards; emulated ranks: their places in the shard array)
         L->off_shard_tab = off;
         off += align_up((int64_t)nd * 16);
         L->off_rank_gather = off;
@@ -425,15 +391,13 @@ struct zero_handle {
     int sms = 0;
     int occ[zk::K_COUNT] = {};
     zk::SegDesc* d_step_segs = nullptr;
-    zk::SegDesc* d_gather_segs = nullptr;
     zk::TmaRun* d_tma_runs = nullptr;
     bool use_tma = false;  // TMA variant and its kernel fits on this device
     int occ_tma = 0;       // fused kernel, or the update pass of the two-pass TMA variant
     zk::TmaRun* d_tma_runs_r = nullptr;  // two-pass TMA variant: the reduce pass's table
     int occ_tma_r = 0;
-    zk::TmaRun* d_tma_gather = nullptr;
-    int occ_gather_tma = 0;
-    // stage-3 rank view: the gather from the Nd ranks' shards
+    // stage 3: the layer gather from the Nd ranks' shards (a real rank: the
+    // ranks' shards, peer-mapped; emulated ranks: places in the shard array)
     const uint16_t** d_shard_tab = nullptr;
     int64_t* d_shard_len = nullptr;
     zg::Run* d_rank_gather = nullptr;
@@ -442,6 +406,8 @@ struct zero_handle {
     bool shard_tab_valid = false;
     int64_t hold_tile = -1;  // test hook for the bounded waits (zero_test_hold_tile)
     unsigned hold_rounds = 0;
+    int64_t hold_update_tile = -1;  // the same for the update pass (zero_test_hold_update_tile)
+    unsigned hold_update_rounds = 0;
     bool async = false;      // between zero_async_begin and zero_async_end
     float async_b1 = 0.0f, async_b2 = 0.0f;
     zk::Ctrl ctrl_host{};    // staging copy of the control block
@@ -592,8 +558,9 @@ cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_
     ta.n_runs = (int)L.tma_runs.size();
     ta.n_tiles = L.tma_tiles;
     ta.n_scal = L.tma_scal;
-    ta.hold_tile = -1;
-    ta.wait_rounds = zk::kTmaWaitRounds;
+    ta.hold_tile = h->hold_update_tile;
+    ta.wait_rounds = h->hold_update_tile >= 0 ? h->hold_update_rounds : zk::kTmaWaitRounds;
+    h->hold_update_tile = -1;
     const int64_t cap = (int64_t)h->sms * h->occ_tma;
     const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
     return zk::launch_pass_tma(zk::kPassUpdate, ta, (int)std::min(want, cap), s, L.bf16);
@@ -716,7 +683,6 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     h->d_grad_tab = reinterpret_cast<const uint16_t**>(h->ws + L.off_grad_tab);
     h->d_out_tab = reinterpret_cast<uint16_t**>(h->ws + L.off_out_tab);
     h->d_step_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_step_segs);
-    h->d_gather_segs = reinterpret_cast<zk::SegDesc*>(h->ws + L.off_gather_segs);
     if (L.tma_ok) {
         h->d_tma_runs = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs);
         if (is_fused(L.variant)) {
@@ -732,15 +698,6 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
             return rc;
         }
         h->use_tma = h->occ_tma >= 1 && h->occ_tma_r >= 1;
-    }
-    if (!L.tma_gather.empty()) {
-        h->d_tma_gather = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_gather);
-        e = zk::tma_gather_prepare(&h->occ_gather_tma);
-        if (e != cudaSuccess) {
-            rc = cuda_fail(h, e);
-            delete h;
-            return rc;
-        }
     }
     if (L.off_shard_tab >= 0) {
         h->d_shard_tab = reinterpret_cast<const uint16_t**>(h->ws + L.off_shard_tab);
@@ -771,12 +728,14 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     if (e == cudaSuccess && !L.tma_runs_r.empty())
         e = cudaMemcpyAsync(h->d_tma_runs_r, L.tma_runs_r.data(), L.tma_runs_r.size() * sizeof(zk::TmaRun),
                             cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && !L.tma_gather.empty())
-        e = cudaMemcpyAsync(h->d_tma_gather, L.tma_gather.data(), L.tma_gather.size() * sizeof(zk::TmaRun),
-                            cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && !L.gather_segs.empty())
-        e = cudaMemcpyAsync(h->d_gather_segs, L.gather_segs.data(),
-                            L.gather_segs.size() * sizeof(zk::SegDesc), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && h->d_shard_tab && L.view < 0) {
+        // emulated ranks: shard r starts at its place in the handle's own shard array
+        const uint16_t* base = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
+        h->shard_tab.resize(L.nd);
+        for (int r = 0; r < L.nd; ++r) h->shard_tab[r] = base + L.shard_begin[r];
+        h->shard_tab_valid = true;
+        e = cudaMemcpyAsync(h->d_shard_tab, h->shard_tab.data(), L.nd * sizeof(uint16_t*), cudaMemcpyHostToDevice, s);
+    }
     if (e == cudaSuccess && h->d_shard_len)
         e = cudaMemcpyAsync(h->d_shard_len, L.shard_len.data(), L.nd * sizeof(int64_t), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && h->d_rank_gather && !L.rank_gather.empty())
@@ -931,7 +890,8 @@ ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
             e = cudaMemsetAsync(h->d_flag + 1, 0, sizeof(unsigned), s);
             if (e == cudaSuccess) e = cudaStreamSynchronize(s);
             if (e != cudaSuccess) return cuda_fail(h, e);
-            return ZERO_ERR_INTERNAL;
+            // the in-place update pass gave up part of the way: nothing to roll back
+            return (h->host_flag[1] & zk::kErrUpdate) ? ZERO_ERR_PARTIAL : ZERO_ERR_INTERNAL;
         }
         if (skipped) *skipped = 1;
         return ZERO_SKIPPED;
@@ -988,6 +948,7 @@ ZERO_API int zero_async_begin(zero_handle* h, const uint16_t* const* grads, cons
     c.interval = sc->growth_interval;
     c.cur = h->cur;
     c.fused = is_fused(L.variant);
+    zk::ctrl_next_constants(&c);
     e = cudaMemcpyAsync(h->d_ctrl, &c, sizeof(zk::Ctrl), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->d_flag, 0, sizeof(unsigned), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -1079,10 +1040,35 @@ ZERO_API int zero_async_end(zero_handle* h, void* stream, zero_async_state* out)
         e = cudaMemsetAsync(h->d_flag + 1, 0, sizeof(unsigned), s);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
         if (e != cudaSuccess) return cuda_fail(h, e);
-        return ZERO_ERR_INTERNAL;
+        return (err & zk::kErrUpdate) ? ZERO_ERR_PARTIAL : ZERO_ERR_INTERNAL;
     }
     return ZERO_OK;
 }
+
+namespace {
+
+// One layer unit from the Nd shards the handle's table points to, with the
+// copy kernel of zero_gather_ranks.cu.
+int launch_rank_gather(zero_handle* h, const Unit& U, uint16_t* out, cudaStream_t s)
+{
+    if (U.rank_tiles == 0) return ZERO_OK;
+    const Layout& L = h->L;
+    zg::Args g{};
+    g.runs = h->d_rank_gather + U.rank_run0;
+    g.n_runs = (int)U.rank_n_runs;
+    g.nd = L.nd;
+    g.n_tiles = U.rank_tiles;
+    g.shards = h->d_shard_tab;
+    g.shard_len = h->d_shard_len;
+    g.dst = out;
+    g.dst_len = U.numel;
+    g.err = h->d_flag + 1;
+    const int64_t cap = (int64_t)h->sms * std::max(h->occ_gather_ranks, 1);
+    const cudaError_t e = zg::launch(g, (int)std::min(U.rank_tiles, cap), s);
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+}
+
+}  // namespace
 
 ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void* stream)
 {
@@ -1094,38 +1080,7 @@ ZERO_API int zero_gather_layer(zero_handle* h, int32_t unit, uint16_t* out, void
     if (unit < 0 || unit >= L.n_units || !out) return ZERO_ERR_ARG;
     if (!aligned16(out)) return ZERO_ERR_ALIGN;
     const Unit& U = L.units[unit];
-    if (U.n_chunks == 0) return ZERO_OK;
-    if (U.tma_ok && h->occ_gather_tma >= 1) {
-        zk::TmaGatherArgs g{};
-        g.runs = h->d_tma_gather + U.tma_run0;
-        g.n_runs = (int)U.tma_n_runs;
-        g.n_tiles = U.tma_tiles;
-        g.n_scal = U.tma_scal;
-        g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
-        g.dst = out;
-        g.err = h->d_flag + 1;
-        g.wait_rounds = h->hold_tile >= 0 ? h->hold_rounds : zk::kTmaWaitRounds;
-        g.hold_tile = h->hold_tile;
-        g.src_len = L.state_elems;
-        g.dst_len = U.numel;
-        h->hold_tile = -1;
-        const int64_t want = std::max<int64_t>(1, std::max(U.tma_tiles, (U.tma_scal + 31) / 32));
-        const int64_t cap = (int64_t)h->sms * h->occ_gather_tma;
-        const cudaError_t e = zk::launch_gather_tma(g, (int)std::min(want, cap), static_cast<cudaStream_t>(stream));
-        return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
-    }
-    zk::GatherArgs g{};
-    g.segs = h->d_gather_segs + U.seg0;
-    g.n_segs = (int)U.n_segs;
-    g.n_chunks = U.n_chunks;
-    g.src = reinterpret_cast<const uint16_t*>(h->ws + L.off_shard16);
-    g.dst = out;
-    g.err = h->d_flag + 1;
-    g.src_len = L.state_elems;
-    g.dst_len = U.numel;
-    const cudaError_t e = zk::launch_gather(g, grid_for(h, zk::K_GATHER, U.n_chunks),
-                                            static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+    return launch_rank_gather(h, U, out, static_cast<cudaStream_t>(stream));
 }
 
 ZERO_API int zero_gather_layer_ranks(zero_handle* h, int32_t unit, const uint16_t* const* shards, uint16_t* out,
@@ -1152,19 +1107,7 @@ ZERO_API int zero_gather_layer_ranks(zero_handle* h, int32_t unit, const uint16_
         if (e != cudaSuccess) return cuda_fail(h, e);
         h->shard_tab_valid = true;
     }
-    zg::Args g{};
-    g.runs = h->d_rank_gather + U.rank_run0;
-    g.n_runs = (int)U.rank_n_runs;
-    g.nd = L.nd;
-    g.n_tiles = U.rank_tiles;
-    g.shards = h->d_shard_tab;
-    g.shard_len = h->d_shard_len;
-    g.dst = out;
-    g.dst_len = U.numel;
-    g.err = h->d_flag + 1;
-    const int64_t cap = (int64_t)h->sms * std::max(h->occ_gather_ranks, 1);
-    const cudaError_t e = zg::launch(g, (int)std::min(U.rank_tiles, cap), s);
-    return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);
+    return launch_rank_gather(h, U, out, s);
 }
 
 ZERO_API int zero_set_state(zero_handle* h, const float* master, const float* m, const float* v, int64_t t,
@@ -1239,6 +1182,15 @@ ZERO_API int zero_test_hold_tile(zero_handle* h, int64_t tile, uint32_t wait_rou
     return ZERO_OK;
 }
 
+ZERO_API int zero_test_hold_update_tile(zero_handle* h, int64_t tile, uint32_t wait_rounds)
+{
+    if (!h || tile < 0 || wait_rounds == 0) return ZERO_ERR_ARG;
+    if (h->L.variant != ZERO_VARIANT_TWO_PASS_TMA || !h->use_tma) return ZERO_ERR_ARG;
+    h->hold_update_tile = tile;
+    h->hold_update_rounds = wait_rounds;
+    return ZERO_OK;
+}
+
 ZERO_API int zero_flag_words(zero_handle* h, uint32_t** words)
 {
     if (!h || !words) return ZERO_ERR_ARG;
@@ -1261,6 +1213,7 @@ ZERO_API const char* zero_error_string(int code)
         case ZERO_ERR_WORKSPACE: return "workspace too small";
         case ZERO_ERR_CUDA: return "CUDA error";
         case ZERO_ERR_INTERNAL: return "internal error";
+        case ZERO_ERR_PARTIAL: return "update pass gave up part of the way: state partly updated, restore it";
         default: return "unknown error code";
     }
 }

@@ -290,11 +290,9 @@ __device__ __forceinline__ Live live_of(const StepArgs& a)
         return L;
     }
     const Ctrl* c = a.ctrl;
-    const double p1 = c->p1 * (double)c->b1;
-    const double p2 = c->p2 * (double)c->b2;
-    L.c.bc1 = (float)(1.0 - p1);
-    L.c.bc2 = (float)(1.0 - p2);
-    L.c.inv_scale = (float)(1.0 / (double)c->scale);
+    L.c.bc1 = c->bc1;  // written by zero_async_begin and by the last commit
+    L.c.bc2 = c->bc2;
+    L.c.inv_scale = c->inv_scale;
     const bool in1 = c->cur != 0;
     const bool out1 = c->fused ? !in1 : in1;
     L.w_in = in1 ? a.st[1][0] : a.st[0][0];

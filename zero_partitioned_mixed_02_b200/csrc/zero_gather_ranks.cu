@@ -2,11 +2,33 @@
 // bound by memory (and, across GPUs, by NVLink) bandwidth. Each block takes
 // tiles of 16 KB in turn; a tile is a piece of one rank's chunk, copied with
 // 16-byte loads and stores where source and destination share their offset
-// within 16 bytes, element by element otherwise.
+// within 16 bytes, element by element otherwise. Launched as a programmatic
+// dependent (zero_pdl.cuh), like the emulated layer gather.
 #include "zero_gather_ranks.h"
+#include "zero_pdl.cuh"
 
 namespace zg {
 namespace {
+
+// Every element is read and written once: streaming loads and stores
+// (ZG_STREAMING) keep them from displacing reusable lines in L2.
+__device__ __forceinline__ uint4 ld16(const uint4* p)
+{
+#if ZG_STREAMING
+    return __ldcs(p);
+#else
+    return *p;
+#endif
+}
+
+__device__ __forceinline__ void st16(uint4* p, uint4 x)
+{
+#if ZG_STREAMING
+    __stcs(p, x);
+#else
+    *p = x;
+#endif
+}
 
 __device__ __forceinline__ void copy_span(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int64_t n)
 {
@@ -23,28 +45,42 @@ __device__ __forceinline__ void copy_span(const uint16_t* __restrict__ src, uint
     const uint4* __restrict__ s4 = reinterpret_cast<const uint4*>(src + head);
     uint4* __restrict__ d4 = reinterpret_cast<uint4*>(dst + head);
     int64_t i = threadIdx.x;
-    for (; i + 3 * bd < body; i += 4 * bd) {  // four loads in flight per thread
-        const uint4 x0 = s4[i], x1 = s4[i + bd], x2 = s4[i + 2 * bd], x3 = s4[i + 3 * bd];
-        d4[i] = x0;
-        d4[i + bd] = x1;
-        d4[i + 2 * bd] = x2;
-        d4[i + 3 * bd] = x3;
+    for (; i + (kUnroll - 1) * bd < body; i += kUnroll * bd) {  // kUnroll loads in flight per thread
+        uint4 x[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) x[k] = ld16(s4 + i + k * bd);
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) st16(d4 + i + k * bd, x[k]);
     }
-    for (; i < body; i += bd) d4[i] = s4[i];
+    for (; i < body; i += bd) st16(d4 + i, ld16(s4 + i));
     for (int64_t j = head + body * 8 + threadIdx.x; j < n; j += bd) dst[j] = src[j];
 }
 
-__global__ void __launch_bounds__(kThreads) gather_ranks_kernel(const Args a)
+// the last run whose first tile is at or before `tile`
+__device__ __forceinline__ int find_run(const Run* runs, int n_runs, int64_t tile)
 {
+    int lo = 0, hi = n_runs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (runs[mid].tile_begin <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Tiles go to blocks round robin (tile = block + k * grid), so the whole grid
+// copies one narrow, advancing window of the unit at a time. kMinBlocks blocks
+// of kThreads per SM with kUnroll 16-byte loads in flight per thread (64 KB
+// per SM) measured fastest on the Llama layer walk: more bytes in flight per
+// SM (more blocks, or 8 loads per thread), contiguous spans of tiles per block,
+// and streaming cache hints were all slower.
+__global__ void __launch_bounds__(kThreads, kMinBlocks) layer_gather_kernel(const Args a)
+{
+    // a programmatic dependent launch: wait for the previous kernel on the stream
+    zk::pdl_wait();
+    zk::pdl_launch_dependents();
     for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
-        // the last run whose first tile is at or before this one
-        int lo = 0, hi = a.n_runs - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (a.runs[mid].tile_begin <= tile) lo = mid;
-            else hi = mid - 1;
-        }
-        const Run r = a.runs[lo];
+        const Run r = a.runs[find_run(a.runs, a.n_runs, tile)];
         const int64_t e0 = (tile - r.tile_begin) * kTile;
         const int64_t n = r.len - e0 < kTile ? r.len - e0 : kTile;
 #ifdef ZK_BOUNDS_CHECK
@@ -62,14 +98,13 @@ __global__ void __launch_bounds__(kThreads) gather_ranks_kernel(const Args a)
 
 cudaError_t occupancy(int* blocks_per_sm)
 {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, gather_ranks_kernel, kThreads, 0);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, layer_gather_kernel, kThreads, 0);
 }
 
 cudaError_t launch(const Args& a, int grid, cudaStream_t s)
 {
     if (a.n_tiles <= 0 || grid <= 0) return cudaSuccess;
-    gather_ranks_kernel<<<grid, kThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return zk::launch_pdl(layer_gather_kernel, dim3(grid), dim3(kThreads), 0, s, a);
 }
 
 }  // namespace zg

@@ -24,8 +24,22 @@ struct Run {
 };
 static_assert(sizeof(Run) == 48, "run layout");
 
-constexpr int64_t kTile = 8192;  // elements per tile (16 KB of fp16)
+#ifndef ZG_TILE
+#define ZG_TILE 8192
+#endif
+#ifndef ZG_UNROLL
+#define ZG_UNROLL 4
+#endif
+#ifndef ZG_STREAMING
+#define ZG_STREAMING 0
+#endif
+#ifndef ZG_MIN_BLOCKS
+#define ZG_MIN_BLOCKS 4
+#endif
+constexpr int64_t kTile = ZG_TILE;  // elements per tile (16 KB of fp16)
 constexpr int kThreads = 256;
+constexpr int kUnroll = ZG_UNROLL;  // 16-byte loads in flight per thread
+constexpr int kMinBlocks = ZG_MIN_BLOCKS;  // resident blocks per SM the registers are capped for
 
 struct Args {
     const Run* runs;

@@ -61,8 +61,24 @@ struct alignas(16) Ctrl {
     int good;            //   current run of good steps
     int cur;             // live state buffer
     int fused;           // 1: a step writes the other buffer, switched on commit
-    int pad[3];
+    // the next step's binary32 constants, written by zero_async_begin and by
+    // each commit (ctrl_next_constants), so that the step kernel loads three
+    // values instead of deriving them in double in every thread
+    float inv_scale, bc1, bc2;
 };
+static_assert(sizeof(Ctrl) == 80, "Ctrl layout");
+
+// inv_scale = (float)(1 / (double)scale); bc_k = (float)(1 - beta_k^(t+1)),
+// beta_k^(t+1) the (t+1)-fold double product continued from p_k: the same
+// operations as the synchronous step's host code, so the results are equal.
+__host__ __device__ inline void ctrl_next_constants(Ctrl* c)
+{
+    const double p1 = c->p1 * (double)c->b1;
+    const double p2 = c->p2 * (double)c->b2;
+    c->bc1 = (float)(1.0 - p1);
+    c->bc2 = (float)(1.0 - p2);
+    c->inv_scale = (float)(1.0 / (double)c->scale);
+}
 
 struct StepArgs {
     const SegDesc* segs;
@@ -155,35 +171,13 @@ constexpr int kPassUpdate = 1;  // reduced gradient, m, v, weight in; m, v, (mas
 // update pass is store-heavy with many outputs: the shape of the fused step
 inline TmaShape tma_pass_shape(int mode, int n_out) { return mode == kPassReduce ? kTmaDeep : tma_shape(n_out); }
 
-// The stage-3 layer gather with bulk copies: each run (one rank's chunk of one
-// tensor) is copied shard -> output through shared memory in tiles of
-// kGatherTile elements, kGatherStages tiles in flight per CTA. TmaRun fields:
-// grad_begin = source (shard) index, out_begin = destination index.
-#ifndef ZK_GATHER_TILE
-#define ZK_GATHER_TILE 8192
-#endif
-#ifndef ZK_GATHER_STAGES
-#define ZK_GATHER_STAGES 3
-#endif
-constexpr int kGatherTile = ZK_GATHER_TILE;
-constexpr int kGatherStages = ZK_GATHER_STAGES;
-
-struct TmaGatherArgs {
-    const TmaRun* runs;
-    int n_runs;
-    long long n_tiles;
-    long long n_scal;
-    const uint16_t* src;
-    uint16_t* dst;
-    unsigned* err;
-    unsigned wait_rounds;
-    long long hold_tile;
-    long long src_len, dst_len;  // element extents (bounds-checked build)
-};
-
 // try_wait rounds (each may suspend about a microsecond) before a wait of the
 // TMA kernels gives up: a few seconds, far beyond any legitimate wait.
 constexpr unsigned kTmaWaitRounds = 1u << 22;
+// Error-word bits set by the in-place update pass of the two-pass TMA step
+// (its failed waits; every other kernel uses the bits below 64).
+constexpr int kErrUpdateShift = 6;
+constexpr unsigned kErrUpdate = 7u << kErrUpdateShift;
 
 enum Kernel : int {
     K_STEP_FUSED = 0,  // reduce + unscale + flag + Adam into the next buffer + fp16 write-back
@@ -210,14 +204,12 @@ cudaError_t launch_commit(Ctrl* ctrl, unsigned* flag, const unsigned* err, cudaS
 // shape and nd ranks, launch.
 cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);
 cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s);
-cudaError_t tma_gather_prepare(int* blocks_per_sm);
 // Two-pass step with TMA staging: attribute set-up and blocks per SM of the
 // two passes (bf16: the bfloat16 codec without master), launch of one pass.
 // Both use TmaArgs; the update pass returns at once if the overflow word holds
 // the call's id or the error word is set.
 cudaError_t tma_pass_prepare(int nd, int n_out, bool bf16, int* occ_reduce, int* occ_update);
 cudaError_t launch_pass_tma(int mode, const TmaArgs& a, int grid, cudaStream_t s, bool bf16);
-cudaError_t launch_gather_tma(const TmaGatherArgs& a, int grid, cudaStream_t s);
 int step_smem_bytes(int nd, int n_out);
 
 }  // namespace zk

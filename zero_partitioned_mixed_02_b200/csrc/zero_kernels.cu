@@ -238,6 +238,7 @@ __global__ void commit_kernel(Ctrl* c, unsigned* flag, const unsigned* err)
             c->good = 0;
         }
     }
+    ctrl_next_constants(c);
     *flag = 0;
 }
 

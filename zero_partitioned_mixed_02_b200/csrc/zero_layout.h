@@ -28,12 +28,7 @@ struct Unit {
     int64_t n_chunks = 0;
     int64_t flat_begin = 0;
     int64_t numel = 0;
-    bool tma_ok = false;  // bulk-copy gather table built (TMA variant, runs in 16-byte phase)
-    int64_t tma_run0 = 0;
-    int64_t tma_n_runs = 0;
-    int64_t tma_tiles = 0;
-    int64_t tma_scal = 0;
-    // stage-3 rank view: the unit's runs from the Nd ranks' shards
+    // the unit's runs from the Nd ranks' shards (the layer gather's table)
     int64_t rank_run0 = 0;
     int64_t rank_n_runs = 0;
     int64_t rank_tiles = 0;
@@ -53,10 +48,9 @@ struct Layout {
     std::vector<int64_t> shard_begin, shard_len;  // per rank, in state elements
     std::vector<zk::SegDesc> step_segs;
     int64_t step_chunks = 0;
-    std::vector<zk::SegDesc> gather_segs;
-    std::vector<zk::TmaRun> tma_gather;  // TMA variant: bulk-copy gather runs of all units
+    std::vector<zk::SegDesc> gather_segs;  // the offloaded step's layer gather (one shard array)
     std::vector<Unit> units;
-    std::vector<zg::Run> rank_gather;  // stage-3 rank view: gather runs of all units
+    std::vector<zg::Run> rank_gather;  // stage 3: the layer gathers' runs of all units, by source rank
     std::vector<zk::TmaRun> tma_runs;  // TMA variants, when every run is eligible
     bool tma_ok = false;
     zk::TmaShape tma_shape = zk::kTmaDeep;
@@ -66,7 +60,7 @@ struct Layout {
     zk::TmaShape tma_shape_r = zk::kTmaDeep;
     int64_t tma_tiles_r = 0, tma_scal_r = 0;
     int64_t off_flag = 0, off_grad_tab = 0, off_out_tab = 0, off_step_segs = 0,
-            off_gather_segs = 0, off_tma_runs = -1, off_tma_runs_r = -1, off_tma_gather = -1, off_reduced = -1,
+            off_tma_runs = -1, off_tma_runs_r = -1, off_reduced = -1,
             off_shard16 = -1, off_shard_tab = -1, off_rank_gather = -1,
             total = 0;
     int64_t off_state[2][3] = {{-1, -1, -1}, {-1, -1, -1}};

@@ -193,111 +193,6 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicMax(b.flag, b.call_id);
 }
 
-__device__ __forceinline__ void bulk_s2g(void* dst, unsigned src, unsigned bytes)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Stage-3 layer gather. One warp per CTA; lane 0 keeps kGatherStages - 1
-// tile loads ahead of the store it issues from the oldest landed stage.
-// Before a stage is reloaded, the store that read it must have finished
-// reading shared memory. All waits are bounded; a CTA that gives up sets the
-// error word, stops issuing and drains what it issued.
-__global__ void __launch_bounds__(32) gather_tma_kernel(const TmaGatherArgs a)
-{
-    extern __shared__ __align__(128) char smem[];
-    constexpr int S = kGatherStages;
-    const unsigned full0 = smem_u32(smem);
-    char* stage0 = smem + 128;
-    const int lane = threadIdx.x;
-    if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
-    if (lane == 0) {
-        // this CTA's tiles are t = blockIdx.x + i * gridDim.x, i = 0 .. n_mine - 1
-        const long long n_mine =
-            a.n_tiles > blockIdx.x ? (a.n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-        int r = 0;
-        long long lo = 0, hi = 0;
-        long long issued = 0;   // loads issued
-        bool failed = false;
-        struct Tile { long long s, d; unsigned bytes; } tiles[S];
-        for (long long i = 0; i < n_mine && !failed; ++i) {
-            // keep S - 1 loads ahead of the store of tile i
-            while (issued < n_mine && issued < i + S) {
-                const int st = (int)(issued % S);
-                if (issued >= S) bulk_wait_read_all();  // the store that read stage st is done reading
-                const long long t = blockIdx.x + issued * gridDim.x;
-                if (t < lo || t >= hi) {
-                    r = find_tma_run<&TmaRun::tile_begin>(a.runs, a.n_runs, t);
-                    lo = a.runs[r].tile_begin;
-                    hi = (r + 1 < a.n_runs) ? a.runs[r + 1].tile_begin : a.n_tiles;
-                }
-                const TmaRun& run = a.runs[r];
-                const long long body = run.len - run.head - run.tail;
-                const long long e0 = run.head + (t - run.tile_begin) * kGatherTile;
-                const long long rem = run.head + body - e0;
-                const unsigned n = (unsigned)(rem < kGatherTile ? rem : kGatherTile);
-                tiles[st].s = run.grad_begin + e0;
-                tiles[st].d = run.out_begin + e0;
-                tiles[st].bytes = 2u * n;
-                const unsigned full = full0 + 8 * st;
-                if (!(in_bounds(tiles[st].s, n, a.src_len, a.err) & in_bounds(tiles[st].d, n, a.dst_len, a.err))) {
-                    tiles[st].bytes = 0;  // bounds-checked build: skip the tile
-                    mbar_expect_tx(full, 0u);
-                } else if (t != a.hold_tile) {  // test hook: leave this stage unarmed
-                    mbar_expect_tx(full, 2u * n);
-                    bulk_g2s(smem_u32(stage0 + st * kGatherTile * 2), a.src + tiles[st].s, 2u * n, full);
-                }
-                ++issued;
-            }
-            const int st = (int)(i % S);
-            if (!mbar_wait(full0 + 8 * st, (unsigned)(i / S) & 1u, a.wait_rounds)) {
-                atomicOr(a.err, 8u);
-                failed = true;
-                break;
-            }
-            if (tiles[st].bytes != 0) {
-                bulk_s2g(a.dst + tiles[st].d, smem_u32(stage0 + st * kGatherTile * 2), tiles[st].bytes);
-                bulk_commit();
-            }
-        }
-        // drain: issued loads must land, issued stores must finish, before exit
-        for (long long i = issued - 1; i >= 0 && i >= issued - S; --i)
-            if (!mbar_wait(full0 + 8 * (int)(i % S), (unsigned)(i / S) & 1u, a.wait_rounds)) atomicOr(a.err, 16u);
-        bulk_wait_all();
-    }
-    __syncwarp();
-    // head and tail elements of the runs
-    int r = 0;
-    long long lo = 0, hi = 0;
-    for (long long j = (long long)blockIdx.x * 32 + lane; j < a.n_scal; j += (long long)gridDim.x * 32) {
-        if (j < lo || j >= hi) {
-            r = find_tma_run<&TmaRun::scal_begin>(a.runs, a.n_runs, j);
-            lo = a.runs[r].scal_begin;
-            hi = (r + 1 < a.n_runs) ? a.runs[r + 1].scal_begin : a.n_scal;
-        }
-        const TmaRun& run = a.runs[r];
-        const long long q = j - run.scal_begin;
-        const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
-        if (!(in_bounds(run.grad_begin + e, 1, a.src_len, a.err) & in_bounds(run.out_begin + e, 1, a.dst_len, a.err)))
-            continue;
-        __stcs(reinterpret_cast<unsigned short*>(a.dst + run.out_begin + e),
-               __ldcs(reinterpret_cast<const unsigned short*>(a.src + run.grad_begin + e)));
-    }
-}
-
-constexpr int kGatherSmem = 128 + kGatherStages * kGatherTile * 2;
-
 int smem_bytes(TmaShape sh, int nd) { return kHdrBytes + sh.stages * (nd * sh.tile * 2 + 3 * sh.tile * 4); }
 
 template <bool ASYNC>
@@ -327,19 +222,6 @@ cudaError_t tma_prepare(TmaShape sh, int nd, int* blocks_per_sm)
     if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, fa, (sh.warps + 1) * 32, smem);
     *blocks_per_sm = occ < occ_a ? occ : occ_a;
     return e;
-}
-
-cudaError_t tma_gather_prepare(int* blocks_per_sm)
-{
-    cudaError_t e = cudaFuncSetAttribute(gather_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherSmem);
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, gather_tma_kernel, 32, kGatherSmem);
-}
-
-cudaError_t launch_gather_tma(const TmaGatherArgs& a, int grid, cudaStream_t s)
-{
-    gather_tma_kernel<<<grid, 32, kGatherSmem, s>>>(a);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_step_tma(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s)

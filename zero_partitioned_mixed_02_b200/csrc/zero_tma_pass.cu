@@ -19,6 +19,8 @@
 // C is the element format of the gradients and parameters (F16 with an fp32
 // master, BF16 without one). Every wait is bounded; a warp that gives up sets
 // the error word and leaves its loop; the producer drains its copies in flight.
+// The update pass sets its own bits of the error word (kErrUpdate): its writes
+// are in place, so the host reports such a failure as a partial update.
 // Heads and tails of the runs are scalar items done from global memory. No
 // cluster multicast.
 #include <cuda_bf16.h>
@@ -32,6 +34,13 @@
 
 namespace zk {
 namespace {
+
+// the error-word bits of a failed wait: the update pass's are shifted into kErrUpdate
+template <int MODE>
+__device__ __forceinline__ unsigned err_bits(unsigned bit)
+{
+    return MODE == kPassUpdate ? bit << kErrUpdateShift : bit;
+}
 
 // bytes of one element staged by the pass
 template <int MODE, class C>
@@ -80,7 +89,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) pass_tma_kernel(const Tma
             const int st = it % STAGES;
             const unsigned ph = (unsigned)(it / STAGES) & 1u;
             if (it >= STAGES && !mbar_wait(empty0 + 8 * st, ph ^ 1u, a.wait_rounds)) {
-                atomicOr(a.err, 1u);
+                atomicOr(a.err, err_bits<MODE>(1u));
                 break;
             }
             if (t < lo || t >= hi) {
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) pass_tma_kernel(const Tma
         for (int k = 0; k < STAGES && k < it; ++k) {
             const int i = it - 1 - k;
             if (!mbar_wait(full0 + 8 * (i % STAGES), (unsigned)(i / STAGES) & 1u, a.wait_rounds))
-                atomicOr(a.err, 2u);
+                atomicOr(a.err, err_bits<MODE>(2u));
         }
         return;
     }
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) pass_tma_kernel(const Tma
         const int st = it % STAGES;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (unsigned)(it / STAGES) & 1u, a.wait_rounds));
         if (!ok) {
-            if (lane == 0) atomicOr(a.err, 4u);
+            if (lane == 0) atomicOr(a.err, err_bits<MODE>(4u));
             break;
         }
         const TileDesc d = desc[st];

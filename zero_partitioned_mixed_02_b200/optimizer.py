@@ -20,6 +20,16 @@ import torch
 from . import _abi as A
 
 
+class ZeroPartialUpdateError(A.ZeroError):
+    """The in-place update pass of a two-pass TMA step gave up a bounded wait
+    part of the way (ZERO_ERR_PARTIAL): some elements of the master (without
+    one, the 16-bit weights), m, v and the parameters hold the new step's
+    values, the others the previous step's, and t did not advance. Nothing can
+    be rolled back inside the library; restore the state saved before the step
+    with load_state_dict (which rewrites the parameters as well) and run the
+    step again."""
+
+
 class ZeroAdam:
     def __init__(self, psi: int, nd: int, stage: int, master_init: torch.Tensor,
                  param_bufs: Sequence[torch.Tensor] | None = None, *, rank_view: int = -1,
@@ -54,7 +64,13 @@ class ZeroAdam:
         if len(ptrs) != self.nd:
             raise ValueError(f"expected {self.nd} gradient buffers, got {len(ptrs)}")
         hp = A.zero_hyper(lr, betas[0], betas[1], eps, weight_decay)
-        rc = A.zero_step(self.h, ptrs, loss_scale, hp, self.stream.cuda_stream)
+        try:
+            rc = A.zero_step(self.h, ptrs, loss_scale, hp, self.stream.cuda_stream)
+        except A.ZeroError as e:
+            if e.code == A.ZERO_ERR_PARTIAL:
+                raise ZeroPartialUpdateError(e.code, "ZeroAdam.step: the state is partly updated; restore a "
+                                                     "saved state_dict with load_state_dict") from e
+            raise
         return rc == A.ZERO_SKIPPED
 
     def gather_layer(self, unit: int, out: torch.Tensor) -> None:
@@ -90,17 +106,39 @@ class ZeroAdam:
         n = self.ledger.state_elems
         return self.workspace[off: off + 2 * n].view(torch.int16)
 
+    def weights16(self) -> torch.Tensor:
+        """The 16-bit parameters of the state's elements, in state order, as
+        int16 bits: the shard (stage 3), this rank's partition of its
+        parameter buffer (a rank view), or the first replica (stage 1/2)."""
+        if self.ledger.off_shard16 >= 0:
+            return self.shard16()
+        if self.cfg.c.rank_view >= 0:
+            b = min(self.cfg.c.rank_view * self.ledger.partition_len, self.cfg.c.psi)
+            return self.param_bufs[0].view(torch.int16)[b: b + self.ledger.state_elems]
+        return self.param_bufs[0].view(torch.int16)[: self.ledger.state_elems]
+
     def state_dict(self) -> dict:
-        """Copies of master (None without one), m, v (state order) and the step count."""
+        """Copies of master (None without one), m, v (state order) and the step
+        count. Without a master (bfloat16) it also holds "weights": the
+        bfloat16 parameters widened to float32 (exact), which load_state_dict
+        writes back; a step that stopped part of the way
+        (ZeroPartialUpdateError) may have changed them."""
         w, m, v = self.state()
-        return {"master": None if w is None else w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
+        sd = {"master": None if w is None else w.clone(), "m": m.clone(), "v": v.clone(), "t": self.t}
+        if w is None:
+            sd["weights"] = self.weights16().view(torch.bfloat16).to(torch.float32)
+        return sd
 
     def load_state_dict(self, sd: dict) -> None:
-        tensors = [x for x in (sd["master"], sd["m"], sd["v"]) if x is not None]
+        """Restore master/m/v and t, and rewrite the 16-bit parameters from
+        the master (without a master: from sd["weights"] if present, else
+        they are left as they are)."""
+        w = sd["master"] if sd["master"] is not None else sd.get("weights")
+        tensors = [x for x in (w, sd["m"], sd["v"]) if x is not None]
         for x in tensors:
             if x.dtype != torch.float32 or not x.is_cuda or x.numel() != self.ledger.state_elems:
                 raise ValueError("state tensors must be CUDA float32 of ledger.state_elems elements")
-        w = None if sd["master"] is None else sd["master"].contiguous()
+        w = None if w is None else w.contiguous()
         m, v = sd["m"].contiguous(), sd["v"].contiguous()
         A.zero_set_state(self.h, 0 if w is None else w.data_ptr(), m.data_ptr(), v.data_ptr(), int(sd["t"]),
                          self.stream.cuda_stream)
