@@ -304,6 +304,28 @@ __device__ __forceinline__ Live live_of(const StepArgs& a)
     return L;
 }
 
+// live_of with the live buffer known at compile time (PAR, the asynchronous
+// step's live index; a fused step writes the other buffer): the state pointers
+// are kernel arguments, the constants come from the control block.
+template <bool ASYNC, int PAR>
+__device__ __forceinline__ Live live_at(const StepArgs& a)
+{
+    if (!ASYNC) return live_of<false>(a);
+    Live L;
+    L.c = a.c;
+    const Ctrl* c = a.ctrl;
+    L.c.bc1 = c->bc1;
+    L.c.bc2 = c->bc2;
+    L.c.inv_scale = c->inv_scale;
+    L.w_in = a.st[PAR][0];
+    L.m_in = a.st[PAR][1];
+    L.v_in = a.st[PAR][2];
+    L.w_out = a.st[1 - PAR][0];
+    L.m_out = a.st[1 - PAR][1];
+    L.v_out = a.st[1 - PAR][2];
+    return L;
+}
+
 // C::kMaster false (no fp32 master): K_INIT writes no master, K_UPDATE reads
 // the weight from the first output (the parameter itself) and writes no
 // master; the state buffers hold m and v only.

@@ -28,8 +28,12 @@
 namespace zk {
 namespace {
 
-template <int WARPS, int STAGES, bool ASYNC>
-__global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const TmaArgs a)
+// The kernel body. ASYNC: PAR is the live state buffer, a compile-time
+// index, so that every state pointer is a kernel argument as in the
+// synchronous form (the kernel branches once, uniformly, on the control
+// block's live index).
+template <int WARPS, int STAGES, bool ASYNC, int PAR>
+__device__ __forceinline__ void step_tma_body(const TmaArgs& a)
 {
     static_assert(STAGES <= kMaxStages, "too many stages");
     constexpr int kTmaConsumerWarps = WARPS;
@@ -37,7 +41,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
     constexpr int kTmaTile = WARPS * 32 * kQuad;
     extern __shared__ __align__(128) char smem[];
     const StepArgs& b = a.b;
-    const Live L = live_of<ASYNC>(b);
+    const Live L = live_at<ASYNC, PAR>(b);
     const int nd = b.nd;
     const unsigned full0 = smem_u32(smem);
     const unsigned empty0 = full0 + 8 * kTmaStages;
@@ -191,6 +195,17 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const Tma
 
     // one atomic per consumer warp that saw a non-finite unscaled gradient
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicMax(b.flag, b.call_id);
+}
+
+template <int WARPS, int STAGES, bool ASYNC>
+__global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const TmaArgs a)
+{
+    if (!ASYNC)
+        step_tma_body<WARPS, STAGES, false, 0>(a);
+    else if (a.b.ctrl->cur == 0)
+        step_tma_body<WARPS, STAGES, true, 0>(a);
+    else
+        step_tma_body<WARPS, STAGES, true, 1>(a);
 }
 
 int smem_bytes(TmaShape sh, int nd) { return kHdrBytes + sh.stages * (nd * sh.tile * 2 + 3 * sh.tile * 4); }
