@@ -40,7 +40,7 @@ CSRC = os.path.join(ROOT, "zero_partitioned_mixed_02_b200", "csrc")
 WORKLOADS = {
     "flat-1m": 1, "stress-16m": 2, "gpt2-1.5b": 3, "7.5b-rank-view": 4, "llama-2.7b": 5,
 }
-PROFILE_WORKLOADS = ("flat-64m", "llama-block")
+PROFILE_WORKLOADS = ("flat-64m", "llama-block", "view-1g")
 
 
 def parse_args():
@@ -58,7 +58,8 @@ def parse_args():
                         "no NCCL comparison)")
     p.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PROFILE_WORKLOADS), default="gpt2-1.5b",
                    help="the five configurations, or a small profiling case of their kernels "
-                        "(flat-64m: the stage-2 step at psi = 2^26; llama-block: one Llama block, stage 3)")
+                        "(flat-64m: the stage-2 step at psi = 2^26; llama-block: one Llama block, stage 3; "
+                        "view-1g: the rank view at psi = 2^30, Nd = 64)")
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass", "two-pass-tma"], default="fused-tma")
     p.add_argument("--precision", choices=["fp16", "bf16"], default="fp16",
                    help="bf16: bfloat16 gradients and parameters without fp32 master weights "
@@ -566,7 +567,10 @@ def measure(args, wl_name, variant_name, e2e_steps, world, rank, local, prefetch
     k_s = statistics.mean(kern_ms) / 1e3
     dom_bytes = floor
     achieved = dom_bytes / k_s / 1e9
-    traffic = recorded_traffic(wl_name, variant_name + ("-bf16" if bf16 else ""))
+    # a TMA variant on an ineligible layout (Nd > 16) runs the plain kernel:
+    # its traffic record is the plain variant's
+    ran = variant_name if (A.zero_uses_tma(h) or "tma" not in variant_name) else variant_name.replace("-tma", "")
+    traffic = recorded_traffic(wl_name, ran + ("-bf16" if bf16 else ""))
     codec = ",bf16" if bf16 else ""
     if two_pass and A.zero_uses_tma(h):
         kname = f"pass_tma_kernel<reduce{codec}>+<update{codec}>"

@@ -134,4 +134,13 @@ def llama_block() -> Workload:
                     tensors=t)
 
 
-PROFILE = {"flat-64m": flat_64m, "llama-block": llama_block}
+def view_1g() -> Workload:
+    """The 7.5B running example's single-rank view at psi = 2^30, Nd = 64:
+    partition 0 of 16,777,216 parameters (64 gradient slices of it, 2.1 GB;
+    the fp16 buffer of psi, 2.1 GB; 0.4 GB of state), 2.6 GB moved per step."""
+    return Workload("view-1G-nd64-rank0-view-stage1", psi=1 << 30, nd=64, stage=1, steps=5,
+                    loss_scale=1024.0, grad=normal(1e-3, 1024.0), master=uniform(-0.1, 0.1),
+                    rank_view=0)
+
+
+PROFILE = {"flat-64m": flat_64m, "llama-block": llama_block, "view-1g": view_1g}
