@@ -1,9 +1,9 @@
-// The layer gather of a real stage-3 rank (zero_gather_ranks.h): a copy kernel
-// bound by memory (and, across GPUs, by NVLink) bandwidth. Each block takes
-// tiles of 16 KB in turn; a tile is a piece of one rank's chunk, copied with
-// 16-byte loads and stores where source and destination share their offset
-// within 16 bytes, element by element otherwise. Launched as a programmatic
-// dependent (zero_pdl.cuh), like the emulated layer gather.
+// The stage-3 layer gather (zero_gather_ranks.h), for emulated ranks and for a
+// rank of a real job: a copy kernel bound by memory (and, across GPUs, by
+// NVLink) bandwidth. Each block takes tiles of 16 KB in turn; a tile is a
+// piece of one rank's chunk, copied with 16-byte loads and stores where source
+// and destination share their offset within 16 bytes, element by element
+// otherwise. Launched as a programmatic dependent (zero_pdl.cuh).
 #include "zero_gather_ranks.h"
 #include "zero_pdl.cuh"
 

@@ -1,9 +1,10 @@
-// Layer gather of rank r of a real stage-3 job ([P1] "The part that sounds too
-// good: communication": stage 3 all-gathers each layer's parameters on demand,
+// The stage-3 layer gather ([P1] "The part that sounds too good:
+// communication": stage 3 all-gathers each layer's parameters on demand,
 // forward and backward; [P2] "ZeRO and the Memory Tricks" -- "The
 // Breakthrough"): the fp16 chunks of one layer unit are copied from the Nd
-// ranks' shards (this rank's own and the others', peer-mapped) into one
-// contiguous buffer in tensor order. Internal to libzero.
+// ranks' shards into one contiguous buffer in tensor order. The shards are
+// places in one shard array when the Nd ranks are emulated on one GPU, or a
+// real rank's own shard and the other ranks' (peer-mapped). Internal to libzero.
 #pragma once
 
 #include <cuda_runtime.h>
