@@ -10,26 +10,6 @@
 namespace zg {
 namespace {
 
-// Every element is read and written once: streaming loads and stores
-// (ZG_STREAMING) keep them from displacing reusable lines in L2.
-__device__ __forceinline__ uint4 ld16(const uint4* p)
-{
-#if ZG_STREAMING
-    return __ldcs(p);
-#else
-    return *p;
-#endif
-}
-
-__device__ __forceinline__ void st16(uint4* p, uint4 x)
-{
-#if ZG_STREAMING
-    __stcs(p, x);
-#else
-    *p = x;
-#endif
-}
-
 __device__ __forceinline__ void copy_span(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int64_t n)
 {
     const int bd = blockDim.x;
@@ -48,11 +28,11 @@ __device__ __forceinline__ void copy_span(const uint16_t* __restrict__ src, uint
     for (; i + (kUnroll - 1) * bd < body; i += kUnroll * bd) {  // kUnroll loads in flight per thread
         uint4 x[kUnroll];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) x[k] = ld16(s4 + i + k * bd);
+        for (int k = 0; k < kUnroll; ++k) x[k] = s4[i + k * bd];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) st16(d4 + i + k * bd, x[k]);
+        for (int k = 0; k < kUnroll; ++k) d4[i + k * bd] = x[k];
     }
-    for (; i < body; i += bd) st16(d4 + i, ld16(s4 + i));
+    for (; i < body; i += bd) d4[i] = s4[i];
     for (int64_t j = head + body * 8 + threadIdx.x; j < n; j += bd) dst[j] = src[j];
 }
 
@@ -73,7 +53,8 @@ __device__ __forceinline__ int find_run(const Run* runs, int n_runs, int64_t til
 // of kThreads per SM with kUnroll 16-byte loads in flight per thread (64 KB
 // per SM) measured fastest on the Llama layer walk: more bytes in flight per
 // SM (more blocks, or 8 loads per thread), contiguous spans of tiles per block,
-// and streaming cache hints were all slower.
+// 512-thread blocks, streaming cache hints and the read-only load path were
+// all slower; 128-thread blocks (8 per SM) were the same within noise.
 __global__ void __launch_bounds__(kThreads, kMinBlocks) layer_gather_kernel(const Args a)
 {
     // a programmatic dependent launch: wait for the previous kernel on the stream

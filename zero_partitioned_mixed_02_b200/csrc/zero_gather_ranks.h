@@ -31,9 +31,6 @@ static_assert(sizeof(Run) == 48, "run layout");
 #ifndef ZG_UNROLL
 #define ZG_UNROLL 4
 #endif
-#ifndef ZG_STREAMING
-#define ZG_STREAMING 0
-#endif
 #ifndef ZG_MIN_BLOCKS
 #define ZG_MIN_BLOCKS 4
 #endif
