@@ -62,8 +62,9 @@ def parse_args():
                         "view-1g: the rank view at psi = 2^30, Nd = 64)")
     p.add_argument("--variant", choices=["fused-tma", "fused", "two-pass", "two-pass-tma"], default="fused-tma")
     p.add_argument("--precision", choices=["fp16", "bf16"], default="fp16",
-                   help="bf16: bfloat16 gradients and parameters without fp32 master weights "
-                        "(two-pass variants only; a fused --variant becomes two-pass-tma)")
+                   help="bf16: bfloat16 gradients and parameters without fp32 master weights (the fused "
+                        "variants need a second replica to roll back to: stage 1/2 with Nd >= 2; otherwise a "
+                        "fused --variant becomes two-pass-tma)")
     p.add_argument("--async", dest="async_steps", action="store_true",
                    help="time zero_step_async: steps enqueued back to back, no host sync")
     p.add_argument("--prefetch", action="store_true",
@@ -84,6 +85,12 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
     return p.parse_args()
+
+
+def bf16_fused_eligible(wl) -> bool:
+    """The fused step without an fp32 master needs a second copy of the weights
+    to roll back to: emulated stage 1/2 ranks with Nd >= 2."""
+    return wl.stage <= 2 and wl.rank_view < 0 and wl.nd >= 2
 
 
 def workload(name):
@@ -115,7 +122,11 @@ def algorithmic_bytes(wl, variant, bf16=False):
         state = 24 * n                       # fp32 master, m, v read and written
     params = 2 * n * n_out                   # 16-bit write-back to every replica / the shard
     floor = grads + state + params
-    if variant in ("fused", "fused-tma"):
+    if variant in ("fused", "fused-tma") and bf16:
+        # without a master: the step reads the weight from the last replica and
+        # writes the others; the replica pass then copies one replica (2 + 2 B)
+        per_launch = {"step_kernel<fused,bf16>": floor - 2 * n, "replica_kernel": 4 * n}
+    elif variant in ("fused", "fused-tma"):
         per_launch = {"step_kernel<fused>": floor}
     else:
         per_launch = {"step_kernel<reduce>": grads + 4 * n,
@@ -453,8 +464,8 @@ def measure(args, wl_name, variant_name, e2e_steps, world, rank, local, prefetch
 
     wl = workload(wl_name)
     bf16 = args.precision == "bf16"
-    if bf16 and variant_name in ("fused", "fused-tma"):
-        variant_name = "two-pass-tma"  # without a master only the two-pass step exists
+    if bf16 and variant_name in ("fused", "fused-tma") and not bf16_fused_eligible(wl):
+        variant_name = "two-pass-tma"  # without a master and a second replica: the two-pass step
     variant = {"fused": A.ZERO_VARIANT_FUSED, "two-pass": A.ZERO_VARIANT_TWO_PASS,
                "fused-tma": A.ZERO_VARIANT_FUSED_TMA, "two-pass-tma": A.ZERO_VARIANT_TWO_PASS_TMA}[variant_name]
     two_pass = variant_name.startswith("two-pass")
@@ -558,21 +569,30 @@ def measure(args, wl_name, variant_name, e2e_steps, world, rank, local, prefetch
 
     n, floor, per_launch, gathers = algorithmic_bytes(wl, variant_name, bf16)
     launches_per_step = (2 if two_pass else 1) + len(order)
-    if args.async_steps:  # + the conditional roll-back (fused variants) and the commit kernel
+    if args.async_steps:  # + the conditional roll-back or replica pass (fused variants) and the commit kernel
         launches_per_step += 1 if two_pass else 2
+    elif bf16 and not two_pass:  # + the replica pass the commit launches
+        launches_per_step += 1
     step_s = total_ms / 1e3 / args.steps
     value = whole_job_value(n, args.steps, world, total_ms)
     peak, peak_src = measured_peak()
-    # dominant kernel: the step kernel (both kernels of the two-pass variant timed together)
+    # dominant kernel: the step kernel (both kernels of the two-pass variant
+    # timed together); the fused bfloat16 step's replica pass runs in the
+    # commit, outside the synchronous events (inside the asynchronous ones)
     k_s = statistics.mean(kern_ms) / 1e3
     dom_bytes = floor
+    if bf16 and not two_pass:
+        dom_bytes = per_launch["step_kernel<fused,bf16>"] + (per_launch["replica_kernel"] if args.async_steps else 0)
     achieved = dom_bytes / k_s / 1e9
     # a TMA variant on an ineligible layout (Nd > 16) runs the plain kernel:
     # its traffic record is the plain variant's
     ran = variant_name if (A.zero_uses_tma(h) or "tma" not in variant_name) else variant_name.replace("-tma", "")
     traffic = recorded_traffic(wl_name, ran + ("-bf16" if bf16 else ""))
     codec = ",bf16" if bf16 else ""
-    if two_pass and A.zero_uses_tma(h):
+    if not two_pass and bf16:
+        kname = ("step_tma_kernel<bf16>" if A.zero_uses_tma(h) else "step_kernel<fused,bf16>") + \
+            (" + replica_kernel" if args.async_steps else "")
+    elif two_pass and A.zero_uses_tma(h):
         kname = f"pass_tma_kernel<reduce{codec}>+<update{codec}>"
     elif two_pass:
         kname = f"step_kernel<reduce{codec}>+<update{codec}>"

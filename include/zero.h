@@ -124,9 +124,18 @@ extern "C" {
  * parameter, runs the same binary32 Adam element and rounds the result back
  * to bfloat16 (nearest even) into every replica / the shard. Updates smaller
  * than half a bfloat16 spacing are lost ([P1] "Why you can't just delete the
- * fp32 copies" describes the same loss for fp16). Requires
- * ZERO_VARIANT_TWO_PASS or ZERO_VARIANT_TWO_PASS_TMA (without a master a
- * speculative write cannot be rolled back). master_init of zero_init is rounded to bfloat16; the ledger's master
+ * fp32 copies" describes the same loss for fp16). Without a master a
+ * speculative write could destroy the only copy of the weights, so the fused
+ * variants (ZERO_VARIANT_FUSED, ZERO_VARIANT_FUSED_TMA) exist only where a
+ * second copy does: stage 1/2 with all Nd >= 2 ranks emulated (rank_view =
+ * -1). Their step reads the weight from the last replica and writes the new
+ * one into the other Nd - 1; a replica pass, enqueued by the commit (or by
+ * zero_step_async), then copies replica 0 into the last one, or on overflow
+ * (or a kernel's failed wait) copies the last one's unchanged values back
+ * over the others. Per element that is 4 B more than the floor instead of the
+ * two-pass variants' 8 B of reduced gradient. Every other configuration needs
+ * ZERO_VARIANT_TWO_PASS or ZERO_VARIANT_TWO_PASS_TMA (ZERO_ERR_ARG otherwise).
+ * master_init of zero_init is rounded to bfloat16; the ledger's master
  * offsets are -1 and zero_current_state returns master = NULL; for
  * zero_set_state master may be NULL (the parameters stay as they are) or
  * fp32 values in state order to round into the parameters. */

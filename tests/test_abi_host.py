@@ -222,10 +222,22 @@ def test_bf16_precision_ledger_and_validation():
                                      precision=BF))
     assert list(Lt.exact_bytes) == list(L2.exact_bytes) and Lt.off_reduced > 0
     assert 0 <= Lt.workspace_bytes - L2.workspace_bytes <= 4096
-    for kw in (dict(precision=2), dict(precision=BF, variant=A.ZERO_VARIANT_FUSED),
-               dict(precision=BF, variant=A.ZERO_VARIANT_FUSED_TMA)):
-        with pytest.raises(A.ZeroError) as ei:
-            A.zero_state_bytes(A.Config(psi, nd, 2, **kw))
-        assert ei.value.code == A.ZERO_ERR_ARG
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_state_bytes(A.Config(psi, nd, 2, precision=2))
+    assert ei.value.code == A.ZERO_ERR_ARG
+    # the fused step without a master rolls back from a second copy of the
+    # weights, the last replica: emulated stage 1/2 ranks with Nd >= 2 only;
+    # it keeps two m/v buffers and no reduced-gradient scratch
+    for variant in (A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_FUSED_TMA):
+        for stage in (1, 2):
+            Lf = A.zero_state_bytes(A.Config(psi, nd, stage, variant=variant, tensors=tensors, precision=BF))
+            assert list(Lf.off_master) == [-1, -1] and min(Lf.off_m) >= 0 and min(Lf.off_v) >= 0
+            assert Lf.off_reduced < 0
+            assert list(Lf.exact_bytes) == list(L2.exact_bytes)
+        for bad in (dict(nd=1, stage=2), dict(nd=nd, stage=3), dict(nd=nd, stage=1, rank_view=0)):
+            with pytest.raises(A.ZeroError) as ei:
+                A.zero_state_bytes(A.Config(psi, bad["nd"], bad["stage"], rank_view=bad.get("rank_view", -1),
+                                            variant=variant, tensors=tensors, precision=BF))
+            assert ei.value.code == A.ZERO_ERR_ARG
     with pytest.raises(A.ZeroError):
         A.zero_offload_bytes(A.Config(psi, nd, 2, variant=A.ZERO_VARIANT_TWO_PASS, precision=BF))

@@ -33,6 +33,13 @@ BF = A.ZERO_PRECISION_BF16
 TWO = A.ZERO_VARIANT_TWO_PASS
 TWO_TMA = A.ZERO_VARIANT_TWO_PASS_TMA
 BF_VARIANTS = [TWO, TWO_TMA]
+# the fused step without a master (emulated stage 1/2 ranks, Nd >= 2): the
+# weight is read from the last replica, the new one written to the others,
+# then a replica pass copies it into the last one (or, on overflow, copies
+# the last one's old values back over the others)
+FUSED = A.ZERO_VARIANT_FUSED
+FUSED_TMA = A.ZERO_VARIANT_FUSED_TMA
+BF_FUSED = [FUSED, FUSED_TMA]
 NO_DECAY = A.ZERO_TENSOR_NO_DECAY
 
 
@@ -219,7 +226,55 @@ def test_bf16_subnormal_and_tiny_values():
     _run(c, 2)
 
 
-@pytest.mark.parametrize("variant", BF_VARIANTS)
+@pytest.mark.parametrize("variant", BF_FUSED)
+@pytest.mark.parametrize("stage", [1, 2])
+@pytest.mark.parametrize("nd", [2, 3, 5, 8, 9])
+def test_bf16_fused_grid(nd, stage, variant):
+    rng = np.random.default_rng(11 * nd + stage)
+    for psi in (1, 7, 64, 257, 4099, 70001):
+        _run(Bf16Case(psi, nd, stage, tensors=_tensors(rng, psi), loss_scale=float(2 ** (psi % 9)),
+                      variant=variant), 2)
+
+
+@pytest.mark.parametrize("nd", [2, 4, 8, 16])
+def test_bf16_fused_tma_engages(nd):
+    """The TMA-staged fused kernel with the bfloat16 codec: whole tiles,
+    partial tiles, heads and tails, an excluded tensor."""
+    for psi in (1024, 8 * 1024 * 5 + 200, 1_000_003):
+        cut = psi // 3 // 64 * 64
+        c = Bf16Case(psi, nd, 2, tensors=[(cut, 0), (psi - cut, 0, NO_DECAY)], variant=FUSED_TMA)
+        assert A.zero_uses_tma(c.h)
+        _run(c, 2)
+
+
+@pytest.mark.parametrize("variant", BF_FUSED)
+def test_bf16_fused_skip_restores_every_replica(variant):
+    psi = 20_000
+    assert _run(Bf16Case(psi, 8, 2, variant=variant), 3, inject=[(1, 7, 5, 0x7F80)]) == [False, True, False]
+    assert _run(Bf16Case(psi, 2, 1, variant=variant), 3, inject=[(0, 0, psi - 1, 0xFFC0)]) == [True, False, False]
+
+
+def test_bf16_fused_wait_that_gives_up_is_rolled_back():
+    """A tile left unarmed (no fault): the step returns ZERO_ERR_INTERNAL, the
+    replica pass restores every replica from the last one, m/v do not switch,
+    and the next step equals the oracle's next step."""
+    c = Bf16Case(200_000, 8, 2, variant=FUSED_TMA)
+    assert A.zero_uses_tma(c.h)
+    c.check("after init")
+    c.step(c.grads(0))
+    c.check("after step 0")
+    A.zero_test_hold_tile(c.h, 3, 1 << 14)
+    c.upload(c.grads(1))
+    with pytest.raises(A.ZeroError) as ei:
+        A.zero_step(c.h, [g.data_ptr() for g in c.g_dev], c.loss_scale, hyper(**c.hp), c.stream)
+    assert ei.value.code == A.ZERO_ERR_INTERNAL
+    c.check("after the failed step: unchanged")
+    c.step(c.grads(2))
+    c.check("after the next step")
+    c.close()
+
+
+@pytest.mark.parametrize("variant", BF_VARIANTS + BF_FUSED)
 def test_bf16_asynchronous_steps(variant):
     c = Bf16Case(50_000, 4, 2, tensors=[(30_000, 0), (20_000, 1, NO_DECAY)], loss_scale=1.0, variant=variant)
     c.check("after init")
@@ -242,10 +297,11 @@ def test_bf16_asynchronous_steps(variant):
     c.close()
 
 
-def test_bf16_set_state():
+@pytest.mark.parametrize("variant", [TWO, FUSED_TMA])
+def test_bf16_set_state(variant):
     """Resume: m, v and t restored; the parameters either stay (master NULL)
     or are rewritten from fp32 values rounded to bfloat16."""
-    c = Bf16Case(10_000, 4, 2)
+    c = Bf16Case(10_000, 4, 2, variant=variant)
     _ = [c.step(c.grads(s)) for s in range(2)]
     n = c.L.state_elems
     rng = np.random.default_rng(1)
@@ -263,10 +319,11 @@ def test_bf16_set_state():
     c.close()
 
 
-def test_bf16_async_step_in_a_cuda_graph():
+@pytest.mark.parametrize("variant", [TWO_TMA, FUSED_TMA])
+def test_bf16_async_step_in_a_cuda_graph(variant):
     """The bfloat16 step without master, asynchronous and captured once in a
     CUDA graph, replayed with fresh gradients (one overflowing)."""
-    c = Bf16Case(40_000, 4, 2, tensors=[(24_000, 0), (16_000, 0, NO_DECAY)], variant=TWO_TMA)
+    c = Bf16Case(40_000, 4, 2, tensors=[(24_000, 0), (16_000, 0, NO_DECAY)], variant=variant)
     c.check("after init")
     cap = torch.cuda.Stream()
     with torch.cuda.stream(cap):

@@ -36,7 +36,8 @@ def jobs(draw):
         tensors.append((n, u, draw(st.sampled_from([0, A.ZERO_TENSOR_NO_DECAY]))))
     stage = draw(st.integers(1, 3))
     bf16 = draw(st.booleans())
-    variant = draw(st.sampled_from(VARIANTS[1::2] if bf16 else VARIANTS))
+    # without a master the fused step exists for emulated stage 1/2 ranks, Nd >= 2
+    variant = draw(st.sampled_from(VARIANTS if (not bf16 or (stage <= 2 and nd >= 2)) else VARIANTS[1::2]))
     scale = float(2 ** draw(st.integers(0, 14)))
     return nd, tensors, stage, variant, bf16, scale
 

@@ -148,14 +148,20 @@ def test_offload_object_equals_device_object():
 
 
 def test_zero_adam_bf16_object():
-    """ZeroAdam with precision=bf16 and the default variant runs the two-pass
-    TMA step; its state has no master; three steps equal the oracle."""
+    """ZeroAdam with precision=bf16 and the default variant runs the fused TMA
+    step (stage 2, Nd = 4: the last replica is its roll-back copy); its state
+    has no master; three steps equal the oracle. Where no second replica
+    exists (one rank) the default becomes the two-pass TMA step."""
     from zero_partitioned_mixed_02_b200 import ZeroAdam
     psi, nd = 20_000, 4
     w0 = S.host_f32(psi, 0, S.key(3, S.STREAM_MASTER, 0, 0), S.uniform(-1.0, 1.0))
     reps = [torch.zeros(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]
     opt = ZeroAdam(psi, nd, 2, torch.from_numpy(w0.copy()).cuda(), reps, precision=A.ZERO_PRECISION_BF16)
-    assert opt.cfg.c.variant == A.ZERO_VARIANT_TWO_PASS_TMA
+    assert opt.cfg.c.variant == A.ZERO_VARIANT_FUSED_TMA
+    one = ZeroAdam(64, 1, 2, torch.zeros(64, dtype=torch.float32, device="cuda"),
+                   [torch.zeros(64, dtype=torch.int16, device="cuda")], precision=A.ZERO_PRECISION_BF16)
+    assert one.cfg.c.variant == A.ZERO_VARIANT_TWO_PASS_TMA
+    one.close()
     w16 = Z.bf16_from_f32(w0)
     m, v, t = np.zeros(psi, np.float32), np.zeros(psi, np.float32), 0
     grads = [torch.empty(psi, dtype=torch.int16, device="cuda") for _ in range(nd)]

@@ -70,8 +70,12 @@ int zl::build_layout(const zero_config* cfg, Layout* L)
         return ZERO_ERR_ARG;
     if (cfg->n_tensors < 0) return ZERO_ERR_ARG;
     if (cfg->precision != ZERO_PRECISION_FP16 && cfg->precision != ZERO_PRECISION_BF16) return ZERO_ERR_ARG;
-    // without a master nothing can be rolled back: the two-pass step only
-    if (cfg->precision == ZERO_PRECISION_BF16 && is_fused(cfg->variant)) return ZERO_ERR_ARG;
+    // without a master the fused step needs a second copy of the old weights
+    // to roll back to: the last replica of emulated stage 1/2 ranks (Nd >= 2);
+    // anything else runs the two-pass step only
+    if (cfg->precision == ZERO_PRECISION_BF16 && is_fused(cfg->variant) &&
+        !(cfg->rank_view < 0 && cfg->stage <= 2 && cfg->nd >= 2))
+        return ZERO_ERR_ARG;
     if (cfg->rank_view < -1 || cfg->rank_view >= cfg->nd) return ZERO_ERR_ARG;
     // a stage-3 rank writes only its own fp16 shard
     if (cfg->rank_view >= 0 && cfg->stage == 3 && cfg->view_outputs > 1) return ZERO_ERR_ARG;
@@ -462,6 +466,16 @@ bool real_rank(const Layout& L) { return L.view >= 0 && (L.n_out > 1 || L.stage 
 
 bool defers_update(const Layout& L) { return real_rank(L) && !is_fused(L.variant); }
 
+// The fused step without a master reads the weight from the last replica and
+// writes all the others; K_REPLICA then completes or restores them.
+void set_replica_roles(const Layout& L, zk::StepArgs& a)
+{
+    if (is_fused(L.variant) && L.bf16) {
+        a.w_src = a.n_out - 1;
+        a.keep_last = 1;
+    }
+}
+
 int cuda_fail(zero_handle* h, cudaError_t e)
 {
     if (h) h->last_cuda = (int)e;
@@ -541,7 +555,7 @@ cudaError_t launch_tma_step(zero_handle* h, const zk::StepArgs& a, int64_t hold_
         ta.n_scal = L.tma_scal;
         const int64_t cap = (int64_t)h->sms * h->occ_tma;
         const int64_t want = std::max<int64_t>(1, std::max(L.tma_tiles, (L.tma_scal + 255) / 256));
-        return zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s);
+        return zk::launch_step_tma(L.tma_shape, ta, (int)std::min(want, cap), s, L.bf16);
     }
     if (passes & kRunReduce) {
         ta.runs = h->d_tma_runs_r;
@@ -686,7 +700,7 @@ ZERO_API int zero_init(const zero_config* cfg, void* workspace, size_t workspace
     if (L.tma_ok) {
         h->d_tma_runs = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs);
         if (is_fused(L.variant)) {
-            e = zk::tma_prepare(L.tma_shape, L.nd, &h->occ_tma);
+            e = zk::tma_prepare(L.tma_shape, L.nd, L.bf16, &h->occ_tma);
             h->occ_tma_r = h->occ_tma;
         } else {
             h->d_tma_runs_r = reinterpret_cast<zk::TmaRun*>(h->ws + L.off_tma_runs_r);
@@ -823,6 +837,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
 
     const bool fused = is_fused(L.variant);
     const int nxt = fused ? 1 - h->cur : h->cur;
+    set_replica_roles(L, a);
     a.w_in = h->state(h->cur, 0);
     a.m_in = h->state(h->cur, 1);
     a.v_in = h->state(h->cur, 2);
@@ -837,7 +852,7 @@ ZERO_API int zero_step_launch(zero_handle* h, const uint16_t* const* grads, floa
                                 passes);
             h->hold_tile = -1;
         } else if (fused) {
-            e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
+            e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s, L.bf16);
         } else {
             a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
             e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s, L.bf16);
@@ -875,12 +890,18 @@ ZERO_API int zero_step_commit(zero_handle* h, void* stream, int* skipped)
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(h, e);
     const bool kernel_error = h->host_flag[1] != 0;
+    if (is_fused(L.variant) && L.bf16 && L.step_chunks > 0) {
+        // without a master: bring the last replica up to date, or on overflow
+        // restore the others from it (the kernel reads the same words)
+        e = zk::launch_step(zk::K_REPLICA, h->args, grid_for(h, zk::K_REPLICA, L.step_chunks), s, true);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+    }
     if (h->host_flag[0] == h->call_id || kernel_error) {
         // Overflow (or a kernel that gave up a wait): the state buffers do not
         // switch (fused) or were never written (two-pass). The fused pass
         // already wrote fp16 parameters, so rewrite them from the unchanged
-        // master.
-        if (is_fused(L.variant) && L.step_chunks > 0) {
+        // master (without a master the replica pass above restored them).
+        if (is_fused(L.variant) && !L.bf16 && L.step_chunks > 0) {
             zk::StepArgs a = h->args;
             a.w_in = h->state(h->cur, 0);
             e = zk::launch_step(zk::K_CAST, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
@@ -992,12 +1013,13 @@ ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
     for (int b = 0; b < 2; ++b)
         for (int k = 0; k < 3; ++k) a.st[b][k] = h->state(b < nb ? b : 0, k);
     const bool fused = is_fused(L.variant);
+    set_replica_roles(L, a);
     cudaError_t e;
     if (h->use_tma) {
         if (!fused) a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
         e = launch_tma_step(h, a, -1, zk::kTmaWaitRounds, s);
     } else if (fused) {
-        e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s);
+        e = zk::launch_step(zk::K_STEP_FUSED, a, grid_for(h, zk::K_STEP_FUSED, L.step_chunks), s, L.bf16);
     } else {
         a.red = reinterpret_cast<float*>(h->ws + L.off_reduced);
         e = zk::launch_step(zk::K_REDUCE, a, grid_for(h, zk::K_REDUCE, L.step_chunks), s, L.bf16);
@@ -1005,8 +1027,11 @@ ZERO_API int zero_step_async(zero_handle* h, const zero_hyper* hp, void* stream)
             e = zk::launch_step(zk::K_UPDATE, a, grid_for(h, zk::K_UPDATE, L.step_chunks), s, L.bf16);
     }
     // the fused passes wrote fp16 parameters: rewrite them from the unchanged
-    // master if the step overflowed (the kernel returns at once otherwise)
-    if (e == cudaSuccess && fused)
+    // master if the step overflowed (the kernel returns at once otherwise);
+    // without a master the replica pass restores or completes them
+    if (e == cudaSuccess && fused && L.bf16)
+        e = zk::launch_step(zk::K_REPLICA, a, grid_for(h, zk::K_REPLICA, L.step_chunks), s, true);
+    else if (e == cudaSuccess && fused)
         e = zk::launch_step(zk::K_CAST_IF, a, grid_for(h, zk::K_CAST, L.step_chunks), s);
     if (e == cudaSuccess) e = zk::launch_commit(h->d_ctrl, h->d_flag, h->d_flag + 1, s);
     return e == cudaSuccess ? ZERO_OK : cuda_fail(h, e);

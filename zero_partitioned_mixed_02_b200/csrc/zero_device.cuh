@@ -326,9 +326,10 @@ __device__ __forceinline__ Live live_at(const StepArgs& a)
     return L;
 }
 
-// C::kMaster false (no fp32 master): K_INIT writes no master, K_UPDATE reads
-// the weight from the first output (the parameter itself) and writes no
-// master; the state buffers hold m and v only.
+// C::kMaster false (no fp32 master): K_INIT writes no master, K_UPDATE and
+// K_STEP_FUSED read the weight from output a.w_src (the parameter itself)
+// and write no master, K_STEP_FUSED leaves the last a.keep_last outputs
+// alone; the state buffers hold m and v only.
 template <int K, class C = F16>
 __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, const uint16_t* const* gp,
                                             uint16_t* const* op, const SegDesc& d, long long e,
@@ -351,7 +352,7 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, co
             if (C::kMaster)
                 w = __ldcs(L.w_in + si);
             else
-                w = C::dec(__ldcs(reinterpret_cast<const unsigned short*>(op[0] + oi)));
+                w = C::dec(__ldcs(reinterpret_cast<const unsigned short*>(op[a.w_src] + oi)));
             m = __ldcs(L.m_in + si);
             v = __ldcs(L.v_in + si);
         }
@@ -370,7 +371,8 @@ __device__ __forceinline__ void step_scalar(const StepArgs& a, const Live& L, co
         __stcs(L.v_out + si, v);
     }
     const unsigned short h = C::enc(w);
-    for (int k = 0; k < a.n_out; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);
+    const int n_write = K == K_STEP_FUSED ? a.n_out - a.keep_last : a.n_out;
+    for (int k = 0; k < n_write; ++k) __stcs(reinterpret_cast<unsigned short*>(op[k] + oi), h);
 }
 
 // Largest run index whose first chunk is <= c.

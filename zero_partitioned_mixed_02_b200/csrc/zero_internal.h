@@ -107,6 +107,12 @@ struct StepArgs {
     // element extents of the buffers (grads and master_init; state arrays and
     // red; outputs), checked by the bounds-checked build (ZK_BOUNDS_CHECK)
     long long grad_len, state_len, out_len;
+    // without an fp32 master: the output the weight is read from (K_UPDATE,
+    // K_STEP_FUSED), and how many of the last outputs K_STEP_FUSED leaves
+    // unwritten (the fused bfloat16 step keeps the last output, the backup
+    // K_REPLICA restores from or brings up to date; 0 elsewhere)
+    int w_src;
+    int keep_last;
 };
 
 struct GatherArgs {
@@ -187,7 +193,9 @@ enum Kernel : int {
     K_INIT = 4,        // master = master_init, m = v = 0, fp16 write-back
     K_GATHER = 5,      // stage-3 layer gather
     K_CAST_IF = 6,     // K_CAST only if the step overflowed (asynchronous step)
-    K_COUNT = 7
+    K_REPLICA = 7,     // fused bfloat16 step: on overflow (or a failed wait) copy the last output
+                       // over the others, else copy output 0 into the last one
+    K_COUNT = 8
 };
 
 // Blocks per SM the kernel reaches with `smem` bytes of dynamic shared memory
@@ -202,8 +210,8 @@ cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int grid, cuda
 cudaError_t launch_commit(Ctrl* ctrl, unsigned* flag, const unsigned* err, cudaStream_t s);
 // TMA-staged fused step: one-time attribute set-up and blocks per SM for the
 // shape and nd ranks, launch.
-cudaError_t tma_prepare(TmaShape shape, int nd, int* blocks_per_sm);
-cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s);
+cudaError_t tma_prepare(TmaShape shape, int nd, bool bf16, int* blocks_per_sm);
+cudaError_t launch_step_tma(TmaShape shape, const TmaArgs& a, int grid, cudaStream_t s, bool bf16);
 // Two-pass step with TMA staging: attribute set-up and blocks per SM of the
 // two passes (bf16: the bfloat16 codec without master), launch of one pass.
 // Both use TmaArgs; the update pass returns at once if the overflow word holds

@@ -67,8 +67,8 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const
             if (C::kMaster) {
                 ld_pair(L.w_in, sa, sb, hb, w);
             } else {
-                unpack_as<C>(ld_hq_any(op[0] + oa), w);
-                unpack_as<C>(hb ? ld_hq_any(op[0] + ob) : make_uint2(0u, 0u), w + 4);
+                unpack_as<C>(ld_hq_any(op[a.w_src] + oa), w);
+                unpack_as<C>(hb ? ld_hq_any(op[a.w_src] + ob) : make_uint2(0u, 0u), w + 4);
             }
             ld_pair(L.m_in, sa, sb, hb, m);
             ld_pair(L.v_in, sa, sb, hb, v);
@@ -94,7 +94,8 @@ __device__ __forceinline__ void step_vec(const StepArgs& a, const Live& L, const
         st_pair(L.v_out, sa, sb, hb, v);
     }
     const uint2 h0 = pack_as<C>(w), h1 = pack_as<C>(w + 4);
-    for (int k = 0; k < a.n_out; ++k) {
+    const int n_write = K == K_STEP_FUSED ? a.n_out - a.keep_last : a.n_out;
+    for (int k = 0; k < n_write; ++k) {
         st_hq(op[k] + oa, h0);
         if (hb) st_hq(op[k] + ob, h1);
     }
@@ -184,6 +185,40 @@ __global__ void __launch_bounds__(kThreads, ZK_MIN_BLOCKS) step_kernel(const Ste
     }
 }
 
+// The commit pass of the fused step without an fp32 master (the 16-bit
+// parameters are the only copy of the weights): the step kernel read the
+// weight from the last output and wrote the new one into all the others. On
+// overflow, or if a kernel gave up a wait, the last output's (old) values are
+// copied back over the others; otherwise output 0's (new) values are copied
+// into the last one. 16-bit patterns are copied as they are.
+__global__ void __launch_bounds__(kThreads) replica_kernel(const StepArgs a)
+{
+    const bool roll_back = *reinterpret_cast<volatile const unsigned*>(a.flag) == a.call_id ||
+                           *reinterpret_cast<volatile const unsigned*>(a.err) != 0;
+    const int last = a.n_out - 1;
+    const int src = roll_back ? last : 0;
+    const int d0 = roll_back ? 0 : last, d1 = roll_back ? last : a.n_out;
+    const uint16_t* sp = a.outs[src];
+    walk(
+        a.segs, a.n_segs, a.n_chunks,
+        [&](const SegDesc& d, const Pair& p) {
+            const long long oa = d.out_begin + p.ea, ob = d.out_begin + p.eb;
+            if (!(in_bounds(oa, 4, a.out_len, a.err) & (!p.hb || in_bounds(ob, 4, a.out_len, a.err)))) return;
+            const uint2 h0 = ld_hq_any(sp + oa);
+            const uint2 h1 = p.hb ? ld_hq_any(sp + ob) : make_uint2(0u, 0u);
+            for (int k = d0; k < d1; ++k) {
+                st_hq(a.outs[k] + oa, h0);
+                if (p.hb) st_hq(a.outs[k] + ob, h1);
+            }
+        },
+        [&](const SegDesc& d, long long e) {
+            const long long oi = d.out_begin + e;
+            if (!in_bounds(oi, 1, a.out_len, a.err)) return;
+            const unsigned short h = __ldcs(reinterpret_cast<const unsigned short*>(sp + oi));
+            for (int k = d0; k < d1; ++k) __stcs(reinterpret_cast<unsigned short*>(a.outs[k] + oi), h);
+        });
+}
+
 __global__ void __launch_bounds__(kThreads) gather_kernel(const GatherArgs a)
 {
     walk(
@@ -246,6 +281,8 @@ const void* kernel_ptr(Kernel k, bool bf16)
 {
     if (bf16) {
         switch (k) {
+            case K_STEP_FUSED: return reinterpret_cast<const void*>(&step_kernel<K_STEP_FUSED, false, BF16>);
+            case K_REPLICA: return reinterpret_cast<const void*>(&replica_kernel);
             case K_REDUCE: return reinterpret_cast<const void*>(&step_kernel<K_REDUCE, false, BF16>);
             case K_UPDATE: return reinterpret_cast<const void*>(&step_kernel<K_UPDATE, false, BF16>);
             case K_CAST: return reinterpret_cast<const void*>(&step_kernel<K_CAST, false, BF16>);
@@ -285,8 +322,13 @@ cudaError_t launch_step(Kernel k, const StepArgs& a, int grid, cudaStream_t s, b
     const int smem = step_smem_bytes(a.nd, a.n_out);
     const bool as = a.ctrl != nullptr;
     if (bf16) {
-        // the step without a master runs the two passes only (nothing to roll back)
+        // without a master: the two passes, or the fused step with its replica pass
         switch (k) {
+            case K_STEP_FUSED:
+                if (as) step_kernel<K_STEP_FUSED, true, BF16><<<grid, kThreads, smem, s>>>(a);
+                else step_kernel<K_STEP_FUSED, false, BF16><<<grid, kThreads, smem, s>>>(a);
+                break;
+            case K_REPLICA: replica_kernel<<<grid, kThreads, 0, s>>>(a); break;
             case K_REDUCE:
                 if (as) step_kernel<K_REDUCE, true, BF16><<<grid, kThreads, smem, s>>>(a);
                 else step_kernel<K_REDUCE, false, BF16><<<grid, kThreads, smem, s>>>(a);

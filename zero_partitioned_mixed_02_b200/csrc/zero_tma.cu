@@ -32,13 +32,17 @@ namespace {
 // index, so that every state pointer is a kernel argument as in the
 // synchronous form (the kernel branches once, uniformly, on the control
 // block's live index).
-template <int WARPS, int STAGES, bool ASYNC, int PAR>
+// C: the element format (F16 with an fp32 master; BF16 without one, whose
+// weight is read from output b.w_src and written to all outputs but the last
+// b.keep_last, the copy a skipped step is restored from).
+template <int WARPS, int STAGES, bool ASYNC, int PAR, class C>
 __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
 {
     static_assert(STAGES <= kMaxStages, "too many stages");
     constexpr int kTmaConsumerWarps = WARPS;
     constexpr int kTmaStages = STAGES;
     constexpr int kTmaTile = WARPS * 32 * kQuad;
+    constexpr int kWBytes = C::kMaster ? 4 : 2;  // bytes of the staged weight
     extern __shared__ __align__(128) char smem[];
     const StepArgs& b = a.b;
     const Live L = live_at<ASYNC, PAR>(b);
@@ -46,7 +50,7 @@ __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
     const unsigned full0 = smem_u32(smem);
     const unsigned empty0 = full0 + 8 * kTmaStages;
     TileDesc* desc = reinterpret_cast<TileDesc*>(smem + 16 * kTmaStages);
-    const int stage_bytes = nd * kTmaTile * 2 + 3 * kTmaTile * 4;
+    const int stage_bytes = nd * kTmaTile * 2 + kTmaTile * (kWBytes + 8);
     char* stage0 = smem + kHdrBytes;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -97,13 +101,16 @@ __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
                 mbar_expect_tx(full, 0u);
                 continue;
             }
-            mbar_expect_tx(full, (unsigned)n * (unsigned)(2 * nd + 12));
+            mbar_expect_tx(full, (unsigned)n * (unsigned)(2 * nd + kWBytes + 8));
             for (int k = 0; k < nd; ++k)
                 bulk_g2s(smem_u32(sp + k * kTmaTile * 2), b.grads[k] + d.gi, 2u * n, full);
             char* sw = sp + nd * kTmaTile * 2;
-            bulk_g2s(smem_u32(sw), L.w_in + d.si, 4u * n, full);
-            bulk_g2s(smem_u32(sw + kTmaTile * 4), L.m_in + d.si, 4u * n, full);
-            bulk_g2s(smem_u32(sw + 2 * kTmaTile * 4), L.v_in + d.si, 4u * n, full);
+            if (C::kMaster)
+                bulk_g2s(smem_u32(sw), L.w_in + d.si, 4u * n, full);
+            else
+                bulk_g2s(smem_u32(sw), b.outs[b.w_src] + d.oi, 2u * n, full);
+            bulk_g2s(smem_u32(sw + kTmaTile * kWBytes), L.m_in + d.si, 4u * n, full);
+            bulk_g2s(smem_u32(sw + kTmaTile * kWBytes + kTmaTile * 4), L.v_in + d.si, 4u * n, full);
         }
         // drain: every stage's last armed phase must have landed before exit
         for (int k = 0; k < kTmaStages && k < it; ++k) {
@@ -132,18 +139,23 @@ __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
         if (active) {
             const char* sp = stage0 + st * stage_bytes;
             const uint16_t* sg = reinterpret_cast<const uint16_t*>(sp);
-            const float* sw = reinterpret_cast<const float*>(sp + nd * kTmaTile * 2);
+            const char* sw = sp + nd * kTmaTile * 2;
+            const float* smv = reinterpret_cast<const float*>(sw + kTmaTile * kWBytes);
             float x[4];
-            unpack(*reinterpret_cast<const uint2*>(sg + q4), g);
+            unpack_as<C>(*reinterpret_cast<const uint2*>(sg + q4), g);
             for (int k = 1; k < nd; ++k) {
-                unpack(*reinterpret_cast<const uint2*>(sg + k * kTmaTile + q4), x);
+                unpack_as<C>(*reinterpret_cast<const uint2*>(sg + k * kTmaTile + q4), x);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) g[j] = __fadd_rn(g[j], x[j]);
             }
-            const float4 w4 = *reinterpret_cast<const float4*>(sw + q4);
-            const float4 m4 = *reinterpret_cast<const float4*>(sw + kTmaTile + q4);
-            const float4 v4 = *reinterpret_cast<const float4*>(sw + 2 * kTmaTile + q4);
-            w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
+            if (C::kMaster) {
+                const float4 w4 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sw) + q4);
+                w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
+            } else {
+                unpack_as<C>(*reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(sw) + q4), w);
+            }
+            const float4 m4 = *reinterpret_cast<const float4*>(smv + q4);
+            const float4 v4 = *reinterpret_cast<const float4*>(smv + kTmaTile + q4);
             m[0] = m4.x; m[1] = m4.y; m[2] = m4.z; m[3] = m4.w;
             v[0] = v4.x; v[1] = v4.y; v[2] = v4.z; v[3] = v4.w;
         }
@@ -159,11 +171,13 @@ __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
             }
             // state indices are 4-element and output indices 8-element aligned
             // with the gradient index (the host's eligibility rule)
-            __stcs(reinterpret_cast<float4*>(L.w_out + d.si + q4), make_float4(w[0], w[1], w[2], w[3]));
+            if (C::kMaster)
+                __stcs(reinterpret_cast<float4*>(L.w_out + d.si + q4), make_float4(w[0], w[1], w[2], w[3]));
             __stcs(reinterpret_cast<float4*>(L.m_out + d.si + q4), make_float4(m[0], m[1], m[2], m[3]));
             __stcs(reinterpret_cast<float4*>(L.v_out + d.si + q4), make_float4(v[0], v[1], v[2], v[3]));
-            const uint2 h = pack(w);
-            for (int k = 0; k < b.n_out; ++k) __stcs(reinterpret_cast<uint2*>(b.outs[k] + d.oi + q4), h);
+            const uint2 h = pack_as<C>(w);
+            const int n_write = b.n_out - b.keep_last;
+            for (int k = 0; k < n_write; ++k) __stcs(reinterpret_cast<uint2*>(b.outs[k] + d.oi + q4), h);
         }
     }
 
@@ -190,46 +204,58 @@ __device__ __forceinline__ void step_tma_body(const TmaArgs& a)
         sd.tail = run.tail;
         sd.decay = run.decay;
         const long long e = q < run.head ? q : run.len - run.tail + (q - run.head);
-        step_scalar<K_STEP_FUSED>(b, L, b.grads, b.outs, sd, e, bad);
+        step_scalar<K_STEP_FUSED, C>(b, L, b.grads, b.outs, sd, e, bad);
     }
 
     // one atomic per consumer warp that saw a non-finite unscaled gradient
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicMax(b.flag, b.call_id);
 }
 
-template <int WARPS, int STAGES, bool ASYNC>
+template <int WARPS, int STAGES, bool ASYNC, class C>
 __global__ void __launch_bounds__((WARPS + 1) * 32, 1) step_tma_kernel(const TmaArgs a)
 {
     if (!ASYNC)
-        step_tma_body<WARPS, STAGES, false, 0>(a);
+        step_tma_body<WARPS, STAGES, false, 0, C>(a);
     else if (a.b.ctrl->cur == 0)
-        step_tma_body<WARPS, STAGES, true, 0>(a);
+        step_tma_body<WARPS, STAGES, true, 0, C>(a);
     else
-        step_tma_body<WARPS, STAGES, true, 1>(a);
+        step_tma_body<WARPS, STAGES, true, 1, C>(a);
 }
 
-int smem_bytes(TmaShape sh, int nd) { return kHdrBytes + sh.stages * (nd * sh.tile * 2 + 3 * sh.tile * 4); }
+int smem_bytes(TmaShape sh, int nd, bool bf16)
+{
+    return kHdrBytes + sh.stages * (nd * sh.tile * 2 + sh.tile * ((bf16 ? 2 : 4) + 8));
+}
 
-template <bool ASYNC>
+template <bool ASYNC, class C>
 const void* kernel_for(TmaShape sh)
 {
     if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages)
-        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaWide.warps, kTmaWide.stages, ASYNC>);
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaWide.warps, kTmaWide.stages, ASYNC, C>);
     if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages)
-        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, ASYNC>);
+        return reinterpret_cast<const void*>(&step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, ASYNC, C>);
     return nullptr;
+}
+
+template <int WARPS, int STAGES, class C>
+void launch_shape(const TmaArgs& a, int grid, int threads, int smem, cudaStream_t s)
+{
+    if (a.b.ctrl != nullptr)
+        step_tma_kernel<WARPS, STAGES, true, C><<<grid, threads, smem, s>>>(a);
+    else
+        step_tma_kernel<WARPS, STAGES, false, C><<<grid, threads, smem, s>>>(a);
 }
 
 }  // namespace
 
 // Both the synchronous and the asynchronous kernel of the shape get the
 // shared-memory attribute; the reported occupancy is the smaller of the two.
-cudaError_t tma_prepare(TmaShape sh, int nd, int* blocks_per_sm)
+cudaError_t tma_prepare(TmaShape sh, int nd, bool bf16, int* blocks_per_sm)
 {
-    const void* f = kernel_for<false>(sh);
-    const void* fa = kernel_for<true>(sh);
+    const void* f = bf16 ? kernel_for<false, BF16>(sh) : kernel_for<false, F16>(sh);
+    const void* fa = bf16 ? kernel_for<true, BF16>(sh) : kernel_for<true, F16>(sh);
     if (!f || !fa) return cudaErrorInvalidValue;
-    const int smem = smem_bytes(sh, nd);
+    const int smem = smem_bytes(sh, nd, bf16);
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fa, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     int occ = 0, occ_a = 0;
@@ -239,21 +265,16 @@ cudaError_t tma_prepare(TmaShape sh, int nd, int* blocks_per_sm)
     return e;
 }
 
-cudaError_t launch_step_tma(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s)
+cudaError_t launch_step_tma(TmaShape sh, const TmaArgs& a, int grid, cudaStream_t s, bool bf16)
 {
-    const int smem = smem_bytes(sh, a.b.nd);
+    const int smem = smem_bytes(sh, a.b.nd, bf16);
     const int threads = (sh.warps + 1) * 32;
-    const bool as = a.b.ctrl != nullptr;
     if (sh.warps == kTmaWide.warps && sh.stages == kTmaWide.stages) {
-        if (as)
-            step_tma_kernel<kTmaWide.warps, kTmaWide.stages, true><<<grid, threads, smem, s>>>(a);
-        else
-            step_tma_kernel<kTmaWide.warps, kTmaWide.stages, false><<<grid, threads, smem, s>>>(a);
+        if (bf16) launch_shape<kTmaWide.warps, kTmaWide.stages, BF16>(a, grid, threads, smem, s);
+        else launch_shape<kTmaWide.warps, kTmaWide.stages, F16>(a, grid, threads, smem, s);
     } else if (sh.warps == kTmaDeep.warps && sh.stages == kTmaDeep.stages) {
-        if (as)
-            step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, true><<<grid, threads, smem, s>>>(a);
-        else
-            step_tma_kernel<kTmaDeep.warps, kTmaDeep.stages, false><<<grid, threads, smem, s>>>(a);
+        if (bf16) launch_shape<kTmaDeep.warps, kTmaDeep.stages, BF16>(a, grid, threads, smem, s);
+        else launch_shape<kTmaDeep.warps, kTmaDeep.stages, F16>(a, grid, threads, smem, s);
     } else {
         return cudaErrorInvalidValue;
     }

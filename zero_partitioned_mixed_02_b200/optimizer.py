@@ -38,9 +38,11 @@ class ZeroAdam:
                  stream: torch.cuda.Stream | None = None,
                  precision: int = A.ZERO_PRECISION_FP16):
         """precision = ZERO_PRECISION_BF16: bfloat16 gradients and parameters
-        without fp32 master weights; only the two-pass variants exist for it,
-        so a fused variant is replaced by ZERO_VARIANT_TWO_PASS_TMA."""
-        if precision == A.ZERO_PRECISION_BF16 and variant in (A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_FUSED_TMA):
+        without fp32 master weights. The fused variants then roll back from the
+        last replica, so they exist for stage 1/2 with all Nd >= 2 ranks; for
+        anything else a fused variant is replaced by ZERO_VARIANT_TWO_PASS_TMA."""
+        if (precision == A.ZERO_PRECISION_BF16 and variant in (A.ZERO_VARIANT_FUSED, A.ZERO_VARIANT_FUSED_TMA)
+                and not (stage <= 2 and rank_view < 0 and nd >= 2)):
             variant = A.ZERO_VARIANT_TWO_PASS_TMA
         self.cfg = A.Config(psi, nd, stage, rank_view=rank_view, variant=variant, tensors=tensors,
                             precision=precision)
