@@ -179,6 +179,9 @@ KERNEL_FILES = {
     "two-pass-bf16": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
     "two-pass-tma": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma_pass.cu"),
     "two-pass-tma-bf16": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma_pass.cu"),
+    # the fused bfloat16 step and its replica pass (zero_kernels.cu)
+    "fused-tma-bf16": ("zero_device.cuh", "zero_internal.h", "zero_tma.cuh", "zero_tma.cu", "zero_kernels.cu"),
+    "fused-bf16": ("zero_device.cuh", "zero_internal.h", "zero_kernels.cu"),
 }
 
 
@@ -194,6 +197,8 @@ def kernel_sha(variant):
 def recorded_traffic(wl_name, variant):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source."""
+    if variant not in KERNEL_FILES:
+        return None
     path = os.path.join(ROOT, "profiles", f"ncu_step_{wl_name}_{variant}.md")
     try:
         txt = open(path).read()
