@@ -846,7 +846,7 @@ def zero_job_bytes(psi: int, world: int, stage: int, n_units_elems: int = 0) -> 
 
 
 def run_zero_job(args):
-    """The real Nd = N job (SURVEY's multi-GPU design): one process per GPU,
+    """The real Nd = N job (the method across GPUs): one process per GPU,
     rank r owns partition r (stage 1/2) or chunk r of every tensor (stage 3)
     of the workload's parameter list; its step pulls the other ranks'
     gradients of that partition through peer mappings, sums them in rank order
