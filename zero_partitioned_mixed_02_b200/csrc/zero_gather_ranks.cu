@@ -53,8 +53,9 @@ __device__ __forceinline__ int find_run(const Run* runs, int n_runs, int64_t til
 // of kThreads per SM with kUnroll 16-byte loads in flight per thread (64 KB
 // per SM) measured fastest on the Llama layer walk: more bytes in flight per
 // SM (more blocks, or 8 loads per thread), contiguous spans of tiles per block,
-// 512-thread blocks, streaming cache hints and the read-only load path were
-// all slower; 128-thread blocks (8 per SM) were the same within noise.
+// 512-thread blocks, streaming cache hints (on loads, on stores, or both) and
+// the read-only load path were all slower; 128-thread blocks (8 per SM) were
+// the same within noise.
 __global__ void __launch_bounds__(kThreads, kMinBlocks) layer_gather_kernel(const Args a)
 {
     // a programmatic dependent launch: wait for the previous kernel on the stream
