@@ -145,3 +145,23 @@ def test_real_job_is_the_default_for_several_gpus(monkeypatch):
     monkeypatch.setattr("sys.argv", ["bench.py"])
     bench.main()
     assert calls[-1] == "replicas"
+
+
+def test_algorithmic_bytes_per_variant():
+    """The floor and per-launch bytes bench.py divides by: 56 B/element for
+    GPT-2's stage-2 step at Nd = 8 (fp16 with master), 50 without a master;
+    the fused bfloat16 step kernel moves the floor less the replica it does
+    not write, and its replica pass 4 B/element; the two passes 64."""
+    wl = bench.workload("gpt2-1.5b")
+    n, floor, per, gathers = bench.algorithmic_bytes(wl, "fused-tma")
+    assert n == wl.psi and floor == 56 * n and per == {"step_kernel<fused>": 56 * n} and gathers == 0
+    n, floor, per, _ = bench.algorithmic_bytes(wl, "fused-tma", bf16=True)
+    assert floor == 50 * n and per == {"step_kernel<fused,bf16>": 48 * n, "replica_kernel": 4 * n}
+    _, floor, per, _ = bench.algorithmic_bytes(wl, "two-pass-tma")
+    assert floor == 56 * n and sum(per.values()) == 64 * n
+    assert bench.bf16_fused_eligible(wl)
+    assert not bench.bf16_fused_eligible(bench.workload("llama-2.7b"))
+    assert not bench.bf16_fused_eligible(bench.workload("7.5b-rank-view"))
+    ll = bench.workload("llama-2.7b")
+    n, floor, _, gathers = bench.algorithmic_bytes(ll, "fused-tma")
+    assert floor == 42 * n and gathers == 8 * ll.psi
